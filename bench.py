@@ -1,0 +1,446 @@
+#!/usr/bin/env python
+"""Benchmark of the spatiotemporal attention hot path on B200.
+
+Default workload (one GPU): Wan2.1-1.3B-like full bidirectional attention
+with fused 3D-RoPE, B=1, 12 heads, head dim 128, latent grid 21x30x52
+(32760 tokens), bf16 N(0,1) synthetic inputs.  One step = one
+vattn_attention call (RoPE fused) on inputs resident in HBM; L2 is flushed
+(256 MiB write) before every timed step.  Throughput is mask-adjusted
+TFLOP/s: 4 * d FLOPs per visible (query, key) pair per head.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Multi-GPU (torchrun): every rank runs its own replica of the workload (the
+path shards over independent problems; no data-path collective); the time is
+the max over ranks and `value` counts the work of all ranks (weak scaling).
+--impl reference times the fp64 CPU oracle on a bounded sample of the same
+workload on the host cores (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import seeded_inputs as si  # noqa: E402
+
+METRIC = "attention TFLOPS (mask-adjusted) & % of B200 BF16 peak; streaming frames/s"
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+KERNEL_SOURCES = ["video_diffusion_transformer_02_b200/csrc/attention.cuh",
+                  "video_diffusion_transformer_02_b200/csrc/sm100.cuh"]
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return PEAKS_FALLBACK, "fallback"
+
+
+def kernel_hash() -> str:
+    h = hashlib.sha256()
+    for rel in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic():
+    """DRAM bytes per launch of the attention kernel from the committed ncu
+    summary, if it was taken on the current kernel source (else None)."""
+    p = os.path.join(ROOT, "profiles", "attn_fwd_traffic.txt")
+    if not os.path.exists(p):
+        return None
+    vals = {}
+    with open(p) as f:
+        for line in f:
+            if "=" in line and not line.startswith("#"):
+                k, v = line.split("=", 1)
+                vals[k.strip()] = v.strip()
+    if vals.get("kernel_hash") != kernel_hash():
+        return None
+    try:
+        return float(vals["bytes_per_launch_wan13b"])
+    except (KeyError, ValueError):
+        return None
+
+
+# ----------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi samples (SM clock, throttle reasons) during the timed region."""
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+    NAMES = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.dev = device_index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.dev), "--query-gpu=" + self.FIELDS,
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if not self.proc:
+            return None
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.thread.join(timeout=2)
+        sm, mx, reasons = [], [], set()
+        for ln in self.lines:
+            parts = [x.strip() for x in ln.split(",")]
+            if len(parts) < 7:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx.append(float(parts[1]))
+            except ValueError:
+                continue
+            for name, val in zip(self.NAMES, parts[3:7]):
+                if val.lower().startswith("active"):
+                    reasons.add(name)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "samples": len(sm),
+                "reasons": sorted(reasons)}
+
+
+# -------------------------------------------------------------- workloads
+def wan13b_workload(va, torch, device):
+    c = si.CONFIGS["wan13b"]
+    B, H, d, T, Hg, Wg = c["B"], c["H"], c["d"], c["T"], c["Hg"], c["Wg"]
+    L = T * Hg * Wg
+    q, k, v = si.qkv("wan13b")
+    dev = lambda x: torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).to(device)
+    rope = va.Rope(Hg=Hg, Wg=Wg, pairs=c["pairs"], max_pos=max(T, Hg, Wg), theta=c["theta"])
+    tab = va.rope_table(rope, d, device=device)
+    w = dict(name="wan13b", B=B, H=H, d=d, L=L, T=T, Hg=Hg, Wg=Wg, rope=rope, tab=tab,
+             q_host=q, k_host=k, v_host=v, q=dev(q), k=dev(k), v=dev(v),
+             o=torch.empty((B, L, H, d), dtype=torch.bfloat16, device=device),
+             flops=4.0 * d * L * L * H * B, scale=d ** -0.5, pairs=c["pairs"], theta=c["theta"])
+    return w
+
+
+def run_ours(args, rank, world, device):
+    import torch
+    import video_diffusion_transformer_02_b200 as va
+
+    torch.cuda.set_device(device)
+    dev_index = torch.cuda.current_device()
+    w = wan13b_workload(va, torch, device)
+    flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=device)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        va.vattn_attention(w["q"], w["k"], w["v"], w["o"], scale=w["scale"], rope=w["rope"],
+                           table=w["tab"])
+
+    for _ in range(args.warmup):
+        step()
+    va.vattn_check()
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    sampler = ClockSampler(dev_index)
+    sampler.start()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps)]
+    torch.cuda.synchronize()
+    for i in range(args.steps):
+        flush.zero_()
+        evs[i][0].record(stream)
+        step()
+        evs[i][1].record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    clocks = sampler.stop()
+    va.vattn_check()
+    step_ms = [a.elapsed_time(b) for a, b in evs]
+    total_ms = float(sum(step_ms))
+    if world > 1:
+        t = torch.tensor([total_ms], dtype=torch.float64, device=device)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        total_ms = float(t.item())
+    ms_per_step = total_ms / args.steps
+    value = world * w["flops"] * args.steps / (total_ms / 1e3) / 1e12
+    kernel_ms = statistics.mean(step_ms)      # one attention launch per step
+    achieved = w["flops"] / (kernel_ms / 1e3) / 1e12
+
+    # end to end through the C ABI with host buffers: H2D of q, k, v from
+    # pinned memory, the call, D2H of o, all inside the timed region
+    qh = torch.from_numpy(w["q_host"].view(np.int16)).view(torch.bfloat16).pin_memory()
+    kh = torch.from_numpy(w["k_host"].view(np.int16)).view(torch.bfloat16).pin_memory()
+    vh = torch.from_numpy(w["v_host"].view(np.int16)).view(torch.bfloat16).pin_memory()
+    oh = torch.empty(w["o"].shape, dtype=torch.bfloat16).pin_memory()
+
+    def e2e_step():
+        w["q"].copy_(qh, non_blocking=True)
+        w["k"].copy_(kh, non_blocking=True)
+        w["v"].copy_(vh, non_blocking=True)
+        step()
+        oh.copy_(w["o"], non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize()
+    e_steps = max(1, min(args.steps, 5))
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1) / e_steps
+    if world > 1:
+        t = torch.tensor([e2e_ms], dtype=torch.float64, device=device)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    h2d = 3 * w["q"].numel() * 2
+    d2h = w["o"].numel() * 2
+
+    secondary = None
+    if not args.no_secondary and rank == 0:
+        secondary = secondary_measurements(va, torch, device, flush)
+
+    pk, src = peaks()
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(w, rows=args.cpu_rows)
+    return dict(
+        metric=METRIC, value=value, unit="TFLOP/s", n_gpus=world, steps=args.steps,
+        warmup=args.warmup, ms_per_step=ms_per_step, higher_is_better=True, scaling="weak",
+        vs_baseline=None, dtype="bf16", data="synthetic",
+        config={"workload": "wan13b full bidirectional attention + fused 3D-RoPE "
+                            "(B=1, H=12, d=128, grid 21x30x52 = 32760 tokens, pairs t22/h21/w21, "
+                            "theta 1e4)",
+                "mask_adjusted_flops_per_step": w["flops"],
+                "l2": "flushed before every timed step (256 MiB write); inputs 300 MB > L2",
+                "parallelism": "replicas x%d" % world},
+        roofline={"bound": "tensor", "achieved": achieved, "peak": pk["bf16_tflops"],
+                  "unit": "TFLOP/s", "frac": achieved / pk["bf16_tflops"],
+                  "frac_of_sustained": achieved / pk.get("bf16_tflops_sustained", pk["bf16_tflops"]),
+                  "peak_source": src + " (burst bf16 GEMM)", "kernel": "attn_fwd_kernel<128,rope>",
+                  "traffic": recorded_traffic()},
+        cpu_baseline=cpu,
+        e2e={"value": w["flops"] / (e2e_ms / 1e3) / 1e12 * world, "unit": "TFLOP/s",
+             "ms_per_step": e2e_ms, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        clocks=clocks, gpu_launches=args.steps, secondary=secondary)
+
+
+def _time_events(torch, fn, n, flush=None):
+    s = torch.cuda.current_stream()
+    tot = 0.0
+    for _ in range(n):
+        if flush is not None:
+            flush.zero_()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(s)
+        fn()
+        b.record(s)
+        torch.cuda.synchronize()
+        tot += a.elapsed_time(b)
+    return tot / n
+
+
+def secondary_measurements(va, torch, device, flush):
+    """The other configurations, briefly: 14B full / chunk-causal TFLOPS,
+    streaming frames/s and append GB/s, hybrid time and scan bandwidth."""
+    out = {}
+    dev = lambda x: torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).to(device)
+    pk, _ = peaks()
+    # Wan2.1-14B-like 720p
+    c = si.CONFIGS["wan14b"]
+    L, H, d = c["T"] * c["Hg"] * c["Wg"], c["H"], c["d"]
+    q, k, v = si.qkv("wan14b")
+    qd, kd, vd = dev(q), dev(k), dev(v)
+    del q, k, v
+    o = torch.empty_like(qd)
+    rope = va.Rope(Hg=c["Hg"], Wg=c["Wg"], pairs=c["pairs"], max_pos=max(c["T"], c["Hg"], c["Wg"]))
+    tab = va.rope_table(rope, d, device=device)
+    F = c["Hg"] * c["Wg"]
+    for name, mode, frac in (("wan14b_full", "full", 1.0), ("wan14b_chunk", "chunk_causal", 28 / 49)):
+        fn = lambda: va.vattn_attention(qd, kd, vd, o, scale=d ** -0.5, mode=mode, tokens_per_frame=F,
+                                        chunk_frames=c["chunk_frames"], rope=rope, table=tab)
+        fn()
+        ms = _time_events(torch, fn, 3)
+        flops = 4.0 * d * L * L * H * frac
+        out[name] = {"ms": ms, "tflops": flops / ms * 1e-9, "frac_of_peak": flops / ms * 1e-9 / pk["bf16_tflops"]}
+    del qd, kd, vd, o
+    # streaming decode: 32 frames, ring of 4, window 4
+    c = si.CONFIGS["stream"]
+    F, H, d, T = c["Hg"] * c["Wg"], c["H"], c["d"], c["T"]
+    q, k, v = si.qkv("stream")
+    qd, kd, vd = dev(q).view(T, F, H, d), dev(k).view(T, F, H, d), dev(v).view(T, F, H, d)
+    cap = c["capacity"]
+    kr = torch.zeros((cap, 1, F, H, d), dtype=torch.bfloat16, device=device)
+    vr = torch.zeros_like(kr)
+    ids = torch.zeros(cap, dtype=torch.int32, device=device)
+    cache = va.KVCache(kr, vr, ids)
+    rope = va.Rope(Hg=c["Hg"], Wg=c["Wg"], pairs=c["pairs"], max_pos=64)
+    tab = va.rope_table(rope, d, device=device)
+    of = torch.empty((1, F, H, d), dtype=torch.bfloat16, device=device)
+    frames = [(qd[f].unsqueeze(0), kd[f].unsqueeze(0), vd[f].unsqueeze(0)) for f in range(T)]
+
+    def stream_all():
+        for f in range(T):
+            qf, kf, vf = frames[f]
+            cache.attend(qf, kf, vf, of, f, c["window_back"], rope=rope, table=tab)
+            cache.append(kf, vf, f)
+
+    stream_all()
+    ms = _time_events(torch, stream_all, 3)
+    total_flops = 4.0 * d * F * F * H * sum(min(f, c["window_back"]) + 1 for f in range(T))
+    steady = lambda: cache.attend(frames[10][0], frames[10][1], frames[10][2], of, T - 1,
+                                  c["window_back"], rope=rope, table=tab)
+    steady()
+    ms_att = _time_events(torch, steady, 10)
+    app = lambda: cache.append(frames[5][1], frames[5][2], 5)
+    app()
+    ms_app = _time_events(torch, lambda: [app() for _ in range(16)], 3) / 16
+    app_bytes = 2 * 2 * F * H * d * 2
+    out["stream"] = {"frames_per_s": T / (ms / 1e3), "ms_per_frame": ms / T, "tflops": total_flops / ms * 1e-9,
+                     "steady_attention_ms": ms_att,
+                     "steady_attention_tflops": 4.0 * d * F * F * H * 5 / ms_att * 1e-9,
+                     "append_us": ms_app * 1e3, "append_gbs": app_bytes / (ms_app / 1e3) / 1e9,
+                     "append_frac_of_hbm": app_bytes / (ms_app / 1e3) / 1e9 / pk["hbm_gbs"]}
+    cache.close()
+    del qd, kd, vd, kr, vr
+    # hybrid chunk attention
+    c = si.CONFIGS["hybrid"]
+    L, H, d = c["T"] * c["Hg"] * c["Wg"], c["H"], c["d"]
+    ct = c["chunk_frames"] * c["Hg"] * c["Wg"]
+    q, k, v = si.qkv("hybrid")
+    qd, kd, vd = dev(q), dev(k), dev(v)
+    o = torch.empty_like(qd)
+    S = torch.zeros((1, H, d, d), dtype=torch.float32, device=device)
+    z = torch.zeros((1, H, d), dtype=torch.float32, device=device)
+    ws = torch.empty(va.vattn_hybrid_workspace_bytes(1, L, H, d, ct), dtype=torch.uint8, device=device)
+    fn = lambda: va.vattn_hybrid_chunk(qd, kd, vd, o, S, z, ct, workspace=ws)
+    fn()
+    ms = _time_events(torch, fn, 5)
+    n_ch = (L + ct - 1) // ct
+    intra = sum(min(ct, L - i * ct) ** 2 for i in range(n_ch))
+    flops = 4.0 * d * intra * H + (4.0 * d * d + 4.0 * d) * L * H * 2
+    out["hybrid"] = {"ms": ms, "tflops": flops / ms * 1e-9}
+    va.vattn_check()
+    return out
+
+
+def cpu_baseline(w, rows=2048):
+    """The fp64 oracle, as it stands, on a bounded sample of the workload."""
+    import oracle
+    rows_arr = si.sample_rows(0xBA5E, rows, w["B"], 2, w["L"])
+    t0 = time.perf_counter()
+    oracle.attention(w["q_host"], w["k_host"], w["v_host"], w["scale"],
+                     rope=dict(Hg=w["Hg"], Wg=w["Wg"], pairs=w["pairs"], theta=w["theta"]), rows=rows_arr)
+    dt = time.perf_counter() - t0
+    flops = 4.0 * w["d"] * w["L"] * len(rows_arr)
+    return {"value": flops / dt / 1e12, "unit": "TFLOP/s", "cores": oracle.num_threads(), "kind": "oracle",
+            "seconds": dt,
+            "sample": "%d query rows (2 of 12 heads) of the wan13b workload, all 32760 keys each, "
+                      "fp64 with 3D-RoPE; TFLOP/s of mask-adjusted work" % len(rows_arr)}
+
+
+def run_reference(args, rank, world):
+    """The oracle timed on the host as the reference arm (rank 0 only)."""
+    if rank != 0:
+        return None
+    import oracle
+    c = si.CONFIGS["wan13b"]
+    q, k, v = si.qkv("wan13b")
+    L, d = c["T"] * c["Hg"] * c["Wg"], c["d"]
+    rope = dict(Hg=c["Hg"], Wg=c["Wg"], pairs=c["pairs"], theta=c["theta"])
+    n = args.ref_rows
+
+    def one(i):
+        rows = si.sample_rows(0xBA5E + i, n, 1, 2, L)
+        oracle.attention(q, k, v, d ** -0.5, rope=rope, rows=rows)
+        return len(rows)
+
+    for i in range(args.warmup):
+        one(i)
+    t0 = time.perf_counter()
+    total_rows = 0
+    for i in range(args.steps):
+        total_rows += one(100 + i)
+    dt = time.perf_counter() - t0
+    flops = 4.0 * d * L * total_rows
+    val = flops / dt / 1e12
+    sample = "%d query rows per step (2 of 12 heads) of the wan13b workload, all 32760 keys, fp64" % n
+    return dict(metric=METRIC, value=val, unit="TFLOP/s", n_gpus=world, steps=args.steps,
+                warmup=args.warmup, ms_per_step=dt / args.steps * 1e3, higher_is_better=True,
+                scaling="weak", vs_baseline=None, dtype="f64", data="synthetic", impl="reference",
+                config={"workload": "wan13b full bidirectional attention + 3D-RoPE (B=1, H=12, d=128, "
+                                    "32760 tokens); bounded row sample per step"},
+                cpu_baseline={"value": val, "unit": "TFLOP/s", "cores": oracle.num_threads(),
+                              "kind": "oracle", "sample": sample},
+                e2e={"value": val, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0})
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--no-secondary", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-rows", type=int, default=2048)
+    ap.add_argument("--ref-rows", type=int, default=512)
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3) if args.impl == "ours" else args.warmup
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        res = run_reference(args, rank, world)
+        if res is not None:
+            print(json.dumps(res), flush=True)
+        return
+    import torch
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                             device_id=torch.device("cuda", local))
+    res = run_ours(args, rank, world, torch.device("cuda", local))
+    if rank == 0:
+        print(json.dumps(res), flush=True)
+    if world > 1:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

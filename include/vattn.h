@@ -1,0 +1,201 @@
+/*
+ * vattn — spatiotemporal attention for video diffusion transformers and
+ * streaming transformer decoders, as hand-written sm_100a (B200) kernels.
+ *
+ * C ABI.  Every pointer argument named q/k/v/o/ring/state/table/workspace is
+ * DEVICE memory owned by the caller (allocate it with any allocator, e.g.
+ * PyTorch); the library never frees caller memory.  Other pointers are host
+ * memory and are read during the call only.
+ *
+ * Common conventions
+ *  - Tensors q, k, v, o are bfloat16, contiguous, layout [B][L][H][d]
+ *    (token-major, heads, then head channels): the layout a DiT QKV
+ *    projection emits.  Base pointers must be 16-byte aligned.
+ *  - Token n of a latent video of T x Hg x Wg tokens sits at
+ *    (t, h, w) = (n / (Hg*Wg), (n / Wg) % Hg, n % Wg): row-major over the
+ *    latent order B x C' x T' x H' x W' of FlashDecoder ("Preliminaries:
+ *    Latent Diffusion Model", Sec. 3.1).  A "frame" is Hg*Wg consecutive
+ *    tokens.
+ *  - Every call is asynchronous on `stream` (a cudaStream_t; NULL = legacy
+ *    default stream), allocates nothing, never synchronises, and may be
+ *    captured in a CUDA graph.  Arguments are checked before any launch;
+ *    on an error nothing is launched and no output is touched.
+ *  - Kernels bound every internal wait.  A wait that gives up records a
+ *    code in a device status word; vattn_check() reports it as
+ *    VATTN_ERR_TIMEOUT.
+ *  - d (head dim) must be 64 or 128; H must be a multiple of Hkv.
+ */
+#ifndef VATTN_H_
+#define VATTN_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t. */
+typedef struct CUstream_st* vattn_stream;
+
+typedef enum {
+  VATTN_OK = 0,
+  VATTN_ERR_INVALID_ARG = 1, /* a pointer, size or option is invalid          */
+  VATTN_ERR_UNSUPPORTED = 2, /* valid, but not a shape this build supports    */
+  VATTN_ERR_CUDA = 3,        /* a CUDA runtime/driver call failed             */
+  VATTN_ERR_TIMEOUT = 4      /* a kernel gave up on a bounded internal wait   */
+} vattn_status;
+
+typedef enum {
+  /* every query sees every key (Wan-style DiT self-attention) */
+  VATTN_FULL = 0,
+  /* key frame fk visible from query frame fq iff floor(fk/c) <= floor(fq/c):
+     bidirectional inside a chunk of c frames, causal across chunks
+     (FlashDecoder, "Effectiveness of Each Component", Sec. 4.2, the
+     "full block causal attention" baseline; MobileWan chunk-wise
+     autoregression) */
+  VATTN_CHUNK_CAUSAL = 1,
+  /* visible iff fq - window_back <= fk <= fq + window_fwd: the per-frame
+     sliding window of FlashDecoder "Streaming with Rolling KV Cache"
+     (Sec. 3.3) — all tokens of the query's own frame and of the window
+     frames, no mask inside a frame */
+  VATTN_SLIDING = 2
+} vattn_mode;
+
+/*
+ * 3D rotary position embedding (FlashDecoder "Transformer Backbone Design",
+ * Sec. 3.2: RoPE applied separately to the temporal and spatial axes; the
+ * channel groups t / x / y of the Kaleido review; frequencies as in
+ * RoFormer).  Channel pair j = (2j, 2j+1) of a head turns by angle
+ * pos * theta^(-i / n_axis), where pairs [0, pairs_t) use pos = t (i = j),
+ * the next pairs_h use pos = h and the last pairs_w use pos = w
+ * (i = index inside the group).  pairs_t + pairs_h + pairs_w = d / 2.
+ */
+typedef struct {
+  int Hg, Wg;                     /* spatial token grid of one frame        */
+  int pairs_t, pairs_h, pairs_w;  /* channel pairs per axis                 */
+  int max_pos;                    /* table rows; every t, h, w < max_pos    */
+  double theta;                   /* base, e.g. 10000                       */
+} vattn_rope;
+
+/* Bytes of the cos/sin table for (rope, d): max_pos * (d/2) * 8.
+   0 if the configuration is invalid. */
+size_t vattn_rope_table_bytes(const vattn_rope* rope, int d);
+
+/* Fill the caller's device table (float2 [max_pos][d/2] of (cos, sin),
+   angles evaluated in double, rounded to fp32).  Build it once per
+   configuration ("precomputed RoPE tables", FlashDecoder "Inference
+   Optimization", Sec. 4.6). */
+vattn_status vattn_rope_table_build(const vattn_rope* rope, int d, float* table,
+                                    vattn_stream stream);
+
+/*
+ * Standalone 3D-RoPE of q [B][L][H][d] and k [B][L][Hkv][d] into q_out /
+ * k_out (same layouts; out-of-place; q_out may not alias k).  Token n is at
+ * frame t = frame_offset + n / (Hg*Wg).  fp32 rotation, bf16 round-to-
+ * nearest-even results.  Either (q, q_out) or (k, k_out) may be NULL.
+ */
+vattn_status vattn_rope_qk(const void* q, const void* k, void* q_out, void* k_out, int B, int L,
+                           int H, int Hkv, int d, const vattn_rope* rope, const float* table,
+                           int frame_offset, vattn_stream stream);
+
+/*
+ * Masked softmax attention with optional fused 3D-RoPE.
+ *   q [B][Lq][H][d], k/v [B][Lk][Hkv][d], o [B][Lq][H][d] (bf16).
+ *   lse (nullable) fp32 [B][H][Lq]: natural log of each row's softmax
+ *   denominator of scale*q.k (for combining partial attentions).
+ *   Query token n is in frame q_frame_offset + n / tokens_per_frame, key
+ *   token n in frame k_frame_offset + n / tokens_per_frame.  The mode picks
+ *   the visible keys (see vattn_mode); tokens_per_frame is ignored by FULL
+ *   unless rope is given.
+ *   rope/table (both nullable): when given, q and k are rotated at their own
+ *   (t, h, w) inside the kernel, on the shared-memory tiles, before the
+ *   products; then tokens_per_frame must equal rope->Hg * rope->Wg.
+ * o = softmax(scale * q k^T restricted to visible keys) v, computed with an
+ * online softmax (fp32 statistics, fp32 accumulation, bf16 P and output).
+ * Tiles with no visible key are never loaded.
+ */
+vattn_status vattn_attention(const void* q, const void* k, const void* v, void* o, float* lse,
+                             int B, int Lq, int Lk, int H, int Hkv, int d, float scale,
+                             vattn_mode mode, int tokens_per_frame, int chunk_frames,
+                             int window_back, int window_fwd, int q_frame_offset,
+                             int k_frame_offset, const vattn_rope* rope, const float* table,
+                             vattn_stream stream);
+
+/*
+ * Rolling KV cache of a fixed number of frames (FlashDecoder "Streaming with
+ * Rolling KV Cache", Sec. 3.3; constant memory regardless of video length,
+ * "Long Video Decoding", Sec. 4.3).  Storage is caller-owned device memory:
+ *   k_ring, v_ring: bf16 [capacity][B][F][Hkv][d]   (raw, un-rotated K/V)
+ *   frame_ids: int32 [capacity]  (frame held by each slot, -1 = empty)
+ * Frame f lives in slot f mod capacity.  The handle is host metadata (with a
+ * host mirror of frame_ids); it does not own the storage.
+ */
+typedef struct vattn_kvcache vattn_kvcache;
+
+/* Create a handle; sets every frame_ids entry to -1 on `stream`. */
+vattn_status vattn_kvcache_init(vattn_kvcache** cache, void* k_ring, void* v_ring,
+                                int32_t* frame_ids, int capacity, int B, int F, int Hkv, int d,
+                                vattn_stream stream);
+/* Copy frame f's K and V (bf16 [B][F][Hkv][d] each) into slot f mod
+   capacity and set frame_ids[slot] = f: a bit-exact 16-byte vector copy. */
+vattn_status vattn_kvcache_append(vattn_kvcache* cache, const void* k, const void* v,
+                                  int frame_idx, vattn_stream stream);
+/*
+ * One streaming step: the F query tokens of frame `frame_idx` (q bf16
+ * [B][F][H][d]) attend to every token of the current frame (k_cur, v_cur,
+ * [B][F][Hkv][d]) and of the cached frames frame_idx-window_back ..
+ * frame_idx-1 that are present in the ring (frames before 0 do not exist).
+ * No mask inside a frame; causality comes from the processing order.  Keys
+ * are rotated at their own absolute frame index, queries at frame_idx.
+ * window_back <= capacity.  o bf16 [B][F][H][d]; lse nullable fp32
+ * [B][H][F].  Call vattn_kvcache_append for the current frame afterwards.
+ */
+vattn_status vattn_attention_stream(vattn_kvcache* cache, const void* q, const void* k_cur,
+                                    const void* v_cur, void* o, float* lse, int H, int frame_idx,
+                                    int window_back, float scale, const vattn_rope* rope,
+                                    const float* table, vattn_stream stream);
+/* Copy the host mirror of frame_ids (capacity entries) into host_ids. */
+vattn_status vattn_kvcache_frame_ids(const vattn_kvcache* cache, int32_t* host_ids);
+/* After the caller restored ring and frame_ids contents (checkpoint /
+   resume), set the host mirror to host_ids (capacity entries). */
+vattn_status vattn_kvcache_restore(vattn_kvcache* cache, const int32_t* host_ids);
+vattn_status vattn_kvcache_destroy(vattn_kvcache* cache);
+
+/*
+ * Hybrid chunk attention (MobileWan recurrence distillation: softmax
+ * attention inside a chunk, causal linear attention across chunks through a
+ * running state (s, z), feature map phi(x) = elu(x) + 1 as in Katharopoulos
+ * et al.).  Tokens are cut into chunks of chunk_tokens (the last may be
+ * shorter).  For query i of chunk c, with s_ij = scale * q_i . k_j:
+ *   o_i = ( sum_{j in c} e^{s_ij} v_j + phi(q_i)^T S_c )
+ *         / ( sum_{j in c} e^{s_ij}     + phi(q_i)^T z_c )
+ * where S_c = S_in + sum_{j in chunks < c} phi(k_j) v_j^T and
+ * z_c = z_in + sum phi(k_j) (phi on raw q, k; no RoPE).
+ *   q/k/v/o bf16 [B][L][H][d]; S fp32 [B][H][d][d] (S[a][e]: key feature a,
+ *   value channel e) and z fp32 [B][H][d] are IN/OUT: they enter as the
+ *   state before token 0 and leave as the state after token L-1, so a
+ *   stream of calls is the model run as an RNN.
+ *   workspace: device scratch of at least vattn_hybrid_workspace_bytes().
+ * Three launches: per-chunk state deltas (tcgen05 MMA), an exclusive scan
+ * over chunks, then the attention with each query tile's online-softmax
+ * state initialised from its linear part (tcgen05 MMA).
+ */
+size_t vattn_hybrid_workspace_bytes(int B, int L, int H, int d, int chunk_tokens);
+vattn_status vattn_hybrid_chunk(const void* q, const void* k, const void* v, void* o, float* S,
+                                float* z, int B, int L, int H, int d, int chunk_tokens,
+                                float scale, void* workspace, size_t workspace_bytes,
+                                vattn_stream stream);
+
+/* Synchronise `stream`, then read and clear the device status word:
+   VATTN_ERR_TIMEOUT if a kernel gave up on a wait since the last check. */
+vattn_status vattn_check(vattn_stream stream);
+
+const char* vattn_status_string(vattn_status status);
+/* Human-readable detail of the last error on the calling thread. */
+const char* vattn_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* VATTN_H_ */

@@ -8,6 +8,25 @@ if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
 
+def load_build_module():
+    """The package's build helper, loaded by path (importing the package
+    itself requires the built library)."""
+    import importlib.util
+    path = os.path.join(ROOT, "video_diffusion_transformer_02_b200", "_build.py")
+    spec = importlib.util.spec_from_file_location("vattn_build", path)
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    return mod
+
+
+def pytest_sessionstart(session):
+    # Build the CUDA library (cross-compiles on a CPU host) and the oracle
+    # before any test imports them.
+    load_build_module().build()
+    import oracle
+    oracle.build()
+
+
 def pytest_configure(config):
     config.addinivalue_line("markers", "gpu: needs a CUDA B200 (sm_100a) device")
 

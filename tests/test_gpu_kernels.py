@@ -1,0 +1,133 @@
+"""GPU parity of the individual kernels against plain definitions and the
+fp64 oracle, on small shapes that still span several tiles and a ragged
+tail.  All calls go through the C ABI (ctypes binding)."""
+import numpy as np
+import pytest
+
+import oracle
+import seeded_inputs as si
+from helpers import assert_parity, bits_of, errors, from_dev, gather_rows, to_dev
+
+pytestmark = pytest.mark.gpu
+LSE_TOL = 1e-2
+
+
+@pytest.fixture(scope="module")
+def va():
+    import video_diffusion_transformer_02_b200 as va
+    return va
+
+
+# ------------------------------------------------------- tensor-core layouts
+@pytest.mark.parametrize("variant", [0, 1, 2, 3])
+def test_umma_layouts(va, variant):
+    import torch
+    a = si.normal_bf16(100 + variant, (128, 128))
+    b = si.normal_bf16(200 + variant, (128, 128))
+    out = torch.full((128, 128), float("nan"), dtype=torch.float32, device="cuda")
+    va.vattn_selftest_umma(variant, to_dev(a), to_dev(b), out)
+    va.vattn_check()
+    A, Bm = si.bf16_bits_to_f64(a), si.bf16_bits_to_f64(b)
+    ref = {0: A @ Bm.T, 1: A @ Bm, 2: A @ Bm, 3: A.T @ Bm}[variant]
+    got = out.cpu().numpy().astype(np.float64)
+    assert np.max(np.abs(got - ref)) < 1e-3 * np.max(np.abs(ref)), "layout variant %d" % variant
+
+
+# ------------------------------------------------------------------- RoPE
+def _rope(va, Hg, Wg, pairs, max_pos):
+    return va.Rope(Hg=Hg, Wg=Wg, pairs=pairs, max_pos=max_pos, theta=10000.0)
+
+
+@pytest.mark.parametrize("shape,grid,pairs,off", [
+    ((1, 48, 2, 64), (4, 4), (12, 10, 10), 0),
+    ((2, 300, 3, 128), (6, 10), (22, 21, 21), 3),
+])
+def test_rope_qk(va, shape, grid, pairs, off):
+    import torch
+    B, L, H, d = shape
+    q = si.normal_bf16(1, shape)
+    k = si.normal_bf16(2, (B, L, 1, d))
+    r = _rope(va, grid[0], grid[1], pairs, 16)
+    tab = va.rope_table(r, d)
+    qo = torch.empty(shape, dtype=torch.bfloat16, device="cuda")
+    ko = torch.empty((B, L, 1, d), dtype=torch.bfloat16, device="cuda")
+    va.vattn_rope_qk(to_dev(q), to_dev(k), qo, ko, r, tab, frame_offset=off)
+    rq = oracle.rope(q, grid[0], grid[1], pairs, 1e4, t_offset=off)
+    rk = oracle.rope(k, grid[0], grid[1], pairs, 1e4, t_offset=off)
+    for got, ref in ((from_dev(qo), rq), (from_dev(ko), rk)):
+        # fp32 rotation rounded once to bf16: within one bf16 ulp of the exact value
+        assert np.all(np.abs(got - ref) <= np.abs(ref) * 2.0 ** -8 + 1e-6)
+
+
+# -------------------------------------------------------------- attention
+CASES = [
+    # (B, T, Hg, Wg, H, Hkv, d, mode, kwargs, rope)
+    (1, 3, 4, 4, 2, 2, 64, "full", {}, True),                       # the tiny config
+    (1, 5, 6, 10, 2, 2, 128, "full", {}, False),                    # 300 tokens: ragged tail
+    (2, 5, 6, 10, 4, 2, 64, "full", {}, True),                      # GQA, batch 2
+    (1, 7, 5, 9, 2, 2, 128, "chunk_causal", dict(chunk=2), True),   # chunks not tile aligned
+    (1, 7, 5, 9, 2, 2, 64, "chunk_causal", dict(chunk=3), False),
+    (1, 9, 4, 10, 2, 2, 128, "sliding", dict(wb=2, wf=0), True),
+    (1, 9, 4, 10, 2, 2, 64, "sliding", dict(wb=1, wf=1), False),
+    (1, 6, 8, 16, 2, 1, 128, "sliding", dict(wb=4, wf=0), True),    # F = 128: tile aligned frames
+]
+
+
+def _attention_case(va, B, T, Hg, Wg, H, Hkv, d, mode, kw, use_rope, seed=0, qoff=0, koff=0):
+    import torch
+    F = Hg * Wg
+    L = T * F
+    q = si.normal_bf16(10 + seed, (B, L, H, d))
+    k = si.normal_bf16(11 + seed, (B, L, Hkv, d))
+    v = si.normal_bf16(12 + seed, (B, L, Hkv, d))
+    scale = d ** -0.5
+    o = torch.full((B, L, H, d), float("nan"), dtype=torch.bfloat16, device="cuda")
+    lse = torch.full((B, H, L), float("nan"), dtype=torch.float32, device="cuda")
+    rope = tab = None
+    orope = None
+    pairs = (12, 10, 10) if d == 64 else (22, 21, 21)
+    if use_rope:
+        rope = _rope(va, Hg, Wg, pairs, max(T + qoff + koff, Hg, Wg) + 1)
+        tab = va.rope_table(rope, d)
+        orope = dict(Hg=Hg, Wg=Wg, pairs=pairs, theta=1e4)
+    va.vattn_attention(to_dev(q), to_dev(k), to_dev(v), o, lse, scale=scale, mode=mode,
+                       tokens_per_frame=F, chunk_frames=kw.get("chunk", 1),
+                       window_back=kw.get("wb", 0), window_fwd=kw.get("wf", 0),
+                       q_frame_offset=qoff, k_frame_offset=koff, rope=rope, table=tab)
+    va.vattn_check()
+    ro, rl = oracle.attention(q, k, v, scale, mode=mode, F=F, chunk=kw.get("chunk", 1),
+                              wb=kw.get("wb", 0), wf=kw.get("wf", 0), q_frame_offset=qoff,
+                              k_frame_offset=koff, rope=orope)
+    return from_dev(o), lse.cpu().numpy().astype(np.float64), ro, rl
+
+
+@pytest.mark.parametrize("case", CASES, ids=lambda c: "%s-d%d-T%dx%dx%d-H%d/%d%s" % (
+    c[7], c[6], c[1], c[2], c[3], c[4], c[5], "-rope" if c[9] else ""))
+def test_attention_parity(va, case):
+    B, T, Hg, Wg, H, Hkv, d, mode, kw, use_rope = case
+    got, glse, ref, rlse = _attention_case(va, B, T, Hg, Wg, H, Hkv, d, mode, kw, use_rope)
+    assert_parity(got, ref, "attention %s" % (case,))
+    # lse: the kernel rounds rotated q, k to bf16 before the products, which
+    # moves each score by ~2e-3 rms (2^-9 relative per operand over d terms);
+    # lse is a convex combination of those score errors.
+    assert np.max(np.abs(glse - rlse)) < LSE_TOL, "lse"
+
+
+def test_attention_frame_offsets(va):
+    # Offsets move the frames of queries and keys (masks and RoPE t).
+    got, _, ref, _ = _attention_case(va, 1, 6, 5, 8, 2, 2, 128, "sliding", dict(wb=1, wf=0), True,
+                                     qoff=2, koff=1)
+    assert_parity(got, ref, "offsets")
+
+
+def test_attention_single_token_and_tiny_lengths(va):
+    import torch
+    for L in (1, 7, 129):
+        q = si.normal_bf16(70, (1, L, 1, 64))
+        k = si.normal_bf16(71, (1, L, 1, 64))
+        v = si.normal_bf16(72, (1, L, 1, 64))
+        o = torch.empty((1, L, 1, 64), dtype=torch.bfloat16, device="cuda")
+        va.vattn_attention(to_dev(q), to_dev(k), to_dev(v), o, scale=0.125)
+        va.vattn_check()
+        ref, _ = oracle.attention(q, k, v, 0.125)
+        assert_parity(from_dev(o), ref, "L=%d" % L)

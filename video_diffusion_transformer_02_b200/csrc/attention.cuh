@@ -1,0 +1,652 @@
+// Attention forward for sm_100a: one CTA per 128-query tile of one head.
+//
+// What it computes (per query row i, visible key set A(i) given by the
+// mode): o_i = sum_{j in A(i)} softmax_j(scale * q_i . k_j) v_j, with q and
+// k optionally rotated by 3D-RoPE at their (t, h, w) positions — the
+// spatiotemporal self-attention of Wan-style DiTs and of FlashDecoder
+// ("Transformer Backbone Design" Sec. 3.2; "Streaming with Rolling KV
+// Cache" Sec. 3.3).  The HYBRID variant adds MobileWan's causal linear
+// attention across chunks: the online-softmax state of each query tile
+// starts from phi(Q) S_c and phi(Q) z_c (one joint normalisation).
+//
+// Warp roles (one elected lane issues for the single-thread roles):
+//   warp 0        TMA producer: Q tile once, then K tiles (multi-stage ring)
+//   warp 1        TMEM allocation + tcgen05.mma issue
+//   warp 2        TMA producer: V tiles
+//   warps 4..7    softmax warpgroup: thread r owns query row r of the tile
+//                 (TMEM lane r); scores, online softmax, P (bf16) into TMEM,
+//                 O rescale, epilogue
+//   warps 8..11   aux warpgroup: RoPE of the Q tile and of every K tile in
+//                 shared memory (ROPE), or the fp32 -> bf16 hi/lo split of
+//                 the chunk state S_c (HYBRID)
+//
+// TMEM columns (512 allocated): S double buffer [0,128) and [128,256) fp32,
+// O [256, 256+D) fp32, P [384, 448) bf16 pairs (also phi(Q) for HYBRID).
+// S = Q K^T is an SS MMA (both operands K-major, 128B swizzle);
+// O += P V is a TS MMA (P from TMEM, V MN-major in shared memory).
+#pragma once
+#include "common.cuh"
+
+namespace vattn {
+namespace attn {
+
+using namespace sm100;
+
+constexpr int kTileM = 128;   // query rows per CTA
+constexpr int kTileN = 128;   // keys per tile
+constexpr int kMaxKeySegments = 8;
+constexpr uint32_t kColS0 = 0, kColS1 = 128, kColO = 256, kColP = 384;
+constexpr uint32_t kTmemCols = 512;
+// Rescale O only when the running max grows by more than this (log2
+// units): stale maxima keep every exp2 argument below it, so fp32 stays
+// far from overflow while most tiles skip the O correction.
+constexpr float kRescaleThreshold = 8.0f;
+
+enum Mode : int { kFull = 0, kChunkCausal = 1, kSliding = 2 };
+
+struct KeySegment {
+  int map;      // 0: k/v maps, 1: k2/v2 maps
+  int c3_base;  // fourth TMA coordinate = c3_base + batch index
+  int tok0;     // first token of the segment along the token axis
+  int n_tok;    // tokens in the segment
+  int frame;    // absolute frame index (RoPE t of every key in it)
+  int tile0;    // number of key tiles in earlier segments
+};
+
+struct Params {
+  __nv_bfloat16* o;
+  float* lse;
+  uint32_t* status;
+  int B, Lq, Lk, H, Hkv;
+  float scale_log2;         // scale * log2(e)
+  int mode, F, chunk, wb, wf, qoff, koff;
+  int q_seg_len;            // query tiles restart at multiples of this
+  int q_tiles_per_seg;
+  int n_q_tiles;
+  int reverse_q;            // heaviest tiles first (chunk-causal)
+  int n_kseg;               // 0: contiguous keys with the mode's masks
+  KeySegment kseg[kMaxKeySegments];
+  // RoPE
+  const float2* rope_tab;   // [max_pos][D/2] (cos, sin)
+  int rope_Hg, rope_Wg, rope_pt, rope_ph, rope_maxpos;
+  // HYBRID: per-chunk exclusive state prefix
+  const float* hyb_S;       // [C][B][H][D][D]
+  const float* hyb_z;       // [C][B][H][D]
+};
+
+template <int D, bool HYBRID>
+struct Cfg {
+  static constexpr int kTileBytes = kTileM * D * 2;  // one 128 x D bf16 tile
+  static constexpr int kBlocks = D / 64;             // 64-column swizzle blocks per tile
+  static constexpr int kStages = (D == 128) ? (HYBRID ? 2 : 3) : 4;
+  static constexpr int kOffQ = 0;
+  static constexpr int kOffK = kOffQ + kTileBytes;
+  static constexpr int kOffV = kOffK + kStages * kTileBytes;
+  static constexpr int kOffShi = kOffV + kStages * kTileBytes;
+  static constexpr int kOffSlo = kOffShi + (HYBRID ? D * D * 2 : 0);
+  static constexpr int kOffBar = kOffSlo + (HYBRID ? D * D * 2 : 0);
+  static constexpr int kNumBars = 2 + 5 * kStages + 4 + 2 + 2 + 1;
+  static constexpr int kOffMisc = kOffBar + kNumBars * 8;
+  static constexpr int kSmemBytes = kOffMisc + 64 + 1024;  // + alignment slack
+};
+
+// Visible key range [lo, hi) of query token n (contiguous keys).  For all
+// three modes the visible keys of one query are an interval and both ends
+// are non-decreasing in n.
+__device__ __forceinline__ void key_range(const Params& p, int n, int& lo, int& hi) {
+  if (p.mode == kFull) {
+    lo = 0;
+    hi = p.Lk;
+    return;
+  }
+  const long long fq = p.qoff + n / p.F;
+  long long a, b;
+  if (p.mode == kChunkCausal) {
+    a = 0;
+    b = ((fq / p.chunk) + 1) * p.chunk - p.koff;
+  } else {
+    a = fq - p.wb - p.koff;
+    b = fq + p.wf + 1 - p.koff;
+  }
+  a *= p.F;
+  b *= p.F;
+  lo = static_cast<int>(a < 0 ? 0 : (a > p.Lk ? p.Lk : a));
+  hi = static_cast<int>(b < 0 ? 0 : (b > p.Lk ? p.Lk : b));
+}
+
+struct TileGeom {
+  int q0, q_end;      // query rows [q0, q_end) of this CTA
+  int kbeg, kend;     // contiguous key range covered by tiles
+  int n_tiles;
+};
+
+__device__ __forceinline__ TileGeom tile_geom(const Params& p, int qt) {
+  TileGeom g;
+  const int seg = qt / p.q_tiles_per_seg;
+  const int t = qt - seg * p.q_tiles_per_seg;
+  g.q0 = seg * p.q_seg_len + t * kTileM;
+  int e = (seg + 1) * p.q_seg_len;
+  if (e > p.Lq) e = p.Lq;
+  g.q_end = min(g.q0 + kTileM, e);
+  if (p.n_kseg == 0) {
+    int lo0, hi0, lo1, hi1;
+    key_range(p, g.q0, lo0, hi0);
+    key_range(p, g.q_end - 1, lo1, hi1);
+    g.kbeg = lo0;
+    g.kend = hi1;
+    g.n_tiles = g.kend > g.kbeg ? (g.kend - g.kbeg + kTileN - 1) / kTileN : 0;
+  } else {
+    g.kbeg = g.kend = 0;
+    const KeySegment& last = p.kseg[p.n_kseg - 1];
+    g.n_tiles = last.tile0 + (last.n_tok + kTileN - 1) / kTileN;
+  }
+  return g;
+}
+
+struct KeyTile {
+  int map, c3, k0;    // TMA source: map, 4th coordinate (minus batch), token start
+  int valid;          // keys in this tile that exist (segment mode)
+  int frame;          // segment frame (segment mode)
+};
+
+__device__ __forceinline__ KeyTile key_tile(const Params& p, const TileGeom& g, int j) {
+  KeyTile kt;
+  if (p.n_kseg == 0) {
+    kt.map = 0;
+    kt.c3 = 0;
+    kt.k0 = g.kbeg + j * kTileN;
+    kt.valid = min(kTileN, g.kend - kt.k0);
+    kt.frame = 0;
+  } else {
+    int s = 0;
+#pragma unroll 1
+    for (int i = 1; i < p.n_kseg; ++i)
+      if (p.kseg[i].tile0 <= j) s = i;
+    const KeySegment& sg = p.kseg[s];
+    const int t = j - sg.tile0;
+    kt.map = sg.map;
+    kt.c3 = sg.c3_base;
+    kt.k0 = sg.tok0 + t * kTileN;
+    kt.valid = min(kTileN, sg.n_tok - t * kTileN);
+    kt.frame = sg.frame;
+  }
+  return kt;
+}
+
+// (t, h, w) -> table rows for the rotation of one token.
+struct RopePos {
+  int t, h, w;
+};
+
+// Rotate one 128-byte-swizzled 128 x D bf16 tile row in place: channel pair
+// j of the row turns by the angle of its axis position.  Row r of a tile is
+// contiguous 64-element blocks, one per swizzle block.
+template <int D>
+__device__ __forceinline__ void rope_row_inplace(uint32_t tile, uint32_t r, RopePos pos,
+                                                 const Params& p) {
+  const float2* tab = p.rope_tab;
+  const int pt = p.rope_pt, pth = p.rope_pt + p.rope_ph;
+  const float2* row_t = tab + pos.t * (D / 2);
+  const float2* row_h = tab + pos.h * (D / 2);
+  const float2* row_w = tab + pos.w * (D / 2);
+#pragma unroll 4
+  for (int c16 = 0; c16 < D / 8; ++c16) {
+    const uint32_t addr = tile + (c16 >> 3) * (kTileM * 128) + sw128_offset(r, c16 & 7);
+    uint4 v = lds128(addr);
+    uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int j = c16 * 4 + e;
+      const float2* src = j < pt ? row_t : (j < pth ? row_h : row_w);
+      const float2 cs = __ldg(src + j);
+      const float x0 = bf16lo_to_f32(w4[e]), x1 = bf16hi_to_f32(w4[e]);
+      const float y0 = x0 * cs.x - x1 * cs.y;
+      const float y1 = x0 * cs.y + x1 * cs.x;
+      w4[e] = pack_bf16x2(y0, y1);
+    }
+    sts128(addr, make_uint4(w4[0], w4[1], w4[2], w4[3]));
+  }
+}
+
+template <int D, bool ROPE, bool HYBRID>
+__global__ void __launch_bounds__(384, 1)
+    attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                    const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmK2,
+                    const __grid_constant__ CUtensorMap tmV2, const Params p) {
+  using C = Cfg<D, HYBRID>;
+  constexpr int NS = C::kStages;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sbase = smem_addr(smem);
+  const uint32_t sQ = sbase + C::kOffQ, sK = sbase + C::kOffK, sV = sbase + C::kOffV;
+  const uint32_t sShi = sbase + C::kOffShi, sSlo = sbase + C::kOffSlo;
+  const uint32_t bar0 = sbase + C::kOffBar;
+  // barrier map
+  const uint32_t bQFull = bar0, bQReady = bar0 + 8;
+  auto bKFull = [&](int s) { return bar0 + 16 + 8 * s; };
+  auto bKReady = [&](int s) { return bar0 + 16 + 8 * (NS + s); };
+  auto bKEmpty = [&](int s) { return bar0 + 16 + 8 * (2 * NS + s); };
+  auto bVFull = [&](int s) { return bar0 + 16 + 8 * (3 * NS + s); };
+  auto bVEmpty = [&](int s) { return bar0 + 16 + 8 * (4 * NS + s); };
+  const uint32_t bx = bar0 + 16 + 8 * 5 * NS;
+  auto bSFull = [&](int b) { return bx + 8 * b; };
+  auto bSFree = [&](int b) { return bx + 16 + 8 * b; };
+  const uint32_t bPFull = bx + 32, bPvDone = bx + 40;
+  const uint32_t bPhiReady = bx + 48, bSReady = bx + 56, bFinal = bx + 64;
+  uint32_t* misc = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
+  volatile uint32_t* tmem_slot = misc;
+  volatile uint32_t* abort_flag = misc + 1;
+  Abort ab{abort_flag, p.status};
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int h = blockIdx.y, b = blockIdx.z;
+  const int kvh = h / (p.H / p.Hkv);
+  const int qt = p.reverse_q ? (p.n_q_tiles - 1 - blockIdx.x) : blockIdx.x;
+  const TileGeom g = tile_geom(p, qt);
+  if (g.q0 >= g.q_end) return;   // tile past the end of a short last segment
+  const int nk = g.n_tiles;
+
+  if (threadIdx.x == 0) {
+    mbar_init(bQFull, 1);
+    mbar_init(bQReady, 4);
+    for (int s = 0; s < NS; ++s) {
+      mbar_init(bKFull(s), 1);
+      mbar_init(bKReady(s), 4);
+      mbar_init(bKEmpty(s), 1);
+      mbar_init(bVFull(s), 1);
+      mbar_init(bVEmpty(s), 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(bSFull(i), 1);
+      mbar_init(bSFree(i), 4);
+    }
+    mbar_init(bPFull, 4);
+    mbar_init(bPvDone, 1);
+    mbar_init(bPhiReady, 4);
+    mbar_init(bSReady, 4);
+    mbar_init(bFinal, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tmQ);
+    tma_prefetch_desc(&tmK);
+    tma_prefetch_desc(&tmV);
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_addr(const_cast<uint32_t*>(tmem_slot)), kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------ producer: Q, then K
+    if (lane == 0) {
+      mbar_arrive_expect_tx(bQFull, C::kTileBytes);
+#pragma unroll
+      for (int blk = 0; blk < C::kBlocks; ++blk)
+        tma_load_4d(sQ + blk * (kTileM * 128), &tmQ, bQFull, blk * 64, h, g.q0, b);
+      int j = 0;
+      for (; j < nk; ++j) {
+        const int s = j % NS;
+        if (j >= NS && !mbar_wait(bKEmpty(s), ((j / NS) - 1) & 1, ab, kStatusTimeoutProducer)) break;
+        const KeyTile kt = key_tile(p, g, j);
+        const CUtensorMap* m = kt.map ? &tmK2 : &tmK;
+        mbar_arrive_expect_tx(bKFull(s), C::kTileBytes);
+#pragma unroll
+        for (int blk = 0; blk < C::kBlocks; ++blk)
+          tma_load_4d(sK + s * C::kTileBytes + blk * (kTileM * 128), m, bKFull(s), blk * 64, kvh, kt.k0,
+                      kt.c3 + b);
+      }
+      // drain: wait until every load issued so far has landed
+      for (int i = max(0, j - NS); i < j; ++i) {
+        const uint64_t t0 = global_timer_ns();
+        while (!mbar_try_wait(bKFull(i % NS), (i / NS) & 1) && global_timer_ns() - t0 < kWaitLimitNs) {
+        }
+      }
+      const uint64_t t0 = global_timer_ns();
+      while (!mbar_try_wait(bQFull, 0) && global_timer_ns() - t0 < kWaitLimitNs) {
+      }
+    }
+  } else if (warp == 2) {
+    // ----------------------------------------------------- producer: V
+    if (lane == 0) {
+      int j = 0;
+      for (; j < nk; ++j) {
+        const int s = j % NS;
+        if (j >= NS && !mbar_wait(bVEmpty(s), ((j / NS) - 1) & 1, ab, kStatusTimeoutProducer)) break;
+        const KeyTile kt = key_tile(p, g, j);
+        const CUtensorMap* m = kt.map ? &tmV2 : &tmV;
+        mbar_arrive_expect_tx(bVFull(s), C::kTileBytes);
+#pragma unroll
+        for (int blk = 0; blk < C::kBlocks; ++blk)
+          tma_load_4d(sV + s * C::kTileBytes + blk * (kTileM * 128), m, bVFull(s), blk * 64, kvh, kt.k0,
+                      kt.c3 + b);
+      }
+      for (int i = max(0, j - NS); i < j; ++i) {
+        const uint64_t t0 = global_timer_ns();
+        while (!mbar_try_wait(bVFull(i % NS), (i / NS) & 1) && global_timer_ns() - t0 < kWaitLimitNs) {
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------- MMA
+    if (lane == 0) {
+      constexpr uint32_t idQK = idesc_bf16_f32(kTileM, kTileN, false, false);
+      constexpr uint32_t idPV = idesc_bf16_f32(kTileM, D, false, true);
+      const uint32_t tO = tmem + kColO, tP = tmem + kColP;
+      bool ok = true;
+      if constexpr (HYBRID) {
+        ok = mbar_wait(bPhiReady, 0, ab, kStatusTimeoutMma) && mbar_wait(bSReady, 0, ab, kStatusTimeoutMma);
+        if (ok) {
+          tc_fence_after();
+          // O = phi(Q) S_hi + phi(Q) S_lo   (B operands MN-major, K = key features)
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk)
+            umma_ts(tO, tP + kk * 8, sdesc_sw128(sShi + kk * 2048, D * 128, 1024), idPV, kk > 0);
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk)
+            umma_ts(tO, tP + kk * 8, sdesc_sw128(sSlo + kk * 2048, D * 128, 1024), idPV, 1);
+          umma_commit(bPvDone);
+        }
+      }
+      if (ok) ok = mbar_wait(ROPE ? bQReady : bQFull, 0, ab, kStatusTimeoutMma);
+      tc_fence_after();
+      auto issue_pv = [&](int i) -> bool {
+        if (!mbar_wait(bPFull, i & 1, ab, kStatusTimeoutMma)) return false;
+        const int s = i % NS;
+        if (!mbar_wait(bVFull(s), (i / NS) & 1, ab, kStatusTimeoutMma)) return false;
+        tc_fence_after();
+        const uint32_t vb = sV + s * C::kTileBytes;
+#pragma unroll
+        for (int kk = 0; kk < kTileN / 16; ++kk)
+          umma_ts(tO, tP + kk * 8, sdesc_sw128(vb + kk * 2048, kTileM * 128, 1024), idPV,
+                  (HYBRID || i > 0 || kk > 0) ? 1u : 0u);
+        umma_commit(bPvDone);
+        umma_commit(bVEmpty(s));
+        return true;
+      };
+      for (int j = 0; ok && j < nk; ++j) {
+        const int s = j % NS, buf = j & 1;
+        if (!mbar_wait(ROPE ? bKReady(s) : bKFull(s), (j / NS) & 1, ab, kStatusTimeoutMma)) break;
+        if (j >= 2 && !mbar_wait(bSFree(buf), ((j - 2) >> 1) & 1, ab, kStatusTimeoutMma)) break;
+        tc_fence_after();
+        const uint32_t kb = sK + s * C::kTileBytes;
+        const uint32_t tS = tmem + (buf ? kColS1 : kColS0);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * (kTileM * 128) + (kk & 3) * 32;
+          umma_ss(tS, sdesc_sw128(sQ + off, 16, 1024), sdesc_sw128(kb + off, 16, 1024), idQK, kk > 0);
+        }
+        umma_commit(bSFull(buf));
+        umma_commit(bKEmpty(s));
+        if (j >= 1 && !issue_pv(j - 1)) {
+          ok = false;
+          break;
+        }
+      }
+      if (ok && nk > 0) issue_pv(nk - 1);
+      // all issued MMAs complete before teardown
+      umma_commit(bFinal);
+      const uint64_t t0 = global_timer_ns();
+      while (!mbar_try_wait(bFinal, 0) && global_timer_ns() - t0 < kWaitLimitNs) {
+      }
+    }
+  } else if (warp >= 4 && warp < 8) {
+    // ---------------------------------------------------------- softmax
+    const int r = threadIdx.x - 128;                 // row of the tile = TMEM lane
+    const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const uint32_t trow = tmem + lane_base;
+    const int qn = g.q0 + r;
+    const bool row_valid = qn < g.q_end;
+    int lo = 0, hi = 0;
+    if (p.n_kseg == 0) key_range(p, row_valid ? qn : g.q_end - 1, lo, hi);
+    float m_run = -INFINITY, l_run = 0.f;
+    const float sl2 = p.scale_log2;
+    bool ok = true;
+    int pv_phase = 0;   // completions of bPvDone observed so far
+    if constexpr (HYBRID) {
+      // phi(q_r) -> TMEM P columns (bf16); D_lin = phi(q_r) . z_c in fp32
+      ok = mbar_wait(bQFull, 0, ab, kStatusTimeoutSoftmax);
+      const int c = g.q0 / p.q_seg_len;
+      const float* zc = p.hyb_z + ((static_cast<size_t>(c) * p.B + b) * p.H + h) * D;
+      float dl = 0.f;
+#pragma unroll
+      for (int half = 0; half < D / 64; ++half) {
+        uint32_t pk[32];
+#pragma unroll
+        for (int c8 = 0; c8 < 8; ++c8) {
+          const uint4 v = lds128(sQ + half * (kTileM * 128) + sw128_offset(r, c8));
+          const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int ch = half * 64 + c8 * 8 + 2 * e;
+            float x0 = bf16lo_to_f32(w4[e]), x1 = bf16hi_to_f32(w4[e]);
+            x0 = x0 > 0.f ? x0 + 1.f : __expf(x0);
+            x1 = x1 > 0.f ? x1 + 1.f : __expf(x1);
+            dl = fmaf(x0, __ldg(zc + ch), dl);
+            dl = fmaf(x1, __ldg(zc + ch + 1), dl);
+            pk[c8 * 4 + e] = pack_bf16x2(x0, x1);
+          }
+        }
+        tmem_st32(trow + kColP + half * 32, pk);
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bPhiReady);
+      m_run = 0.f;            // the linear part enters with reference max 0
+      l_run = dl;
+    }
+    for (int j = 0; ok && j < nk; ++j) {
+      const int buf = j & 1;
+      if (!mbar_wait(bSFull(buf), (j >> 1) & 1, ab, kStatusTimeoutSoftmax)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const uint32_t tS = trow + (buf ? kColS1 : kColS0);
+      int col_lo = 0, col_hi = kTileN;
+      if (p.n_kseg == 0) {
+        const int k0 = g.kbeg + j * kTileN;
+        col_lo = lo - k0;
+        col_hi = hi - k0;
+      } else {
+        const KeyTile kt = key_tile(p, g, j);
+        col_hi = kt.valid;
+      }
+      const bool masked = col_lo > 0 || col_hi < kTileN;
+      // pass 1: row max
+      float mx = -INFINITY;
+#pragma unroll
+      for (int q4 = 0; q4 < 4; ++q4) {
+        uint32_t sr[32];
+        tmem_ld32(tS + q4 * 32, sr);
+        tmem_ld_wait();
+#pragma unroll
+        for (int c = 0; c < 32; ++c) {
+          const int col = q4 * 32 + c;
+          const float x = __uint_as_float(sr[c]);
+          const bool vis = !masked || (col >= col_lo && col < col_hi);
+          mx = fmaxf(mx, vis ? x : -INFINITY);
+        }
+      }
+      const float m_tile = mx * sl2;
+      const float m_new = fmaxf(m_run, m_tile);
+      float factor = 1.f;
+      bool resc = false;
+      if (m_new > m_run + kRescaleThreshold) {
+        factor = ex2_approx(m_run - m_new);   // 0 when m_run = -inf
+        m_run = m_new;
+        resc = true;
+      }
+      const float m_use = (m_run == -INFINITY) ? 0.f : m_run;
+      // pass 2: P = exp2(s*scale*log2e - m), row sum, bf16 pack
+      uint32_t pkA[32], pkB[32];   // P columns [0, 32) and [32, 64): keys 0-63, 64-127
+      float rs = 0.f;
+#pragma unroll
+      for (int q4 = 0; q4 < 4; ++q4) {
+        uint32_t sr[32];
+        tmem_ld32(tS + q4 * 32, sr);
+        tmem_ld_wait();
+#pragma unroll
+        for (int c = 0; c < 32; c += 2) {
+          const int col = q4 * 32 + c;
+          const bool v0 = !masked || (col >= col_lo && col < col_hi);
+          const bool v1 = !masked || (col + 1 >= col_lo && col + 1 < col_hi);
+          const float p0 = v0 ? ex2_approx(fmaf(__uint_as_float(sr[c]), sl2, -m_use)) : 0.f;
+          const float p1 = v1 ? ex2_approx(fmaf(__uint_as_float(sr[c + 1]), sl2, -m_use)) : 0.f;
+          rs += p0 + p1;
+          const uint32_t w = pack_bf16x2(p0, p1);
+          if (q4 < 2) pkA[q4 * 16 + c / 2] = w; else pkB[(q4 - 2) * 16 + c / 2] = w;
+        }
+      }
+      // S buffer consumed
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bSFree(buf));
+      // previous P V (or the hybrid linear init) must be complete before
+      // touching O or overwriting P
+      const int need = j + (HYBRID ? 1 : 0);   // bPvDone completions required
+      if (pv_phase < need) {
+        if (!mbar_wait(bPvDone, (need - 1) & 1, ab, kStatusTimeoutSoftmax)) {
+          ok = false;
+          break;
+        }
+        pv_phase = need;
+        tc_fence_after();
+      }
+      const bool o_valid = HYBRID || j > 0;
+      if (__any_sync(0xffffffffu, resc && o_valid)) {
+        const float f = (resc && o_valid) ? factor : 1.f;
+#pragma unroll 1
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t orr[32];
+          tmem_ld32(trow + kColO + c * 32, orr);
+          tmem_ld_wait();
+#pragma unroll
+          for (int e = 0; e < 32; ++e) orr[e] = __float_as_uint(__uint_as_float(orr[e]) * f);
+          tmem_st32(trow + kColO + c * 32, orr);
+        }
+      }
+      tmem_st32(trow + kColP, pkA);
+      tmem_st32(trow + kColP + 32, pkB);
+      tmem_st_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bPFull);
+      l_run = l_run * factor + rs;
+    }
+    // epilogue: O / l -> bf16, lse
+    const int need = nk + (HYBRID ? 1 : 0);
+    if (ok && need > 0 && pv_phase < need) {
+      ok = mbar_wait(bPvDone, (need - 1) & 1, ab, kStatusTimeoutSoftmax);
+      tc_fence_after();
+    }
+    if (ok) {
+      const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
+      __nv_bfloat16* orow = p.o + ((static_cast<size_t>(b) * p.Lq + qn) * p.H + h) * D;
+#pragma unroll 1
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t orr[32];
+        if (need > 0) {
+          tmem_ld32(trow + kColO + c * 32, orr);
+          tmem_ld_wait();
+        } else {
+#pragma unroll
+          for (int e = 0; e < 32; ++e) orr[e] = 0u;
+        }
+        uint32_t w[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e)
+          w[e] = pack_bf16x2(__uint_as_float(orr[2 * e]) * inv, __uint_as_float(orr[2 * e + 1]) * inv);
+        if (row_valid) {
+          uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) dst[e] = make_uint4(w[4 * e], w[4 * e + 1], w[4 * e + 2], w[4 * e + 3]);
+        }
+      }
+      if (p.lse && row_valid) {
+        const float lse = l_run > 0.f ? (m_run + __log2f(l_run)) * 0.69314718055994531f : -INFINITY;
+        p.lse[(static_cast<size_t>(b) * p.H + h) * p.Lq + qn] = lse;
+      }
+    }
+  } else if (warp >= 8) {
+    // ------------------------------------------------------ aux warpgroup
+    const int r = threadIdx.x - 256;
+    if constexpr (ROPE) {
+      const int Fr = p.rope_Hg * p.rope_Wg;
+      bool ok = mbar_wait(bQFull, 0, ab, kStatusTimeoutAux);
+      if (ok) {
+        const int n = g.q0 + r;
+        RopePos pos{0, 0, 0};
+        if (n < g.q_end) {
+          const int in = n % Fr;
+          pos = RopePos{p.qoff + n / Fr, in / p.rope_Wg, in % p.rope_Wg};
+        }
+        rope_row_inplace<D>(sQ, r, pos, p);
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bQReady);
+      }
+      for (int j = 0; ok && j < nk; ++j) {
+        const int s = j % NS;
+        if (!mbar_wait(bKFull(s), (j / NS) & 1, ab, kStatusTimeoutAux)) break;
+        const KeyTile kt = key_tile(p, g, j);
+        RopePos pos{0, 0, 0};
+        if (p.n_kseg == 0) {
+          const int n = kt.k0 + r;
+          if (n < p.Lk) {
+            const int in = n % Fr;
+            pos = RopePos{p.koff + n / Fr, in / p.rope_Wg, in % p.rope_Wg};
+          }
+        } else if (r < kt.valid) {
+          const int in = kt.k0 + r;   // token index inside its frame
+          pos = RopePos{kt.frame, in / p.rope_Wg, in % p.rope_Wg};
+        }
+        rope_row_inplace<D>(sK + s * C::kTileBytes, r, pos, p);
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bKReady(s));
+      }
+    } else if constexpr (HYBRID) {
+      // S_c (fp32 [D][D], row a = key feature) -> bf16 hi + lo, MN-major
+      // 128B-swizzled B operand tiles (64-column blocks of D rows).
+      const int c = g.q0 / p.q_seg_len;
+      const float* src = p.hyb_S + (((static_cast<size_t>(c) * p.B + b) * p.H + h) * D + r) * D;
+      if (r < D) {
+#pragma unroll 2
+        for (int c8 = 0; c8 < D / 8; ++c8) {
+          const float4 a0 = __ldg(reinterpret_cast<const float4*>(src + c8 * 8));
+          const float4 a1 = __ldg(reinterpret_cast<const float4*>(src + c8 * 8 + 4));
+          const float x[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+          uint32_t hi4[4], lo4[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            hi4[e] = pack_bf16x2(x[2 * e], x[2 * e + 1]);
+            lo4[e] = pack_bf16x2(x[2 * e] - bf16lo_to_f32(hi4[e]), x[2 * e + 1] - bf16hi_to_f32(hi4[e]));
+          }
+          const uint32_t off = (c8 >> 3) * (D * 128) + sw128_offset(r, c8 & 7);
+          sts128(sShi + off, make_uint4(hi4[0], hi4[1], hi4[2], hi4[3]));
+          sts128(sSlo + off, make_uint4(lo4[0], lo4[1], lo4[2], lo4[3]));
+        }
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bSReady);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+}  // namespace attn
+}  // namespace vattn

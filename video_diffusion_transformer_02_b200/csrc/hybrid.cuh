@@ -1,0 +1,235 @@
+// Hybrid chunk attention, state part (MobileWan recurrence distillation:
+// causal linear attention across chunks carried in a running state (s, z),
+// feature map phi(x) = elu(x) + 1 after Katharopoulos et al.).
+//
+//   dS_c = sum_{j in chunk c} phi(k_j) v_j^T   (D x D, fp32)   -- tcgen05 MMA
+//   dz_c = sum_{j in chunk c} phi(k_j)          (D, fp32)       -- CUDA cores
+//   S_c  = S_in + sum_{c' < c} dS_c'  (exclusive scan over chunks), same for z
+//
+// The attention part (softmax inside the chunk plus the linear read-out of
+// S_c, z_c) is the HYBRID variant of the attention kernel.
+#pragma once
+#include "common.cuh"
+
+namespace vattn {
+namespace hyb {
+
+using namespace sm100;
+
+struct DeltaParams {
+  float* wsS;        // [C][B][H][D][D]
+  float* wsz;        // [C][B][H][D]
+  uint32_t* status;
+  int B, L, H, chunk;
+};
+
+constexpr int kRows = 128;   // tokens per tile
+
+template <int D>
+struct DeltaCfg {
+  static constexpr int kTileBytes = kRows * D * 2;
+  static constexpr int kStages = 3;
+  static constexpr int kOffK = 0;
+  static constexpr int kOffV = kStages * kTileBytes;
+  static constexpr int kOffBar = 2 * kStages * kTileBytes;
+  static constexpr int kNumBars = 3 * kStages + 1;
+  static constexpr int kOffMisc = kOffBar + kNumBars * 8;
+  static constexpr int kSmemBytes = kOffMisc + 64 + 1024;
+};
+
+// grid (C, H, B), 256 threads: warp 0 TMA, warp 1 TMEM + MMA, warps 4..7
+// feature map / column sums / epilogue.
+template <int D>
+__global__ void __launch_bounds__(256, 1)
+    delta_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                 const DeltaParams p) {
+  static_assert(D == 128, "state delta supports head_dim 128");
+  using C = DeltaCfg<D>;
+  constexpr int NS = C::kStages;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sbase = smem_addr(smem);
+  const uint32_t sK = sbase + C::kOffK, sV = sbase + C::kOffV, bar0 = sbase + C::kOffBar;
+  auto bFull = [&](int s) { return bar0 + 8 * s; };
+  auto bPhi = [&](int s) { return bar0 + 8 * (NS + s); };
+  auto bEmpty = [&](int s) { return bar0 + 8 * (2 * NS + s); };
+  const uint32_t bDone = bar0 + 8 * 3 * NS;
+  uint32_t* misc = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
+  volatile uint32_t* tmem_slot = misc;
+  volatile uint32_t* abort_flag = misc + 1;
+  Abort ab{abort_flag, p.status};
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int c = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  const int c0 = c * p.chunk;
+  const int c1 = min(p.L, c0 + p.chunk);
+  const int nt = (c1 - c0 + kRows - 1) / kRows;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < NS; ++s) {
+      mbar_init(bFull(s), 1);
+      mbar_init(bPhi(s), 4);
+      mbar_init(bEmpty(s), 1);
+    }
+    mbar_init(bDone, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_addr(const_cast<uint32_t*>(tmem_slot)), 128);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      int t = 0;
+      for (; t < nt; ++t) {
+        const int s = t % NS;
+        if (t >= NS && !mbar_wait(bEmpty(s), ((t / NS) - 1) & 1, ab, kStatusTimeoutProducer)) break;
+        mbar_arrive_expect_tx(bFull(s), 2 * C::kTileBytes);
+        const int r0 = c0 + t * kRows;
+#pragma unroll
+        for (int blk = 0; blk < D / 64; ++blk) {
+          tma_load_4d(sK + s * C::kTileBytes + blk * (kRows * 128), &tmK, bFull(s), blk * 64, h, r0, b);
+          tma_load_4d(sV + s * C::kTileBytes + blk * (kRows * 128), &tmV, bFull(s), blk * 64, h, r0, b);
+        }
+      }
+      for (int i = max(0, t - NS); i < t; ++i) {
+        const uint64_t t0 = global_timer_ns();
+        while (!mbar_try_wait(bFull(i % NS), (i / NS) & 1) && global_timer_ns() - t0 < kWaitLimitNs) {
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // D[a][e] += sum_tokens phiK[token][a] * V[token][e]: A = phiK^T and
+      // B = V are both MN-major (tokens are the K dimension of the MMA).
+      constexpr uint32_t id = idesc_bf16_f32(D, D, true, true);
+      for (int t = 0; t < nt; ++t) {
+        const int s = t % NS;
+        if (!mbar_wait(bPhi(s), (t / NS) & 1, ab, kStatusTimeoutMma)) break;
+        tc_fence_after();
+        const uint32_t kb = sK + s * C::kTileBytes, vb = sV + s * C::kTileBytes;
+#pragma unroll
+        for (int kk = 0; kk < kRows / 16; ++kk)
+          umma_ss(tmem, sdesc_sw128(kb + kk * 2048, kRows * 128, 1024),
+                  sdesc_sw128(vb + kk * 2048, kRows * 128, 1024), id, (t > 0 || kk > 0) ? 1u : 0u);
+        umma_commit(bEmpty(s));
+      }
+      umma_commit(bDone);
+      const uint64_t t0 = global_timer_ns();
+      while (!mbar_try_wait(bDone, 0) && global_timer_ns() - t0 < kWaitLimitNs) {
+      }
+    }
+  } else if (warp >= 4) {
+    const int r = threadIdx.x - 128;   // token row of a tile; later feature column
+    float zacc = 0.f;
+    bool ok = true;
+    for (int t = 0; t < nt; ++t) {
+      const int s = t % NS;
+      if (!mbar_wait(bFull(s), (t / NS) & 1, ab, kStatusTimeoutAux)) {
+        ok = false;
+        break;
+      }
+      const uint32_t kb = sK + s * C::kTileBytes;
+      const bool valid = c0 + t * kRows + r < c1;   // rows past the chunk end weigh 0
+#pragma unroll 4
+      for (int c16 = 0; c16 < D / 8; ++c16) {
+        const uint32_t addr = kb + (c16 >> 3) * (kRows * 128) + sw128_offset(r, c16 & 7);
+        const uint4 v = lds128(addr);
+        uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          float x0 = bf16lo_to_f32(w4[e]), x1 = bf16hi_to_f32(w4[e]);
+          x0 = valid ? (x0 > 0.f ? x0 + 1.f : __expf(x0)) : 0.f;
+          x1 = valid ? (x1 > 0.f ? x1 + 1.f : __expf(x1)) : 0.f;
+          w4[e] = pack_bf16x2(x0, x1);
+        }
+        sts128(addr, make_uint4(w4[0], w4[1], w4[2], w4[3]));
+      }
+      fence_proxy_async_smem();
+      asm volatile("bar.sync 1, 128;" ::: "memory");
+      // column sums of the (bf16) feature map: thread r owns feature r
+      {
+        const uint32_t colbase = kb + (r >> 6) * (kRows * 128);
+        const uint32_t chunk = (r & 63) >> 3, within = (r & 7) * 2;
+#pragma unroll 8
+        for (int row = 0; row < kRows; ++row) {
+          uint16_t hv;
+          asm volatile("ld.shared.u16 %0, [%1];" : "=h"(hv) : "r"(colbase + sw128_offset(row, chunk) + within));
+          zacc += __uint_as_float(static_cast<uint32_t>(hv) << 16);
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bPhi(s));
+    }
+    if (ok && nt > 0) {
+      ok = mbar_wait(bDone, 0, ab, kStatusTimeoutAux);
+      tc_fence_after();
+    }
+    if (ok) {
+      const uint32_t trow = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
+      float* dst = p.wsS + ((((static_cast<size_t>(c) * p.B + b) * p.H + h) * D) + r) * D;
+#pragma unroll 1
+      for (int q = 0; q < D / 32; ++q) {
+        uint32_t v[32];
+        if (nt > 0) {
+          tmem_ld32(trow + q * 32, v);
+          tmem_ld_wait();
+        } else {
+#pragma unroll
+          for (int e = 0; e < 32; ++e) v[e] = 0u;
+        }
+        float4* d4 = reinterpret_cast<float4*>(dst + q * 32);
+#pragma unroll
+        for (int e = 0; e < 8; ++e)
+          d4[e] = make_float4(__uint_as_float(v[4 * e]), __uint_as_float(v[4 * e + 1]),
+                              __uint_as_float(v[4 * e + 2]), __uint_as_float(v[4 * e + 3]));
+      }
+      p.wsz[((static_cast<size_t>(c) * p.B + b) * p.H + h) * D + r] = zacc;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 128);
+  }
+}
+
+// Exclusive scan over chunks, in place in the workspace, starting from the
+// caller's state; the caller's state leaves as the total.  One float4 per
+// thread and element, coalesced 16-byte loads and stores.
+__global__ void __launch_bounds__(256) scan_kernel(float4* __restrict__ wsS, float4* __restrict__ S, long long nS4,
+                                                   float4* __restrict__ wsz, float4* __restrict__ z, long long nz4,
+                                                   int C) {
+  const long long total = nS4 + nz4;
+  for (long long idx = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; idx < total;
+       idx += static_cast<long long>(gridDim.x) * blockDim.x) {
+    const bool isS = idx < nS4;
+    const long long e = isS ? idx : idx - nS4;
+    const long long n = isS ? nS4 : nz4;
+    float4* ws = isS ? wsS : wsz;
+    float4* st = isS ? S : z;
+    float4 run = st[e];
+    float4 nxt = C > 0 ? ws[e] : make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int c = 0; c < C; ++c) {
+      const float4 d = nxt;
+      if (c + 1 < C) nxt = ws[(c + 1) * n + e];
+      ws[c * n + e] = run;
+      run.x += d.x;
+      run.y += d.y;
+      run.z += d.z;
+      run.w += d.w;
+    }
+    st[e] = run;
+  }
+}
+
+}  // namespace hyb
+}  // namespace vattn

@@ -1,0 +1,580 @@
+// C ABI of libvattn: argument checks, TMA descriptors, launch
+// configuration.  All kernels live in this one translation unit.
+#include <cudaTypedefs.h>
+
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <string>
+#include <vector>
+
+#include "../../include/vattn.h"
+#include "attention.cuh"
+#include "hybrid.cuh"
+#include "kvcache.cuh"
+#include "rope.cuh"
+#include "selftest.cuh"
+
+// Device status word: a kernel that gives up on a bounded wait records a
+// nonzero code here (first code wins); vattn_check() reads and clears it.
+__device__ uint32_t g_vattn_status;
+
+namespace {
+
+thread_local std::string t_last_error;
+
+vattn_status fail(vattn_status s, const char* fmt, ...) __attribute__((format(printf, 2, 3)));
+vattn_status fail(vattn_status s, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  t_last_error = buf;
+  return s;
+}
+
+vattn_status cuda_fail(cudaError_t e, const char* where) {
+  return fail(VATTN_ERR_CUDA, "%s: %s", where, cudaGetErrorString(e));
+}
+
+#define VATTN_CUDA(call)                              \
+  do {                                                \
+    cudaError_t e_ = (call);                          \
+    if (e_ != cudaSuccess) return cuda_fail(e_, #call); \
+  } while (0)
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// ---------------------------------------------------------------- devices
+constexpr int kMaxDevices = 64;
+uint32_t* g_status_ptr[kMaxDevices];
+std::mutex g_mu;
+
+vattn_status current_device(int* dev) {
+  VATTN_CUDA(cudaGetDevice(dev));
+  if (*dev < 0 || *dev >= kMaxDevices) return fail(VATTN_ERR_UNSUPPORTED, "device index %d", *dev);
+  return VATTN_OK;
+}
+
+vattn_status status_ptr(uint32_t** out) {
+  int dev;
+  vattn_status st = current_device(&dev);
+  if (st) return st;
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (!g_status_ptr[dev]) {
+    void* p = nullptr;
+    VATTN_CUDA(cudaGetSymbolAddress(&p, g_vattn_status));
+    g_status_ptr[dev] = static_cast<uint32_t*>(p);
+  }
+  *out = g_status_ptr[dev];
+  return VATTN_OK;
+}
+
+// Opt a kernel into its dynamic shared memory size once per device.
+template <typename K>
+vattn_status ensure_smem(K kernel, int bytes, uint64_t* done_mask) {
+  int dev;
+  vattn_status st = current_device(&dev);
+  if (st) return st;
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (!(done_mask[dev / 64] & (1ull << (dev % 64)))) {
+    VATTN_CUDA(cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes));
+    done_mask[dev / 64] |= 1ull << (dev % 64);
+  }
+  return VATTN_OK;
+}
+
+// ------------------------------------------------------------ tensor maps
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+
+vattn_status get_encode(PFN_cuTensorMapEncodeTiled_v12000* fn) {
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (!g_encode) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    VATTN_CUDA(cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q));
+    if (q != cudaDriverEntryPointSuccess || !p)
+      return fail(VATTN_ERR_CUDA, "cuTensorMapEncodeTiled not available from the driver");
+    g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  *fn = g_encode;
+  return VATTN_OK;
+}
+
+// bf16 tensor [n3][n2][n1][d] (d innermost) as a 4-D TMA map whose box is
+// 64 channels x 1 x `rows` x 1, 128-byte swizzle, zero fill out of range.
+vattn_status make_map(CUtensorMap* m, const void* base, int d, int n1, int n2, int n3, int rows) {
+  PFN_cuTensorMapEncodeTiled_v12000 enc;
+  vattn_status st = get_encode(&enc);
+  if (st) return st;
+  const cuuint64_t dims[4] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(n1),
+                              static_cast<cuuint64_t>(n2), static_cast<cuuint64_t>(n3)};
+  const cuuint64_t strides[3] = {static_cast<cuuint64_t>(d) * 2, static_cast<cuuint64_t>(d) * 2 * n1,
+                                 static_cast<cuuint64_t>(d) * 2 * n1 * n2};
+  const cuuint32_t box[4] = {64, 1, static_cast<cuuint32_t>(rows), 1};
+  const cuuint32_t es[4] = {1, 1, 1, 1};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, es,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(VATTN_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
+  return VATTN_OK;
+}
+
+// ------------------------------------------------------------------ rope
+vattn_status check_rope(const vattn_rope* r, int d) {
+  if (!r) return fail(VATTN_ERR_INVALID_ARG, "rope is NULL");
+  if (d % 2) return fail(VATTN_ERR_INVALID_ARG, "odd head dim");
+  if (r->Hg < 1 || r->Wg < 1) return fail(VATTN_ERR_INVALID_ARG, "rope grid Hg=%d Wg=%d", r->Hg, r->Wg);
+  if (r->pairs_t < 0 || r->pairs_h < 0 || r->pairs_w < 0 || r->pairs_t + r->pairs_h + r->pairs_w != d / 2)
+    return fail(VATTN_ERR_INVALID_ARG, "rope pairs %d+%d+%d != d/2=%d", r->pairs_t, r->pairs_h, r->pairs_w,
+                d / 2);
+  if (r->max_pos < 1 || r->max_pos > (1 << 20)) return fail(VATTN_ERR_INVALID_ARG, "rope max_pos %d", r->max_pos);
+  if (r->Hg > r->max_pos || r->Wg > r->max_pos)
+    return fail(VATTN_ERR_INVALID_ARG, "rope max_pos %d smaller than the grid", r->max_pos);
+  if (!(r->theta > 0.0) || !std::isfinite(r->theta)) return fail(VATTN_ERR_INVALID_ARG, "rope theta");
+  return VATTN_OK;
+}
+
+bool supported_d(int d) { return d == 64 || d == 128; }
+
+uint64_t g_attn_smem_done[10][1];
+
+template <int D, bool ROPE, bool HYB>
+vattn_status launch_attention(const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v,
+                              const CUtensorMap& k2, const CUtensorMap& v2, const vattn::attn::Params& p,
+                              cudaStream_t s, int slot) {
+  using Cfg = vattn::attn::Cfg<D, HYB>;
+  auto kern = vattn::attn::attn_fwd_kernel<D, ROPE, HYB>;
+  vattn_status st = ensure_smem(kern, Cfg::kSmemBytes, g_attn_smem_done[slot]);
+  if (st) return st;
+  const dim3 grid(p.n_q_tiles, p.H, p.B);
+  kern<<<grid, 384, Cfg::kSmemBytes, s>>>(q, k, v, k2, v2, p);
+  VATTN_CUDA(cudaGetLastError());
+  return VATTN_OK;
+}
+
+vattn_status dispatch_attention(int d, bool rope, const CUtensorMap& q, const CUtensorMap& k,
+                                const CUtensorMap& v, const CUtensorMap& k2, const CUtensorMap& v2,
+                                const vattn::attn::Params& p, cudaStream_t s) {
+  if (d == 64) {
+    return rope ? launch_attention<64, true, false>(q, k, v, k2, v2, p, s, 0)
+                : launch_attention<64, false, false>(q, k, v, k2, v2, p, s, 1);
+  }
+  return rope ? launch_attention<128, true, false>(q, k, v, k2, v2, p, s, 2)
+              : launch_attention<128, false, false>(q, k, v, k2, v2, p, s, 3);
+}
+
+void fill_rope_params(vattn::attn::Params& p, const vattn_rope* r, const float* table) {
+  if (!r) return;
+  p.rope_tab = reinterpret_cast<const float2*>(table);
+  p.rope_Hg = r->Hg;
+  p.rope_Wg = r->Wg;
+  p.rope_pt = r->pairs_t;
+  p.rope_ph = r->pairs_h;
+  p.rope_maxpos = r->max_pos;
+}
+
+}  // namespace
+
+// ============================================================ C interface
+struct vattn_kvcache {
+  void* k_ring;
+  void* v_ring;
+  int32_t* frame_ids;
+  int capacity, B, F, Hkv, d;
+  std::vector<int32_t> host_ids;
+  CUtensorMap map_k, map_v;
+};
+
+extern "C" {
+
+const char* vattn_status_string(vattn_status s) {
+  switch (s) {
+    case VATTN_OK: return "ok";
+    case VATTN_ERR_INVALID_ARG: return "invalid argument";
+    case VATTN_ERR_UNSUPPORTED: return "unsupported";
+    case VATTN_ERR_CUDA: return "CUDA error";
+    case VATTN_ERR_TIMEOUT: return "kernel wait timed out";
+  }
+  return "unknown status";
+}
+
+const char* vattn_last_error(void) { return t_last_error.c_str(); }
+
+vattn_status vattn_check(vattn_stream stream) {
+  VATTN_CUDA(cudaStreamSynchronize(stream));
+  uint32_t v = 0;
+  VATTN_CUDA(cudaMemcpyFromSymbol(&v, g_vattn_status, sizeof(v)));
+  if (v) {
+    const uint32_t zero = 0;
+    VATTN_CUDA(cudaMemcpyToSymbol(g_vattn_status, &zero, sizeof(zero)));
+    return fail(VATTN_ERR_TIMEOUT, "a kernel gave up on a bounded wait (code %u)", v);
+  }
+  return VATTN_OK;
+}
+
+size_t vattn_rope_table_bytes(const vattn_rope* rope, int d) {
+  if (check_rope(rope, d)) return 0;
+  return static_cast<size_t>(rope->max_pos) * (d / 2) * sizeof(float2);
+}
+
+vattn_status vattn_rope_table_build(const vattn_rope* rope, int d, float* table, vattn_stream stream) {
+  if (vattn_status st = check_rope(rope, d)) return st;
+  if (!table || (reinterpret_cast<uintptr_t>(table) & 7u))
+    return fail(VATTN_ERR_INVALID_ARG, "table must be a non-NULL 8-byte aligned device pointer");
+  const int n = rope->max_pos * (d / 2);
+  vattn::rope::table_kernel<<<(n + 255) / 256, 256, 0, stream>>>(
+      reinterpret_cast<float2*>(table), rope->max_pos, d / 2, rope->pairs_t, rope->pairs_h, rope->pairs_w,
+      rope->theta);
+  VATTN_CUDA(cudaGetLastError());
+  return VATTN_OK;
+}
+
+vattn_status vattn_rope_qk(const void* q, const void* k, void* q_out, void* k_out, int B, int L, int H, int Hkv,
+                           int d, const vattn_rope* rope, const float* table, int frame_offset,
+                           vattn_stream stream) {
+  if (B < 1 || L < 1 || H < 1 || Hkv < 1) return fail(VATTN_ERR_INVALID_ARG, "sizes must be >= 1");
+  if (d < 8 || d % 8) return fail(VATTN_ERR_UNSUPPORTED, "head dim %d (multiple of 8 required)", d);
+  if (vattn_status st = check_rope(rope, d)) return st;
+  if (!table) return fail(VATTN_ERR_INVALID_ARG, "table is NULL");
+  if ((q == nullptr) != (q_out == nullptr) || (k == nullptr) != (k_out == nullptr))
+    return fail(VATTN_ERR_INVALID_ARG, "q/q_out and k/k_out must be given together");
+  if ((q && (!aligned16(q) || !aligned16(q_out))) || (k && (!aligned16(k) || !aligned16(k_out))))
+    return fail(VATTN_ERR_INVALID_ARG, "tensors must be 16-byte aligned");
+  if (frame_offset < 0) return fail(VATTN_ERR_INVALID_ARG, "frame_offset < 0");
+  const long long F = static_cast<long long>(rope->Hg) * rope->Wg;
+  if (frame_offset + (L - 1) / F >= rope->max_pos)
+    return fail(VATTN_ERR_INVALID_ARG, "frame index beyond rope max_pos");
+  vattn::rope::QKParams p{};
+  p.src[0] = static_cast<const uint4*>(q);
+  p.dst[0] = static_cast<uint4*>(q_out);
+  p.n16[0] = q ? static_cast<long long>(B) * L * H * d / 8 : 0;
+  p.src[1] = static_cast<const uint4*>(k);
+  p.dst[1] = static_cast<uint4*>(k_out);
+  p.n16[1] = k ? static_cast<long long>(B) * L * Hkv * d / 8 : 0;
+  p.heads[0] = H;
+  p.heads[1] = Hkv;
+  p.L = L;
+  p.d = d;
+  p.Hg = rope->Hg;
+  p.Wg = rope->Wg;
+  p.pt = rope->pairs_t;
+  p.ph = rope->pairs_h;
+  p.frame_offset = frame_offset;
+  p.tab = reinterpret_cast<const float2*>(table);
+  const long long total = p.n16[0] + p.n16[1];
+  if (total == 0) return VATTN_OK;
+  int sms = 148;
+  int dev;
+  if (current_device(&dev) == VATTN_OK) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const long long want = (total + 255) / 256;
+  const int blocks = static_cast<int>(want < sms * 16LL ? want : sms * 16LL);
+  vattn::rope::rope_qk_kernel<<<blocks, 256, 0, stream>>>(p);
+  VATTN_CUDA(cudaGetLastError());
+  return VATTN_OK;
+}
+
+vattn_status vattn_attention(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Lq,
+                             int Lk, int H, int Hkv, int d, float scale, vattn_mode mode, int tokens_per_frame,
+                             int chunk_frames, int window_back, int window_fwd, int q_frame_offset,
+                             int k_frame_offset, const vattn_rope* rope, const float* table,
+                             vattn_stream stream) {
+  if (!q || !k || !v || !o) return fail(VATTN_ERR_INVALID_ARG, "q, k, v, o must be non-NULL");
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o))
+    return fail(VATTN_ERR_INVALID_ARG, "q, k, v, o must be 16-byte aligned");
+  if (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)) return fail(VATTN_ERR_INVALID_ARG, "lse misaligned");
+  if (B < 1 || Lq < 1 || Lk < 1 || H < 1 || Hkv < 1) return fail(VATTN_ERR_INVALID_ARG, "sizes must be >= 1");
+  if (B > 65535 || H > 65535) return fail(VATTN_ERR_UNSUPPORTED, "B or H above 65535");
+  if (H % Hkv) return fail(VATTN_ERR_INVALID_ARG, "H=%d not a multiple of Hkv=%d", H, Hkv);
+  if (!supported_d(d)) return fail(VATTN_ERR_UNSUPPORTED, "head dim %d (64 or 128 supported)", d);
+  if (!std::isfinite(scale)) return fail(VATTN_ERR_INVALID_ARG, "scale not finite");
+  if (mode != VATTN_FULL && mode != VATTN_CHUNK_CAUSAL && mode != VATTN_SLIDING)
+    return fail(VATTN_ERR_INVALID_ARG, "mode %d", static_cast<int>(mode));
+  if (q_frame_offset < 0 || k_frame_offset < 0) return fail(VATTN_ERR_INVALID_ARG, "negative frame offset");
+  if (mode != VATTN_FULL && tokens_per_frame < 1)
+    return fail(VATTN_ERR_INVALID_ARG, "tokens_per_frame must be >= 1 for masked modes");
+  if (mode == VATTN_CHUNK_CAUSAL && chunk_frames < 1) return fail(VATTN_ERR_INVALID_ARG, "chunk_frames < 1");
+  if (mode == VATTN_SLIDING && (window_back < 0 || window_fwd < 0))
+    return fail(VATTN_ERR_INVALID_ARG, "negative window");
+  if ((rope == nullptr) != (table == nullptr)) return fail(VATTN_ERR_INVALID_ARG, "rope and table go together");
+  if (rope) {
+    if (vattn_status st = check_rope(rope, d)) return st;
+    const long long Fr = static_cast<long long>(rope->Hg) * rope->Wg;
+    if (mode != VATTN_FULL && tokens_per_frame != Fr)
+      return fail(VATTN_ERR_INVALID_ARG, "tokens_per_frame %d != Hg*Wg %lld", tokens_per_frame, Fr);
+    if (q_frame_offset + (Lq - 1) / Fr >= rope->max_pos || k_frame_offset + (Lk - 1) / Fr >= rope->max_pos)
+      return fail(VATTN_ERR_INVALID_ARG, "frame index beyond rope max_pos");
+  }
+  const int wb = window_back > (1 << 24) ? (1 << 24) : window_back;
+  const int wf = window_fwd > (1 << 24) ? (1 << 24) : window_fwd;
+
+  vattn::attn::Params p{};
+  p.o = static_cast<__nv_bfloat16*>(o);
+  p.lse = lse;
+  if (vattn_status st = status_ptr(&p.status)) return st;
+  p.B = B;
+  p.Lq = Lq;
+  p.Lk = Lk;
+  p.H = H;
+  p.Hkv = Hkv;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.mode = static_cast<int>(mode);
+  p.F = tokens_per_frame > 0 ? tokens_per_frame : 1;
+  p.chunk = chunk_frames > 0 ? chunk_frames : 1;
+  p.wb = wb;
+  p.wf = wf;
+  p.qoff = q_frame_offset;
+  p.koff = k_frame_offset;
+  p.q_seg_len = Lq;
+  p.q_tiles_per_seg = (Lq + 127) / 128;
+  p.n_q_tiles = p.q_tiles_per_seg;
+  p.reverse_q = mode == VATTN_CHUNK_CAUSAL ? 1 : 0;
+  p.n_kseg = 0;
+  fill_rope_params(p, rope, table);
+
+  CUtensorMap mq, mk, mv;
+  if (vattn_status st = make_map(&mq, q, d, H, Lq, B, 128)) return st;
+  if (vattn_status st = make_map(&mk, k, d, Hkv, Lk, B, 128)) return st;
+  if (vattn_status st = make_map(&mv, v, d, Hkv, Lk, B, 128)) return st;
+  return dispatch_attention(d, rope != nullptr, mq, mk, mv, mk, mv, p, stream);
+}
+
+// ------------------------------------------------------------- KV cache
+vattn_status vattn_kvcache_init(vattn_kvcache** cache, void* k_ring, void* v_ring, int32_t* frame_ids,
+                                int capacity, int B, int F, int Hkv, int d, vattn_stream stream) {
+  if (!cache || !k_ring || !v_ring || !frame_ids) return fail(VATTN_ERR_INVALID_ARG, "NULL pointer");
+  if (!aligned16(k_ring) || !aligned16(v_ring) || (reinterpret_cast<uintptr_t>(frame_ids) & 3u))
+    return fail(VATTN_ERR_INVALID_ARG, "ring buffers must be 16-byte aligned");
+  if (capacity < 1 || capacity > vattn::attn::kMaxKeySegments - 1)
+    return fail(VATTN_ERR_UNSUPPORTED, "capacity %d (1..%d)", capacity, vattn::attn::kMaxKeySegments - 1);
+  if (B < 1 || F < 1 || Hkv < 1) return fail(VATTN_ERR_INVALID_ARG, "sizes must be >= 1");
+  if (!supported_d(d)) return fail(VATTN_ERR_UNSUPPORTED, "head dim %d", d);
+  if (static_cast<long long>(capacity) * B > 65535) return fail(VATTN_ERR_UNSUPPORTED, "capacity*B too large");
+  vattn_kvcache* c = new vattn_kvcache();
+  c->k_ring = k_ring;
+  c->v_ring = v_ring;
+  c->frame_ids = frame_ids;
+  c->capacity = capacity;
+  c->B = B;
+  c->F = F;
+  c->Hkv = Hkv;
+  c->d = d;
+  c->host_ids.assign(capacity, -1);
+  vattn_status st = make_map(&c->map_k, k_ring, d, Hkv, F, capacity * B, 128);
+  if (!st) st = make_map(&c->map_v, v_ring, d, Hkv, F, capacity * B, 128);
+  if (st) {
+    delete c;
+    return st;
+  }
+  cudaError_t e = cudaMemsetAsync(frame_ids, 0xFF, sizeof(int32_t) * capacity, stream);
+  if (e != cudaSuccess) {
+    delete c;
+    return cuda_fail(e, "cudaMemsetAsync(frame_ids)");
+  }
+  *cache = c;
+  return VATTN_OK;
+}
+
+vattn_status vattn_kvcache_append(vattn_kvcache* c, const void* k, const void* v, int frame_idx,
+                                  vattn_stream stream) {
+  if (!c || !k || !v) return fail(VATTN_ERR_INVALID_ARG, "NULL pointer");
+  if (!aligned16(k) || !aligned16(v)) return fail(VATTN_ERR_INVALID_ARG, "k, v must be 16-byte aligned");
+  if (frame_idx < 0) return fail(VATTN_ERR_INVALID_ARG, "frame_idx < 0");
+  const int slot = frame_idx % c->capacity;
+  const long long bytes = static_cast<long long>(c->B) * c->F * c->Hkv * c->d * 2;
+  const long long n16 = bytes / 16;
+  uint4* kr = reinterpret_cast<uint4*>(static_cast<uint8_t*>(c->k_ring) + slot * bytes);
+  uint4* vr = reinterpret_cast<uint4*>(static_cast<uint8_t*>(c->v_ring) + slot * bytes);
+  int sms = 148, dev;
+  if (current_device(&dev) == VATTN_OK) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const long long want = (n16 + 255) / 256;
+  const int blocks = static_cast<int>(want < sms * 8LL ? want : sms * 8LL);
+  vattn::kv::append_kernel<<<blocks, 256, 0, stream>>>(static_cast<const uint4*>(k), static_cast<const uint4*>(v),
+                                                       kr, vr, n16, c->frame_ids, slot, frame_idx);
+  VATTN_CUDA(cudaGetLastError());
+  c->host_ids[slot] = frame_idx;
+  return VATTN_OK;
+}
+
+vattn_status vattn_attention_stream(vattn_kvcache* c, const void* q, const void* k_cur, const void* v_cur, void* o,
+                                    float* lse, int H, int frame_idx, int window_back, float scale,
+                                    const vattn_rope* rope, const float* table, vattn_stream stream) {
+  if (!c || !q || !k_cur || !v_cur || !o) return fail(VATTN_ERR_INVALID_ARG, "NULL pointer");
+  if (!aligned16(q) || !aligned16(k_cur) || !aligned16(v_cur) || !aligned16(o))
+    return fail(VATTN_ERR_INVALID_ARG, "tensors must be 16-byte aligned");
+  if (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)) return fail(VATTN_ERR_INVALID_ARG, "lse misaligned");
+  if (H < 1 || H % c->Hkv) return fail(VATTN_ERR_INVALID_ARG, "H=%d vs Hkv=%d", H, c->Hkv);
+  if (H > 65535) return fail(VATTN_ERR_UNSUPPORTED, "H above 65535");
+  if (frame_idx < 0) return fail(VATTN_ERR_INVALID_ARG, "frame_idx < 0");
+  if (window_back < 0 || window_back > c->capacity)
+    return fail(VATTN_ERR_INVALID_ARG, "window_back %d outside 0..capacity(%d)", window_back, c->capacity);
+  if (!std::isfinite(scale)) return fail(VATTN_ERR_INVALID_ARG, "scale not finite");
+  if ((rope == nullptr) != (table == nullptr)) return fail(VATTN_ERR_INVALID_ARG, "rope and table go together");
+  if (rope) {
+    if (vattn_status st = check_rope(rope, c->d)) return st;
+    if (static_cast<long long>(rope->Hg) * rope->Wg != c->F)
+      return fail(VATTN_ERR_INVALID_ARG, "rope grid Hg*Wg != frame tokens %d", c->F);
+    if (frame_idx >= rope->max_pos) return fail(VATTN_ERR_INVALID_ARG, "frame index beyond rope max_pos");
+  }
+  vattn::attn::Params p{};
+  p.o = static_cast<__nv_bfloat16*>(o);
+  p.lse = lse;
+  if (vattn_status st = status_ptr(&p.status)) return st;
+  p.B = c->B;
+  p.Lq = c->F;
+  p.Lk = c->F;
+  p.H = H;
+  p.Hkv = c->Hkv;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.mode = 0;
+  p.F = c->F;
+  p.chunk = 1;
+  p.qoff = frame_idx;
+  p.q_seg_len = c->F;
+  p.q_tiles_per_seg = (c->F + 127) / 128;
+  p.n_q_tiles = p.q_tiles_per_seg;
+  p.reverse_q = 0;
+  int n = 0, tiles = 0;
+  const int per = (c->F + 127) / 128;
+  for (int fr = frame_idx - window_back; fr < frame_idx; ++fr) {
+    if (fr < 0) continue;
+    const int slot = fr % c->capacity;
+    if (c->host_ids[slot] != fr) continue;
+    p.kseg[n] = vattn::attn::KeySegment{0, slot * c->B, 0, c->F, fr, tiles};
+    tiles += per;
+    ++n;
+  }
+  p.kseg[n] = vattn::attn::KeySegment{1, 0, 0, c->F, frame_idx, tiles};
+  ++n;
+  p.n_kseg = n;
+  fill_rope_params(p, rope, table);
+  CUtensorMap mq, mk2, mv2;
+  if (vattn_status st = make_map(&mq, q, c->d, H, c->F, c->B, 128)) return st;
+  if (vattn_status st = make_map(&mk2, k_cur, c->d, c->Hkv, c->F, c->B, 128)) return st;
+  if (vattn_status st = make_map(&mv2, v_cur, c->d, c->Hkv, c->F, c->B, 128)) return st;
+  return dispatch_attention(c->d, rope != nullptr, mq, c->map_k, c->map_v, mk2, mv2, p, stream);
+}
+
+vattn_status vattn_kvcache_frame_ids(const vattn_kvcache* c, int32_t* host_ids) {
+  if (!c || !host_ids) return fail(VATTN_ERR_INVALID_ARG, "NULL pointer");
+  std::memcpy(host_ids, c->host_ids.data(), sizeof(int32_t) * c->capacity);
+  return VATTN_OK;
+}
+
+vattn_status vattn_kvcache_restore(vattn_kvcache* c, const int32_t* host_ids) {
+  if (!c || !host_ids) return fail(VATTN_ERR_INVALID_ARG, "NULL pointer");
+  for (int i = 0; i < c->capacity; ++i)
+    if (host_ids[i] >= 0 && host_ids[i] % c->capacity != i)
+      return fail(VATTN_ERR_INVALID_ARG, "frame %d cannot sit in slot %d", host_ids[i], i);
+  std::memcpy(c->host_ids.data(), host_ids, sizeof(int32_t) * c->capacity);
+  return VATTN_OK;
+}
+
+vattn_status vattn_kvcache_destroy(vattn_kvcache* c) {
+  delete c;
+  return VATTN_OK;
+}
+
+// ---------------------------------------------------------------- hybrid
+size_t vattn_hybrid_workspace_bytes(int B, int L, int H, int d, int chunk_tokens) {
+  if (B < 1 || L < 1 || H < 1 || d < 1 || chunk_tokens < 1) return 0;
+  const size_t C = (static_cast<size_t>(L) + chunk_tokens - 1) / chunk_tokens;
+  return C * B * H * (static_cast<size_t>(d) * d + d) * sizeof(float);
+}
+
+vattn_status vattn_hybrid_chunk(const void* q, const void* k, const void* v, void* o, float* S, float* z, int B,
+                                int L, int H, int d, int chunk_tokens, float scale, void* workspace,
+                                size_t workspace_bytes, vattn_stream stream) {
+  if (!q || !k || !v || !o || !S || !z || !workspace) return fail(VATTN_ERR_INVALID_ARG, "NULL pointer");
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(S) || !aligned16(z) ||
+      !aligned16(workspace))
+    return fail(VATTN_ERR_INVALID_ARG, "pointers must be 16-byte aligned");
+  if (B < 1 || L < 1 || H < 1 || chunk_tokens < 1) return fail(VATTN_ERR_INVALID_ARG, "sizes must be >= 1");
+  if (B > 65535 || H > 65535) return fail(VATTN_ERR_UNSUPPORTED, "B or H above 65535");
+  if (d != 128) return fail(VATTN_ERR_UNSUPPORTED, "hybrid supports head dim 128 (got %d)", d);
+  if (!std::isfinite(scale)) return fail(VATTN_ERR_INVALID_ARG, "scale not finite");
+  const size_t need = vattn_hybrid_workspace_bytes(B, L, H, d, chunk_tokens);
+  if (workspace_bytes < need)
+    return fail(VATTN_ERR_INVALID_ARG, "workspace %zu bytes < %zu required", workspace_bytes, need);
+  const int C = (L + chunk_tokens - 1) / chunk_tokens;
+  if (C > 65535) return fail(VATTN_ERR_UNSUPPORTED, "more than 65535 chunks");
+  float* wsS = static_cast<float*>(workspace);
+  float* wsz = wsS + static_cast<size_t>(C) * B * H * d * d;
+  uint32_t* status;
+  if (vattn_status st = status_ptr(&status)) return st;
+
+  CUtensorMap mq, mk, mv;
+  if (vattn_status st = make_map(&mq, q, d, H, L, B, 128)) return st;
+  if (vattn_status st = make_map(&mk, k, d, H, L, B, 128)) return st;
+  if (vattn_status st = make_map(&mv, v, d, H, L, B, 128)) return st;
+
+  // (1) per-chunk state deltas
+  {
+    static uint64_t done[1];
+    auto kern = vattn::hyb::delta_kernel<128>;
+    const int smem = vattn::hyb::DeltaCfg<128>::kSmemBytes;
+    if (vattn_status st = ensure_smem(kern, smem, done)) return st;
+    vattn::hyb::DeltaParams dp{wsS, wsz, status, B, L, H, chunk_tokens};
+    kern<<<dim3(C, H, B), 256, smem, stream>>>(mk, mv, dp);
+    VATTN_CUDA(cudaGetLastError());
+  }
+  // (2) exclusive scan over chunks (+ state out)
+  {
+    const long long nS4 = static_cast<long long>(B) * H * d * d / 4, nz4 = static_cast<long long>(B) * H * d / 4;
+    int sms = 148, dev;
+    if (current_device(&dev) == VATTN_OK) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const long long want = (nS4 + nz4 + 255) / 256;
+    const int blocks = static_cast<int>(want < sms * 8LL ? want : sms * 8LL);
+    vattn::hyb::scan_kernel<<<blocks, 256, 0, stream>>>(reinterpret_cast<float4*>(wsS), reinterpret_cast<float4*>(S),
+                                                        nS4, reinterpret_cast<float4*>(wsz),
+                                                        reinterpret_cast<float4*>(z), nz4, C);
+    VATTN_CUDA(cudaGetLastError());
+  }
+  // (3) attention with linear-state initialisation
+  vattn::attn::Params p{};
+  p.o = static_cast<__nv_bfloat16*>(o);
+  p.lse = nullptr;
+  p.status = status;
+  p.B = B;
+  p.Lq = L;
+  p.Lk = L;
+  p.H = H;
+  p.Hkv = H;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.mode = vattn::attn::kSliding;   // keys = the query's own chunk
+  p.F = chunk_tokens;
+  p.chunk = 1;
+  p.wb = 0;
+  p.wf = 0;
+  p.q_seg_len = chunk_tokens;
+  p.q_tiles_per_seg = (chunk_tokens + 127) / 128;
+  p.n_q_tiles = C * p.q_tiles_per_seg;
+  p.hyb_S = wsS;
+  p.hyb_z = wsz;
+  return launch_attention<128, false, true>(mq, mk, mv, mk, mv, p, stream, 4);
+}
+
+// ------------------------------------------------------------- self-test
+// Not part of the attention interface: checks the tensor-core operand
+// layouts (see include/vattn_selftest.h).
+vattn_status vattn_selftest_umma(int variant, const void* a, const void* b, float* out, vattn_stream stream) {
+  if (variant < 0 || variant > 3) return fail(VATTN_ERR_INVALID_ARG, "variant %d", variant);
+  if (!a || !b || !out || !aligned16(a) || !aligned16(b) || !aligned16(out))
+    return fail(VATTN_ERR_INVALID_ARG, "pointers must be non-NULL and 16-byte aligned");
+  uint32_t* status;
+  if (vattn_status st = status_ptr(&status)) return st;
+  CUtensorMap ma, mb;
+  if (vattn_status st = make_map(&ma, a, 128, 1, 128, 1, 128)) return st;
+  if (vattn_status st = make_map(&mb, b, 128, 1, 128, 1, 128)) return st;
+  static uint64_t done[1];
+  const int smem = 65536 + 64 + 1024;
+  if (vattn_status st = ensure_smem(vattn::selftest::umma_kernel, smem, done)) return st;
+  vattn::selftest::umma_kernel<<<1, 128, smem, stream>>>(ma, mb, out, variant, status);
+  VATTN_CUDA(cudaGetLastError());
+  return VATTN_OK;
+}
+
+}  // extern "C"
