@@ -109,8 +109,11 @@ vattn_status vattn_rope_qk(const void* q, const void* k, void* q_out, void* k_ou
  *   the visible keys (see vattn_mode); tokens_per_frame is ignored by FULL
  *   unless rope is given.
  *   rope/table (both nullable): when given, q and k are rotated at their own
- *   (t, h, w) inside the kernel, on the shared-memory tiles, before the
- *   products; then tokens_per_frame must equal rope->Hg * rope->Wg.
+ *   (t, h, w) before the products; then tokens_per_frame must equal
+ *   rope->Hg * rope->Wg.  The query tile is rotated inside the kernel on its
+ *   shared-memory copy.  Keys: see vattn_attention_workspace_bytes.
+ *   workspace (nullable, device, 16-byte aligned) of workspace_bytes: scratch
+ *   for the rotated keys; unused without rope.
  * o = softmax(scale * q k^T restricted to visible keys) v, computed with an
  * online softmax (fp32 statistics, fp32 accumulation, bf16 P and output).
  * Tiles with no visible key are never loaded.
@@ -120,7 +123,14 @@ vattn_status vattn_attention(const void* q, const void* k, const void* v, void* 
                              vattn_mode mode, int tokens_per_frame, int chunk_frames,
                              int window_back, int window_fwd, int q_frame_offset,
                              int k_frame_offset, const vattn_rope* rope, const float* table,
-                             vattn_stream stream);
+                             void* workspace, size_t workspace_bytes, vattn_stream stream);
+
+/* Bytes of workspace that let vattn_attention rotate K once per call
+   (B * Lk * Hkv * d * 2 when rope is given, else 0).  With a workspace the
+   call writes the rotated keys there in one HBM pass and the attention
+   kernel rotates only its Q tile (once per tile); with workspace == NULL
+   the kernel also rotates every K tile it loads, in shared memory. */
+size_t vattn_attention_workspace_bytes(int B, int Lk, int Hkv, int d, const vattn_rope* rope);
 
 /*
  * Rolling KV cache of a fixed number of frames (FlashDecoder "Streaming with

@@ -53,13 +53,13 @@ def test_status_strings(lib):
 
 def test_attention_argument_checks(lib):
     att = _sig(lib, "vattn_attention", I, P, P, P, P, P, I, I, I, I, I, I, F, I, I, I, I, I, I, I, P,
-               P, P)
+               P, P, ctypes.c_size_t, P)
     good = dict(B=1, Lq=48, Lk=48, H=2, Hkv=2, d=64)
 
     def call(q=FAKE, k=FAKE, v=FAKE, o=FAKE, d=64, H=2, Hkv=2, mode=0, tpf=16, chunk=1, wb=0, wf=0,
              qoff=0, koff=0, scale=0.125):
         return att(q, k, v, o, None, 1, 48, 48, H, Hkv, d, scale, mode, tpf, chunk, wb, wf, qoff, koff,
-                   None, None, None)
+                   None, None, None, 0, None)
 
     assert call(q=None) == 1                       # NULL
     assert call(q=FAKE + 8) == 1                   # misaligned

@@ -73,7 +73,8 @@ CASES = [
 ]
 
 
-def _attention_case(va, B, T, Hg, Wg, H, Hkv, d, mode, kw, use_rope, seed=0, qoff=0, koff=0):
+def _attention_case(va, B, T, Hg, Wg, H, Hkv, d, mode, kw, use_rope, seed=0, qoff=0, koff=0,
+                    fuse_k=False):
     import torch
     F = Hg * Wg
     L = T * F
@@ -93,7 +94,8 @@ def _attention_case(va, B, T, Hg, Wg, H, Hkv, d, mode, kw, use_rope, seed=0, qof
     va.vattn_attention(to_dev(q), to_dev(k), to_dev(v), o, lse, scale=scale, mode=mode,
                        tokens_per_frame=F, chunk_frames=kw.get("chunk", 1),
                        window_back=kw.get("wb", 0), window_fwd=kw.get("wf", 0),
-                       q_frame_offset=qoff, k_frame_offset=koff, rope=rope, table=tab)
+                       q_frame_offset=qoff, k_frame_offset=koff, rope=rope, table=tab,
+                       fuse_k_rope=fuse_k)
     va.vattn_check()
     ro, rl = oracle.attention(q, k, v, scale, mode=mode, F=F, chunk=kw.get("chunk", 1),
                               wb=kw.get("wb", 0), wf=kw.get("wf", 0), q_frame_offset=qoff,
@@ -103,9 +105,12 @@ def _attention_case(va, B, T, Hg, Wg, H, Hkv, d, mode, kw, use_rope, seed=0, qof
 
 @pytest.mark.parametrize("case", CASES, ids=lambda c: "%s-d%d-T%dx%dx%d-H%d/%d%s" % (
     c[7], c[6], c[1], c[2], c[3], c[4], c[5], "-rope" if c[9] else ""))
-def test_attention_parity(va, case):
+@pytest.mark.parametrize("fuse_k", [False, True], ids=["k-prerotated", "k-fused"])
+def test_attention_parity(va, case, fuse_k):
     B, T, Hg, Wg, H, Hkv, d, mode, kw, use_rope = case
-    got, glse, ref, rlse = _attention_case(va, B, T, Hg, Wg, H, Hkv, d, mode, kw, use_rope)
+    if fuse_k and not use_rope:
+        pytest.skip("no rope")
+    got, glse, ref, rlse = _attention_case(va, B, T, Hg, Wg, H, Hkv, d, mode, kw, use_rope, fuse_k=fuse_k)
     assert_parity(got, ref, "attention %s" % (case,))
     # lse: the kernel rounds rotated q, k to bf16 before the products, which
     # moves each score by ~2e-3 rms (2^-9 relative per operand over d terms);
@@ -113,10 +118,11 @@ def test_attention_parity(va, case):
     assert np.max(np.abs(glse - rlse)) < LSE_TOL, "lse"
 
 
-def test_attention_frame_offsets(va):
+@pytest.mark.parametrize("fuse_k", [False, True])
+def test_attention_frame_offsets(va, fuse_k):
     # Offsets move the frames of queries and keys (masks and RoPE t).
     got, _, ref, _ = _attention_case(va, 1, 6, 5, 8, 2, 2, 128, "sliding", dict(wb=1, wf=0), True,
-                                     qoff=2, koff=1)
+                                     qoff=2, koff=1, fuse_k=fuse_k)
     assert_parity(got, ref, "offsets")
 
 

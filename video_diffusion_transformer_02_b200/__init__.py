@@ -73,7 +73,8 @@ _table_bytes = _sig("vattn_rope_table_bytes", _S, _RP, _I)
 _table_build = _sig("vattn_rope_table_build", _I, _RP, _I, _P, _P)
 _rope_qk = _sig("vattn_rope_qk", _I, _P, _P, _P, _P, _I, _I, _I, _I, _I, _RP, _P, _I, _P)
 _attention = _sig("vattn_attention", _I, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _I, _I, _I,
-                  _I, _I, _I, _I, _RP, _P, _P)
+                  _I, _I, _I, _I, _RP, _P, _P, _S, _P)
+_attn_ws = _sig("vattn_attention_workspace_bytes", _S, _I, _I, _I, _I, _RP)
 _kv_init = _sig("vattn_kvcache_init", _I, ctypes.POINTER(_P), _P, _P, _P, _I, _I, _I, _I, _I, _P)
 _kv_append = _sig("vattn_kvcache_append", _I, _P, _P, _P, _I, _P)
 _attention_stream = _sig("vattn_attention_stream", _I, _P, _P, _P, _P, _P, _P, _I, _I, _I, _F, _RP,
@@ -158,19 +159,35 @@ def vattn_rope_qk(q, k, q_out, k_out, rope: Rope, table, frame_offset=0, stream=
 
 
 # -------------------------------------------------------------- attention
+def vattn_attention_workspace_bytes(B, Lk, Hkv, d, rope: Rope | None) -> int:
+    return _attn_ws(B, Lk, Hkv, d, _rope_c(rope))
+
+
 def vattn_attention(q, k, v, o, lse=None, scale=None, mode="full", tokens_per_frame=0,
                     chunk_frames=1, window_back=0, window_fwd=0, q_frame_offset=0,
-                    k_frame_offset=0, rope: Rope | None = None, table=None, stream=None):
-    """o = masked softmax attention (see include/vattn.h); q/k/v/o [B, L, H, d] bf16."""
+                    k_frame_offset=0, rope: Rope | None = None, table=None, workspace=None,
+                    fuse_k_rope=False, stream=None):
+    """o = masked softmax attention (see include/vattn.h); q/k/v/o [B, L, H, d] bf16.
+
+    With rope, keys are rotated once into `workspace` (allocated here with
+    torch when not given); fuse_k_rope=True passes no workspace, so the kernel
+    rotates every K tile in shared memory instead.
+    """
     B, Lq, H, d = q.shape
     Lk, Hkv = k.shape[1], k.shape[2]
     if scale is None:
         scale = d ** -0.5
     m = MODES[mode] if isinstance(mode, str) else int(mode)
+    ws_ptr, ws_bytes = None, 0
+    if rope is not None and not fuse_k_rope:
+        need = vattn_attention_workspace_bytes(B, Lk, Hkv, d, rope)
+        if workspace is None:
+            workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+        ws_ptr, ws_bytes = _ptr(workspace), workspace.numel() * workspace.element_size()
     _ok(_attention(_bf16(q, "q"), _bf16(k, "k"), _bf16(v, "v"), _bf16(o, "o"), _ptr(lse), B, Lq, Lk,
                    H, Hkv, d, float(scale), m, tokens_per_frame, chunk_frames, window_back,
-                   window_fwd, q_frame_offset, k_frame_offset, _rope_c(rope), _ptr(table),
-                   _stream(stream)))
+                   window_fwd, q_frame_offset, k_frame_offset, _rope_c(rope), _ptr(table), ws_ptr,
+                   ws_bytes, _stream(stream)))
 
 
 # ---------------------------------------------------------------- KV ring

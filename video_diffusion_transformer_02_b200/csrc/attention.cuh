@@ -182,34 +182,53 @@ struct RopePos {
 // j of the row turns by the angle of its axis position.  Row r of a tile is
 // contiguous 64-element blocks, one per swizzle block.
 template <int D>
-__device__ __forceinline__ void rope_row_inplace(uint32_t tile, uint32_t r, RopePos pos,
-                                                 const Params& p) {
-  const float2* tab = p.rope_tab;
+__device__ __forceinline__ void rope_row_inplace(uint8_t* tile, uint32_t r, RopePos pos, const Params& p) {
+  const float2* row_t = p.rope_tab + pos.t * (D / 2);
+  const float2* row_h = p.rope_tab + pos.h * (D / 2);
+  const float2* row_w = p.rope_tab + pos.w * (D / 2);
   const int pt = p.rope_pt, pth = p.rope_pt + p.rope_ph;
-  const float2* row_t = tab + pos.t * (D / 2);
-  const float2* row_h = tab + pos.h * (D / 2);
-  const float2* row_w = tab + pos.w * (D / 2);
-#pragma unroll 4
-  for (int c16 = 0; c16 < D / 8; ++c16) {
-    const uint32_t addr = tile + (c16 >> 3) * (kTileM * 128) + sw128_offset(r, c16 & 7);
-    uint4 v = lds128(addr);
-    uint32_t w4[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const int j = c16 * 4 + e;
-      const float2* src = j < pt ? row_t : (j < pth ? row_h : row_w);
-      const float2 cs = __ldg(src + j);
-      const float x0 = bf16lo_to_f32(w4[e]), x1 = bf16hi_to_f32(w4[e]);
-      const float y0 = x0 * cs.x - x1 * cs.y;
-      const float y1 = x0 * cs.y + x1 * cs.x;
-      w4[e] = pack_bf16x2(y0, y1);
+  for (int g = 0; g < D / 32; ++g) {   // 4 chunks of 16 bytes = 16 channel pairs per group
+    uint4 v[4];
+    float2 cs[16];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int c16 = g * 4 + u;
+      v[u] = *reinterpret_cast<const uint4*>(tile + (c16 >> 3) * (kTileM * 128) + sw128_offset(r, c16 & 7));
     }
-    sts128(addr, make_uint4(w4[0], w4[1], w4[2], w4[3]));
+#pragma unroll
+    for (int e = 0; e < 16; ++e) {
+      const int j = g * 16 + e;
+      const float2* src = j < pt ? row_t : (j < pth ? row_h : row_w);
+      cs[e] = __ldg(src + j);
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      uint32_t w4[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float2 c2 = cs[u * 4 + e];
+        const float x0 = bf16lo_to_f32(w4[e]), x1 = bf16hi_to_f32(w4[e]);
+        w4[e] = pack_bf16x2(x0 * c2.x - x1 * c2.y, x0 * c2.y + x1 * c2.x);
+      }
+      const int c16 = g * 4 + u;
+      *reinterpret_cast<uint4*>(tile + (c16 >> 3) * (kTileM * 128) + sw128_offset(r, c16 & 7)) =
+          make_uint4(w4[0], w4[1], w4[2], w4[3]);
+    }
   }
 }
 
-template <int D, bool ROPE, bool HYBRID>
-__global__ void __launch_bounds__(384, 1)
+// RoPE modes: 0 none; 1 Q rotated here (softmax warpgroup, once per CTA),
+// K already rotated by the caller path; 2 Q and every K tile rotated here
+// (aux warpgroup).
+constexpr int kRopeNone = 0, kRopeQ = 1, kRopeQK = 2;
+
+__host__ __device__ constexpr int attn_threads(int rope, bool hybrid) {
+  return (rope == kRopeQK || hybrid) ? 384 : 256;
+}
+
+template <int D, int ROPE, bool HYBRID>
+__global__ void __launch_bounds__(attn_threads(ROPE, HYBRID), 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmK2,
                     const __grid_constant__ CUtensorMap tmV2, const Params p) {
@@ -353,7 +372,7 @@ __global__ void __launch_bounds__(384, 1)
           umma_commit(bPvDone);
         }
       }
-      if (ok) ok = mbar_wait(ROPE ? bQReady : bQFull, 0, ab, kStatusTimeoutMma);
+      if (ok) ok = mbar_wait(ROPE != kRopeNone ? bQReady : bQFull, 0, ab, kStatusTimeoutMma);
       tc_fence_after();
       auto issue_pv = [&](int i) -> bool {
         if (!mbar_wait(bPFull, i & 1, ab, kStatusTimeoutMma)) return false;
@@ -371,7 +390,7 @@ __global__ void __launch_bounds__(384, 1)
       };
       for (int j = 0; ok && j < nk; ++j) {
         const int s = j % NS, buf = j & 1;
-        if (!mbar_wait(ROPE ? bKReady(s) : bKFull(s), (j / NS) & 1, ab, kStatusTimeoutMma)) break;
+        if (!mbar_wait(ROPE == kRopeQK ? bKReady(s) : bKFull(s), (j / NS) & 1, ab, kStatusTimeoutMma)) break;
         if (j >= 2 && !mbar_wait(bSFree(buf), ((j - 2) >> 1) & 1, ab, kStatusTimeoutMma)) break;
         tc_fence_after();
         const uint32_t kb = sK + s * C::kTileBytes;
@@ -408,6 +427,20 @@ __global__ void __launch_bounds__(384, 1)
     const float sl2 = p.scale_log2;
     bool ok = true;
     int pv_phase = 0;   // completions of bPvDone observed so far
+    if constexpr (ROPE == kRopeQ) {
+      // rotate this thread's query row of the Q tile in place, once
+      ok = mbar_wait(bQFull, 0, ab, kStatusTimeoutSoftmax);
+      const int Fr = p.rope_Hg * p.rope_Wg;
+      RopePos pos{0, 0, 0};
+      if (row_valid) {
+        const int in = qn % Fr;
+        pos = RopePos{p.qoff + qn / Fr, in / p.rope_Wg, in % p.rope_Wg};
+      }
+      rope_row_inplace<D>(smem + C::kOffQ, r, pos, p);
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bQReady);
+    }
     if constexpr (HYBRID) {
       // phi(q_r) -> TMEM P columns (bf16); D_lin = phi(q_r) . z_c in fp32
       ok = mbar_wait(bQFull, 0, ab, kStatusTimeoutSoftmax);
@@ -459,21 +492,33 @@ __global__ void __launch_bounds__(384, 1)
         col_hi = kt.valid;
       }
       const bool masked = col_lo > 0 || col_hi < kTileN;
-      // pass 1: row max
-      float mx = -INFINITY;
+      // pass 1: row max over the visible columns (8 independent maxima)
+      float mx8[8];
 #pragma unroll
-      for (int q4 = 0; q4 < 4; ++q4) {
-        uint32_t sr[32];
-        tmem_ld32(tS + q4 * 32, sr);
-        tmem_ld_wait();
+      for (int i = 0; i < 8; ++i) mx8[i] = -INFINITY;
 #pragma unroll
-        for (int c = 0; c < 32; ++c) {
-          const int col = q4 * 32 + c;
-          const float x = __uint_as_float(sr[c]);
-          const bool vis = !masked || (col >= col_lo && col < col_hi);
-          mx = fmaxf(mx, vis ? x : -INFINITY);
+      for (int hf = 0; hf < 2; ++hf) {
+        uint32_t a[32], bb[32];
+        tmem_ld32(tS + hf * 64, a);
+        tmem_ld32(tS + hf * 64 + 32, bb);
+        tmem_ld_wait_dep2(a, bb);
+        if (!masked) {
+#pragma unroll
+          for (int c = 0; c < 32; ++c) {
+            mx8[c & 7] = fmaxf(mx8[c & 7], __uint_as_float(a[c]));
+            mx8[c & 7] = fmaxf(mx8[c & 7], __uint_as_float(bb[c]));
+          }
+        } else {
+#pragma unroll
+          for (int c = 0; c < 32; ++c) {
+            const int ca = hf * 64 + c, cb = ca + 32;
+            mx8[c & 7] = fmaxf(mx8[c & 7], (ca >= col_lo && ca < col_hi) ? __uint_as_float(a[c]) : -INFINITY);
+            mx8[c & 7] = fmaxf(mx8[c & 7], (cb >= col_lo && cb < col_hi) ? __uint_as_float(bb[c]) : -INFINITY);
+          }
         }
       }
+      const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                             fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
       const float m_tile = mx * sl2;
       const float m_new = fmaxf(m_run, m_tile);
       float factor = 1.f;
@@ -484,60 +529,87 @@ __global__ void __launch_bounds__(384, 1)
         resc = true;
       }
       const float m_use = (m_run == -INFINITY) ? 0.f : m_run;
-      // pass 2: P = exp2(s*scale*log2e - m), row sum, bf16 pack
-      uint32_t pkA[32], pkB[32];   // P columns [0, 32) and [32, 64): keys 0-63, 64-127
-      float rs = 0.f;
+      // pass 2: P = exp2(s*scale*log2e - m) in bf16, row sum in fp32.  One
+      // pair in four takes the polynomial exp2 on the FMA pipe, the rest the
+      // MUFU ex2; TMEM loads run one 32-column chunk ahead.  P is published
+      // in two halves of 64 keys; before the first half is stored, the
+      // previous P V (or the hybrid linear init) must have completed, since
+      // it reads the P columns and accumulates into O.
+      float rs4[4] = {0.f, 0.f, 0.f, 0.f};
+      uint32_t cur[32];
+      tmem_ld32(tS, cur);
+      tmem_ld_wait_dep(cur);
 #pragma unroll
-      for (int q4 = 0; q4 < 4; ++q4) {
-        uint32_t sr[32];
-        tmem_ld32(tS + q4 * 32, sr);
-        tmem_ld_wait();
+      for (int hf = 0; hf < 2; ++hf) {
+        uint32_t pk[32];
 #pragma unroll
-        for (int c = 0; c < 32; c += 2) {
-          const int col = q4 * 32 + c;
-          const bool v0 = !masked || (col >= col_lo && col < col_hi);
-          const bool v1 = !masked || (col + 1 >= col_lo && col + 1 < col_hi);
-          const float p0 = v0 ? ex2_approx(fmaf(__uint_as_float(sr[c]), sl2, -m_use)) : 0.f;
-          const float p1 = v1 ? ex2_approx(fmaf(__uint_as_float(sr[c + 1]), sl2, -m_use)) : 0.f;
-          rs += p0 + p1;
-          const uint32_t w = pack_bf16x2(p0, p1);
-          if (q4 < 2) pkA[q4 * 16 + c / 2] = w; else pkB[(q4 - 2) * 16 + c / 2] = w;
+        for (int qq = 0; qq < 2; ++qq) {
+          const int q4 = hf * 2 + qq;
+          uint32_t nxt[32];
+          if (q4 < 3) tmem_ld32(tS + (q4 + 1) * 32, nxt);
+#pragma unroll
+          for (int c = 0; c < 32; c += 2) {
+            const int col = q4 * 32 + c;
+            const float x0 = fmaf(__uint_as_float(cur[c]), sl2, -m_use);
+            const float x1 = fmaf(__uint_as_float(cur[c + 1]), sl2, -m_use);
+            float p0, p1;
+            if (((c >> 1) & 3) == 3) {
+              p0 = ex2_poly(x0);
+              p1 = ex2_poly(x1);
+            } else {
+              p0 = ex2_approx(x0);
+              p1 = ex2_approx(x1);
+            }
+            if (masked) {
+              p0 = (col >= col_lo && col < col_hi) ? p0 : 0.f;
+              p1 = (col + 1 >= col_lo && col + 1 < col_hi) ? p1 : 0.f;
+            }
+            rs4[(c >> 1) & 3] += p0 + p1;
+            pk[qq * 16 + c / 2] = pack_bf16x2(p0, p1);
+          }
+          if (q4 < 3) {
+            tmem_ld_wait_dep(nxt);
+#pragma unroll
+            for (int c = 0; c < 32; ++c) cur[c] = nxt[c];
+          }
+          if (q4 == 2) {
+            // the last S chunk is in registers: the S buffer may be rewritten
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bSFree(buf));
+          }
         }
-      }
-      // S buffer consumed
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(bSFree(buf));
-      // previous P V (or the hybrid linear init) must be complete before
-      // touching O or overwriting P
-      const int need = j + (HYBRID ? 1 : 0);   // bPvDone completions required
-      if (pv_phase < need) {
-        if (!mbar_wait(bPvDone, (need - 1) & 1, ab, kStatusTimeoutSoftmax)) {
-          ok = false;
-          break;
-        }
-        pv_phase = need;
-        tc_fence_after();
-      }
-      const bool o_valid = HYBRID || j > 0;
-      if (__any_sync(0xffffffffu, resc && o_valid)) {
-        const float f = (resc && o_valid) ? factor : 1.f;
+        if (hf == 0) {
+          const int need = j + (HYBRID ? 1 : 0);   // bPvDone completions required
+          if (pv_phase < need) {
+            if (!mbar_wait(bPvDone, (need - 1) & 1, ab, kStatusTimeoutSoftmax)) {
+              ok = false;
+            }
+            pv_phase = need;
+            tc_fence_after();
+          }
+          const bool o_valid = HYBRID || j > 0;
+          if (__any_sync(0xffffffffu, resc && o_valid)) {
+            const float f = (resc && o_valid) ? factor : 1.f;
 #pragma unroll 1
-        for (int c = 0; c < D / 32; ++c) {
-          uint32_t orr[32];
-          tmem_ld32(trow + kColO + c * 32, orr);
-          tmem_ld_wait();
+            for (int c = 0; c < D / 32; ++c) {
+              uint32_t orr[32];
+              tmem_ld32(trow + kColO + c * 32, orr);
+              tmem_ld_wait_dep(orr);
 #pragma unroll
-          for (int e = 0; e < 32; ++e) orr[e] = __float_as_uint(__uint_as_float(orr[e]) * f);
-          tmem_st32(trow + kColO + c * 32, orr);
+              for (int e = 0; e < 32; ++e) orr[e] = __float_as_uint(__uint_as_float(orr[e]) * f);
+              tmem_st32(trow + kColO + c * 32, orr);
+            }
+          }
         }
+        tmem_st32(trow + kColP + hf * 32, pk);
       }
-      tmem_st32(trow + kColP, pkA);
-      tmem_st32(trow + kColP + 32, pkB);
       tmem_st_wait();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(bPFull);
+      if (!ok) break;
+      const float rs = (rs4[0] + rs4[1]) + (rs4[2] + rs4[3]);
       l_run = l_run * factor + rs;
     }
     // epilogue: O / l -> bf16, lse
@@ -577,7 +649,7 @@ __global__ void __launch_bounds__(384, 1)
   } else if (warp >= 8) {
     // ------------------------------------------------------ aux warpgroup
     const int r = threadIdx.x - 256;
-    if constexpr (ROPE) {
+    if constexpr (ROPE == kRopeQK) {
       const int Fr = p.rope_Hg * p.rope_Wg;
       bool ok = mbar_wait(bQFull, 0, ab, kStatusTimeoutAux);
       if (ok) {
@@ -587,7 +659,7 @@ __global__ void __launch_bounds__(384, 1)
           const int in = n % Fr;
           pos = RopePos{p.qoff + n / Fr, in / p.rope_Wg, in % p.rope_Wg};
         }
-        rope_row_inplace<D>(sQ, r, pos, p);
+        rope_row_inplace<D>(smem + C::kOffQ, r, pos, p);
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) mbar_arrive(bQReady);
@@ -607,7 +679,7 @@ __global__ void __launch_bounds__(384, 1)
           const int in = kt.k0 + r;   // token index inside its frame
           pos = RopePos{kt.frame, in / p.rope_Wg, in % p.rope_Wg};
         }
-        rope_row_inplace<D>(sK + s * C::kTileBytes, r, pos, p);
+        rope_row_inplace<D>(smem + C::kOffK + s * C::kTileBytes, r, pos, p);
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) mbar_arrive(bKReady(s));

@@ -158,6 +158,22 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
 __device__ __forceinline__ void tmem_ld_wait() {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
+#define VATTN_RW8(i) "+r"(r[i]), "+r"(r[i + 1]), "+r"(r[i + 2]), "+r"(r[i + 3]), \
+                     "+r"(r[i + 4]), "+r"(r[i + 5]), "+r"(r[i + 6]), "+r"(r[i + 7])
+// Wait for this thread's TMEM loads and tie the destination registers to the
+// wait, so no use of them can be scheduled before it.
+__device__ __forceinline__ void tmem_ld_wait_dep(uint32_t (&r)[32]) {
+  asm volatile("tcgen05.wait::ld.sync.aligned;"
+               : VATTN_RW8(0), VATTN_RW8(8), VATTN_RW8(16), VATTN_RW8(24)::"memory");
+}
+__device__ __forceinline__ void tmem_ld_wait_dep2(uint32_t (&r)[32], uint32_t (&s)[32]) {
+  tmem_ld_wait_dep(r);
+  asm volatile("" : "+r"(s[0]), "+r"(s[1]), "+r"(s[2]), "+r"(s[3]), "+r"(s[4]), "+r"(s[5]), "+r"(s[6]),
+               "+r"(s[7]), "+r"(s[8]), "+r"(s[9]), "+r"(s[10]), "+r"(s[11]), "+r"(s[12]), "+r"(s[13]),
+               "+r"(s[14]), "+r"(s[15]), "+r"(s[16]), "+r"(s[17]), "+r"(s[18]), "+r"(s[19]), "+r"(s[20]),
+               "+r"(s[21]), "+r"(s[22]), "+r"(s[23]), "+r"(s[24]), "+r"(s[25]), "+r"(s[26]), "+r"(s[27]),
+               "+r"(s[28]), "+r"(s[29]), "+r"(s[30]), "+r"(s[31]));
+}
 // Warp-collective store of 32 consecutive columns (same lane mapping).
 __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
   asm volatile(
@@ -222,6 +238,18 @@ __device__ __forceinline__ void umma_commit(uint32_t bar) {
       : "memory");
 }
 
+// Per-warpgroup register budget (all four warps of a warpgroup execute the
+// same instruction).  The launch reserves threads x launch registers; the
+// decreases must free at least what the increases take.
+template <uint32_t N>
+__device__ __forceinline__ void regs_inc() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <uint32_t N>
+__device__ __forceinline__ void regs_dec() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+
 // ------------------------------------------------------------ conversions
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   uint32_t r;
@@ -230,6 +258,22 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 }
 __device__ __forceinline__ float bf16lo_to_f32(uint32_t v) { return __uint_as_float(v << 16); }
 __device__ __forceinline__ float bf16hi_to_f32(uint32_t v) { return __uint_as_float(v & 0xFFFF0000u); }
+
+// 2^x on the FMA pipe (offloads the MUFU unit): Cody-Waite reduction
+// x = j + f with j = round(x) (via the 1.5*2^23 shifter), f in [-0.5, 0.5],
+// degree-3 minimax polynomial for 2^f (max relative error 7.5e-5; the
+// coefficients come from fit_exp2_poly.py), then j added to the exponent
+// field.  Arguments below -126 return a value below 2^-126 (consumers
+// treat it as zero after bf16 rounding of the probability).
+__device__ __forceinline__ float ex2_poly(float x) {
+  x = fmaxf(x, -126.0f);
+  const float t = x + 12582912.0f;
+  const float f = x - (t - 12582912.0f);
+  float p = fmaf(5.517166853e-02f, f, 2.426111251e-01f);
+  p = fmaf(p, f, 6.932609677e-01f);
+  p = fmaf(p, f, 9.999280572e-01f);
+  return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
+}
 
 __device__ __forceinline__ float ex2_approx(float x) {
   float y;

@@ -140,31 +140,42 @@ vattn_status check_rope(const vattn_rope* r, int d) {
 
 bool supported_d(int d) { return d == 64 || d == 128; }
 
-uint64_t g_attn_smem_done[10][1];
+uint64_t g_attn_smem_done[16][1];
 
-template <int D, bool ROPE, bool HYB>
+template <int D, int ROPE, bool HYB>
 vattn_status launch_attention(const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v,
                               const CUtensorMap& k2, const CUtensorMap& v2, const vattn::attn::Params& p,
-                              cudaStream_t s, int slot) {
+                              cudaStream_t s) {
   using Cfg = vattn::attn::Cfg<D, HYB>;
+  constexpr int slot = (D == 64 ? 0 : 4) + ROPE + (HYB ? 8 : 0);
+  constexpr int threads = vattn::attn::attn_threads(ROPE, HYB);
   auto kern = vattn::attn::attn_fwd_kernel<D, ROPE, HYB>;
   vattn_status st = ensure_smem(kern, Cfg::kSmemBytes, g_attn_smem_done[slot]);
   if (st) return st;
   const dim3 grid(p.n_q_tiles, p.H, p.B);
-  kern<<<grid, 384, Cfg::kSmemBytes, s>>>(q, k, v, k2, v2, p);
+  kern<<<grid, threads, Cfg::kSmemBytes, s>>>(q, k, v, k2, v2, p);
   VATTN_CUDA(cudaGetLastError());
   return VATTN_OK;
 }
 
-vattn_status dispatch_attention(int d, bool rope, const CUtensorMap& q, const CUtensorMap& k,
+vattn_status dispatch_attention(int d, int rope_mode, const CUtensorMap& q, const CUtensorMap& k,
                                 const CUtensorMap& v, const CUtensorMap& k2, const CUtensorMap& v2,
                                 const vattn::attn::Params& p, cudaStream_t s) {
+  using namespace vattn::attn;
   if (d == 64) {
-    return rope ? launch_attention<64, true, false>(q, k, v, k2, v2, p, s, 0)
-                : launch_attention<64, false, false>(q, k, v, k2, v2, p, s, 1);
+    if (rope_mode == kRopeQK) return launch_attention<64, kRopeQK, false>(q, k, v, k2, v2, p, s);
+    if (rope_mode == kRopeQ) return launch_attention<64, kRopeQ, false>(q, k, v, k2, v2, p, s);
+    return launch_attention<64, kRopeNone, false>(q, k, v, k2, v2, p, s);
   }
-  return rope ? launch_attention<128, true, false>(q, k, v, k2, v2, p, s, 2)
-              : launch_attention<128, false, false>(q, k, v, k2, v2, p, s, 3);
+  if (rope_mode == kRopeQK) return launch_attention<128, kRopeQK, false>(q, k, v, k2, v2, p, s);
+  if (rope_mode == kRopeQ) return launch_attention<128, kRopeQ, false>(q, k, v, k2, v2, p, s);
+  return launch_attention<128, kRopeNone, false>(q, k, v, k2, v2, p, s);
+}
+
+// Rotate K once into k_out (the standalone RoPE kernel on keys only).
+vattn_status launch_rope_k(const void* k, void* k_out, int B, int L, int Hkv, int d, const vattn_rope* rope,
+                           const float* table, int frame_offset, cudaStream_t stream) {
+  return vattn_rope_qk(nullptr, k, nullptr, k_out, B, L, 1, Hkv, d, rope, table, frame_offset, stream);
 }
 
 void fill_rope_params(vattn::attn::Params& p, const vattn_rope* r, const float* table) {
@@ -277,11 +288,16 @@ vattn_status vattn_rope_qk(const void* q, const void* k, void* q_out, void* k_ou
   return VATTN_OK;
 }
 
+size_t vattn_attention_workspace_bytes(int B, int Lk, int Hkv, int d, const vattn_rope* rope) {
+  if (!rope || B < 1 || Lk < 1 || Hkv < 1 || d < 1) return 0;
+  return static_cast<size_t>(B) * Lk * Hkv * d * 2;
+}
+
 vattn_status vattn_attention(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Lq,
                              int Lk, int H, int Hkv, int d, float scale, vattn_mode mode, int tokens_per_frame,
                              int chunk_frames, int window_back, int window_fwd, int q_frame_offset,
                              int k_frame_offset, const vattn_rope* rope, const float* table,
-                             vattn_stream stream) {
+                             void* workspace, size_t workspace_bytes, vattn_stream stream) {
   if (!q || !k || !v || !o) return fail(VATTN_ERR_INVALID_ARG, "q, k, v, o must be non-NULL");
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o))
     return fail(VATTN_ERR_INVALID_ARG, "q, k, v, o must be 16-byte aligned");
@@ -307,6 +323,12 @@ vattn_status vattn_attention(const void* q, const void* k, const void* v, void* 
       return fail(VATTN_ERR_INVALID_ARG, "tokens_per_frame %d != Hg*Wg %lld", tokens_per_frame, Fr);
     if (q_frame_offset + (Lq - 1) / Fr >= rope->max_pos || k_frame_offset + (Lk - 1) / Fr >= rope->max_pos)
       return fail(VATTN_ERR_INVALID_ARG, "frame index beyond rope max_pos");
+  }
+  if (workspace) {
+    if (!aligned16(workspace)) return fail(VATTN_ERR_INVALID_ARG, "workspace must be 16-byte aligned");
+    if (rope && workspace_bytes < vattn_attention_workspace_bytes(B, Lk, Hkv, d, rope))
+      return fail(VATTN_ERR_INVALID_ARG, "workspace %zu bytes < %zu required", workspace_bytes,
+                  vattn_attention_workspace_bytes(B, Lk, Hkv, d, rope));
   }
   const int wb = window_back > (1 << 24) ? (1 << 24) : window_back;
   const int wf = window_fwd > (1 << 24) ? (1 << 24) : window_fwd;
@@ -339,7 +361,16 @@ vattn_status vattn_attention(const void* q, const void* k, const void* v, void* 
   if (vattn_status st = make_map(&mq, q, d, H, Lq, B, 128)) return st;
   if (vattn_status st = make_map(&mk, k, d, Hkv, Lk, B, 128)) return st;
   if (vattn_status st = make_map(&mv, v, d, Hkv, Lk, B, 128)) return st;
-  return dispatch_attention(d, rope != nullptr, mq, mk, mv, mk, mv, p, stream);
+    if (rope && workspace) {
+    // rotate K once into the workspace; the kernel rotates Q tiles itself
+    if (vattn_status st = launch_rope_k(k, workspace, B, Lk, Hkv, d, rope, table, k_frame_offset, stream))
+      return st;
+    CUtensorMap mkr;
+    if (vattn_status st = make_map(&mkr, workspace, d, Hkv, Lk, B, 128)) return st;
+    return dispatch_attention(d, vattn::attn::kRopeQ, mq, mkr, mv, mkr, mv, p, stream);
+  }
+  return dispatch_attention(d, rope ? vattn::attn::kRopeQK : vattn::attn::kRopeNone, mq, mk, mv, mk, mv, p,
+                            stream);
 }
 
 // ------------------------------------------------------------- KV cache
@@ -455,7 +486,8 @@ vattn_status vattn_attention_stream(vattn_kvcache* c, const void* q, const void*
   if (vattn_status st = make_map(&mq, q, c->d, H, c->F, c->B, 128)) return st;
   if (vattn_status st = make_map(&mk2, k_cur, c->d, c->Hkv, c->F, c->B, 128)) return st;
   if (vattn_status st = make_map(&mv2, v_cur, c->d, c->Hkv, c->F, c->B, 128)) return st;
-  return dispatch_attention(c->d, rope != nullptr, mq, c->map_k, c->map_v, mk2, mv2, p, stream);
+  return dispatch_attention(c->d, rope ? vattn::attn::kRopeQK : vattn::attn::kRopeNone, mq, c->map_k,
+                            c->map_v, mk2, mv2, p, stream);
 }
 
 vattn_status vattn_kvcache_frame_ids(const vattn_kvcache* c, int32_t* host_ids) {
@@ -554,7 +586,7 @@ vattn_status vattn_hybrid_chunk(const void* q, const void* k, const void* v, voi
   p.n_q_tiles = C * p.q_tiles_per_seg;
   p.hyb_S = wsS;
   p.hyb_z = wsz;
-  return launch_attention<128, false, true>(mq, mk, mv, mk, mv, p, stream, 4);
+  return launch_attention<128, vattn::attn::kRopeNone, true>(mq, mk, mv, mk, mv, p, stream);
 }
 
 // ------------------------------------------------------------- self-test
