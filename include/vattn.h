@@ -197,6 +197,34 @@ vattn_status vattn_hybrid_chunk(const void* q, const void* k, const void* v, voi
                                 float scale, void* workspace, size_t workspace_bytes,
                                 vattn_stream stream);
 
+/*
+ * vattn_hybrid_chunk without a caller workspace.  The pages have no
+ * counterpart: this entry point exists for callers that cannot call
+ * cudaMalloc — for instance plug-ins whose host application owns every
+ * device allocation, or code that runs where no allocator is reachable —
+ * and so cannot supply the scratch that vattn_hybrid_chunk needs.
+ *
+ * Same arguments and results as vattn_hybrid_chunk, minus the workspace.
+ * The scratch (per-chunk state deltas and prefixes) lives instead in one
+ * static device array of VATTN_HYBRID_NOALLOC_MAX_BYTES inside libvattn,
+ * which every GPU that loads the library holds until the process exits.
+ * The call allocates nothing.
+ *  - A shape needing more than VATTN_HYBRID_NOALLOC_MAX_BYTES of scratch
+ *    (vattn_hybrid_workspace_bytes) is rejected with VATTN_ERR_UNSUPPORTED
+ *    before anything is launched.
+ *  - The first call on a device looks up the array's device address
+ *    (cudaGetSymbolAddress) with that device current; make that first call
+ *    before any stream capture.
+ *  - All calls share the one array, which keeps the previous call's
+ *    contents; each call writes every scratch element before reading it.
+ *    Calls whose kernels overlap on the GPU (e.g. on two streams) race on
+ *    the array: order them on one stream or with events.
+ */
+#define VATTN_HYBRID_NOALLOC_MAX_BYTES ((size_t)32 << 20)
+vattn_status vattn_hybrid_chunk_noalloc(const void* q, const void* k, const void* v, void* o, float* S,
+                                        float* z, int B, int L, int H, int d, int chunk_tokens,
+                                        float scale, vattn_stream stream);
+
 /* Synchronise `stream`, then read and clear the device status word:
    VATTN_ERR_TIMEOUT if a kernel gave up on a wait since the last check. */
 vattn_status vattn_check(vattn_stream stream);

@@ -84,7 +84,9 @@ _kv_restore = _sig("vattn_kvcache_restore", _I, _P, _P)
 _kv_destroy = _sig("vattn_kvcache_destroy", _I, _P)
 _hyb_ws = _sig("vattn_hybrid_workspace_bytes", _S, _I, _I, _I, _I, _I)
 _hybrid = _sig("vattn_hybrid_chunk", _I, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _P, _S, _P)
+_hybrid_noalloc = _sig("vattn_hybrid_chunk_noalloc", _I, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _P)
 _selftest = _sig("vattn_selftest_umma", _I, _I, _P, _P, _P, _P)
+HYBRID_NOALLOC_MAX_BYTES = 32 << 20
 
 
 def status_string(status: int) -> str:
@@ -267,6 +269,17 @@ def vattn_hybrid_chunk(q, k, v, o, S, z, chunk_tokens, scale=None, workspace=Non
     _ok(_hybrid(_bf16(q, "q"), _bf16(k, "k"), _bf16(v, "v"), _bf16(o, "o"), _ptr(S), _ptr(z), B, L,
                 H, d, chunk_tokens, float(scale), _ptr(workspace), workspace.numel() * workspace.element_size(),
                 _stream(stream)))
+
+
+def vattn_hybrid_chunk_noalloc(q, k, v, o, S, z, chunk_tokens, scale=None, stream=None):
+    """vattn_hybrid_chunk for callers that cannot allocate device memory: the
+    scratch is a static array inside libvattn (HYBRID_NOALLOC_MAX_BYTES);
+    nothing is allocated here or in the library."""
+    B, L, H, d = q.shape
+    if scale is None:
+        scale = d ** -0.5
+    _ok(_hybrid_noalloc(_bf16(q, "q"), _bf16(k, "k"), _bf16(v, "v"), _bf16(o, "o"), _ptr(S), _ptr(z), B, L,
+                        H, d, chunk_tokens, float(scale), _stream(stream)))
 
 
 # ------------------------------------------------------------------ misc

@@ -589,6 +589,51 @@ vattn_status vattn_hybrid_chunk(const void* q, const void* k, const void* v, voi
   return launch_attention<128, vattn::attn::kRopeNone, true>(mq, mk, mv, mk, mv, p, stream);
 }
 
+// ------------------------------------------------- hybrid without workspace
+// Scratch of vattn_hybrid_chunk_noalloc, for callers that cannot allocate
+// device memory themselves.  The host code below must not hand the symbol
+// itself to a kernel (in host code it names a host-side stand-in); it passes
+// the device address that cudaGetSymbolAddress returns for the current
+// device.
+static __device__ __align__(256) unsigned char g_hybrid_noalloc_scratch[VATTN_HYBRID_NOALLOC_MAX_BYTES];
+
+namespace {
+void* g_noalloc_ptr[kMaxDevices];
+
+// Device address of the static scratch on the current device, looked up
+// once per device.
+vattn_status noalloc_scratch(void** out) {
+  int dev;
+  if (vattn_status st = current_device(&dev)) return st;
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (!g_noalloc_ptr[dev]) {
+    void* p = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_hybrid_noalloc_scratch);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(g_hybrid_noalloc_scratch)");
+    if (!p) return fail(VATTN_ERR_CUDA, "no device address for the static scratch");
+    g_noalloc_ptr[dev] = p;
+  }
+  *out = g_noalloc_ptr[dev];
+  return VATTN_OK;
+}
+}  // namespace
+
+vattn_status vattn_hybrid_chunk_noalloc(const void* q, const void* k, const void* v, void* o, float* S,
+                                        float* z, int B, int L, int H, int d, int chunk_tokens, float scale,
+                                        vattn_stream stream) {
+  const size_t need = vattn_hybrid_workspace_bytes(B, L, H, d, chunk_tokens);
+  if (need == 0) return fail(VATTN_ERR_INVALID_ARG, "sizes must be >= 1");
+  if (need > VATTN_HYBRID_NOALLOC_MAX_BYTES)
+    return fail(VATTN_ERR_UNSUPPORTED,
+                "this shape needs %zu bytes of scratch; the static scratch of "
+                "vattn_hybrid_chunk_noalloc holds %zu (use vattn_hybrid_chunk with a workspace)",
+                need, static_cast<size_t>(VATTN_HYBRID_NOALLOC_MAX_BYTES));
+  void* scratch = nullptr;
+  if (vattn_status st = noalloc_scratch(&scratch)) return st;
+  return vattn_hybrid_chunk(q, k, v, o, S, z, B, L, H, d, chunk_tokens, scale, scratch,
+                            VATTN_HYBRID_NOALLOC_MAX_BYTES, stream);
+}
+
 // ------------------------------------------------------------- self-test
 // Not part of the attention interface: checks the tensor-core operand
 // layouts (see include/vattn_selftest.h).
