@@ -13,12 +13,16 @@
 //   warp 0        TMA producer: Q tile once, then K tiles (multi-stage ring)
 //   warp 1        TMEM allocation + tcgen05.mma issue
 //   warp 2        TMA producer: V tiles
-//   warps 4..7    softmax warpgroup: thread r owns query row r of the tile
-//                 (TMEM lane r); scores, online softmax, P (bf16) into TMEM,
-//                 O rescale, epilogue
-//   warps 8..11   aux warpgroup: RoPE of the Q tile and of every K tile in
-//                 shared memory (ROPE), or the fp32 -> bf16 hi/lo split of
-//                 the chunk state S_c (HYBRID)
+//   warps 4..11   two softmax warpgroups: thread r of either owns query row
+//                 r of the tile (TMEM lane r); warpgroup 0 takes score
+//                 columns 0-63 of every key tile, warpgroup 1 columns 64-127
+//                 (row max exchanged in shared memory each tile, row sums
+//                 combined at the end); P (bf16) into TMEM, O rescale,
+//                 epilogue.  Warpgroup 0 also rotates the Q tile (RoPE Q
+//                 mode) or computes phi(Q) (HYBRID); warpgroup 1 splits the
+//                 chunk state S_c into bf16 hi/lo operand tiles (HYBRID).
+//   warps 12..15  (fully fused RoPE only) RoPE of the Q tile and of every K
+//                 tile in shared memory
 //
 // TMEM columns (512 allocated): S double buffer [0,128) and [128,256) fp32,
 // O [256, 256+D) fp32, P [384, 448) bf16 pairs (also phi(Q) for HYBRID).
@@ -87,7 +91,10 @@ struct Cfg {
   static constexpr int kOffBar = kOffSlo + (HYBRID ? D * D * 2 : 0);
   static constexpr int kNumBars = 2 + 5 * kStages + 4 + 2 + 2 + 1;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
-  static constexpr int kSmemBytes = kOffMisc + 64 + 1024;  // + alignment slack
+  static constexpr int kOffXchg = kOffMisc + 64;   // row max exchange [2 parities][2 wg][128] fp32
+  // The dynamic shared-memory window starts 1024-byte aligned (checked at
+  // kernel entry), so no alignment slack is reserved.
+  static constexpr int kSmemBytes = kOffXchg + 2048;
 };
 
 // Visible key range [lo, hi) of query token n (contiguous keys).  For all
@@ -187,7 +194,7 @@ __device__ __forceinline__ void rope_row_inplace(uint8_t* tile, uint32_t r, Rope
   const float2* row_h = p.rope_tab + pos.h * (D / 2);
   const float2* row_w = p.rope_tab + pos.w * (D / 2);
   const int pt = p.rope_pt, pth = p.rope_pt + p.rope_ph;
-#pragma unroll
+#pragma unroll 2
   for (int g = 0; g < D / 32; ++g) {   // 4 chunks of 16 bytes = 16 channel pairs per group
     uint4 v[4];
     float2 cs[16];
@@ -224,7 +231,7 @@ __device__ __forceinline__ void rope_row_inplace(uint8_t* tile, uint32_t r, Rope
 constexpr int kRopeNone = 0, kRopeQ = 1, kRopeQK = 2;
 
 __host__ __device__ constexpr int attn_threads(int rope, bool hybrid) {
-  return (rope == kRopeQK || hybrid) ? 384 : 256;
+  return rope == kRopeQK ? 512 : 384;
 }
 
 template <int D, int ROPE, bool HYBRID>
@@ -234,9 +241,13 @@ __global__ void __launch_bounds__(attn_threads(ROPE, HYBRID), 1)
                     const __grid_constant__ CUtensorMap tmV2, const Params p) {
   using C = Cfg<D, HYBRID>;
   constexpr int NS = C::kStages;
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = smem_raw;
   const uint32_t sbase = smem_addr(smem);
+  if (sbase & 1023u) {   // 128B-swizzled operand tiles need 1024-byte alignment
+    if (threadIdx.x == 0 && p.status) atomicCAS(p.status, 0u, kStatusSmemAlign);
+    return;
+  }
   const uint32_t sQ = sbase + C::kOffQ, sK = sbase + C::kOffK, sV = sbase + C::kOffV;
   const uint32_t sShi = sbase + C::kOffShi, sSlo = sbase + C::kOffSlo;
   const uint32_t bar0 = sbase + C::kOffBar;
@@ -277,9 +288,9 @@ __global__ void __launch_bounds__(attn_threads(ROPE, HYBRID), 1)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(bSFull(i), 1);
-      mbar_init(bSFree(i), 4);
+      mbar_init(bSFree(i), 8);
     }
-    mbar_init(bPFull, 4);
+    mbar_init(bPFull, 8);
     mbar_init(bPvDone, 1);
     mbar_init(bPhiReady, 4);
     mbar_init(bSReady, 4);
@@ -414,66 +425,102 @@ __global__ void __launch_bounds__(attn_threads(ROPE, HYBRID), 1)
       while (!mbar_try_wait(bFinal, 0) && global_timer_ns() - t0 < kWaitLimitNs) {
       }
     }
-  } else if (warp >= 4 && warp < 8) {
+  } else if (warp >= 4 && warp < 12) {
     // ---------------------------------------------------------- softmax
-    const int r = threadIdx.x - 128;                 // row of the tile = TMEM lane
+    // Two warpgroups share every row: wg 0 owns score columns [0, 64), wg 1
+    // columns [64, 128) of each 128-key tile (and the matching halves of P
+    // and of the O columns).  The row max is exchanged through shared memory
+    // once per tile; the row sums stay per warpgroup until the epilogue.
+    const int wg = (warp - 4) >> 2;
+    const int r = (threadIdx.x - 128) & 127;         // row of the tile = TMEM lane
     const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
     const uint32_t trow = tmem + lane_base;
     const int qn = g.q0 + r;
     const bool row_valid = qn < g.q_end;
     int lo = 0, hi = 0;
     if (p.n_kseg == 0) key_range(p, row_valid ? qn : g.q_end - 1, lo, hi);
+    float* xmax = reinterpret_cast<float*>(smem + C::kOffXchg);   // [2 parities][2 wg][128]
     float m_run = -INFINITY, l_run = 0.f;
     const float sl2 = p.scale_log2;
     bool ok = true;
     int pv_phase = 0;   // completions of bPvDone observed so far
     if constexpr (ROPE == kRopeQ) {
-      // rotate this thread's query row of the Q tile in place, once
-      ok = mbar_wait(bQFull, 0, ab, kStatusTimeoutSoftmax);
-      const int Fr = p.rope_Hg * p.rope_Wg;
-      RopePos pos{0, 0, 0};
-      if (row_valid) {
-        const int in = qn % Fr;
-        pos = RopePos{p.qoff + qn / Fr, in / p.rope_Wg, in % p.rope_Wg};
+      if (wg == 0) {
+        // rotate this thread's query row of the Q tile in place, once
+        ok = mbar_wait(bQFull, 0, ab, kStatusTimeoutSoftmax);
+        const int Fr = p.rope_Hg * p.rope_Wg;
+        RopePos pos{0, 0, 0};
+        if (row_valid) {
+          const int in = qn % Fr;
+          pos = RopePos{p.qoff + qn / Fr, in / p.rope_Wg, in % p.rope_Wg};
+        }
+        rope_row_inplace<D>(smem + C::kOffQ, r, pos, p);
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bQReady);
       }
-      rope_row_inplace<D>(smem + C::kOffQ, r, pos, p);
-      fence_proxy_async_smem();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(bQReady);
     }
     if constexpr (HYBRID) {
-      // phi(q_r) -> TMEM P columns (bf16); D_lin = phi(q_r) . z_c in fp32
-      ok = mbar_wait(bQFull, 0, ab, kStatusTimeoutSoftmax);
-      const int c = g.q0 / p.q_seg_len;
-      const float* zc = p.hyb_z + ((static_cast<size_t>(c) * p.B + b) * p.H + h) * D;
-      float dl = 0.f;
+      if (wg == 0) {
+        // phi(q_r) -> TMEM P columns (bf16); D_lin = phi(q_r) . z_c in fp32
+        ok = mbar_wait(bQFull, 0, ab, kStatusTimeoutSoftmax);
+        const int c = g.q0 / p.q_seg_len;
+        const float* zc = p.hyb_z + ((static_cast<size_t>(c) * p.B + b) * p.H + h) * D;
+        float dl = 0.f;
 #pragma unroll
-      for (int half = 0; half < D / 64; ++half) {
-        uint32_t pk[32];
+        for (int half = 0; half < D / 64; ++half) {
+          uint32_t pk[32];
 #pragma unroll
-        for (int c8 = 0; c8 < 8; ++c8) {
-          const uint4 v = lds128(sQ + half * (kTileM * 128) + sw128_offset(r, c8));
-          const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+          for (int c8 = 0; c8 < 8; ++c8) {
+            const uint4 v = lds128(sQ + half * (kTileM * 128) + sw128_offset(r, c8));
+            const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int ch = half * 64 + c8 * 8 + 2 * e;
-            float x0 = bf16lo_to_f32(w4[e]), x1 = bf16hi_to_f32(w4[e]);
-            x0 = x0 > 0.f ? x0 + 1.f : __expf(x0);
-            x1 = x1 > 0.f ? x1 + 1.f : __expf(x1);
-            dl = fmaf(x0, __ldg(zc + ch), dl);
-            dl = fmaf(x1, __ldg(zc + ch + 1), dl);
-            pk[c8 * 4 + e] = pack_bf16x2(x0, x1);
+            for (int e = 0; e < 4; ++e) {
+              const int ch = half * 64 + c8 * 8 + 2 * e;
+              float x0 = bf16lo_to_f32(w4[e]), x1 = bf16hi_to_f32(w4[e]);
+              x0 = x0 > 0.f ? x0 + 1.f : __expf(x0);
+              x1 = x1 > 0.f ? x1 + 1.f : __expf(x1);
+              dl = fmaf(x0, __ldg(zc + ch), dl);
+              dl = fmaf(x1, __ldg(zc + ch + 1), dl);
+              pk[c8 * 4 + e] = pack_bf16x2(x0, x1);
+            }
+          }
+          tmem_st32(trow + kColP + half * 32, pk);
+        }
+        tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bPhiReady);
+        l_run = dl;
+      } else {
+        // S_c (fp32 [D][D], row a = key feature) -> bf16 hi + lo, MN-major
+        // 128B-swizzled B operand tiles (64-column blocks of D rows).
+        const int c = g.q0 / p.q_seg_len;
+        const float* src = p.hyb_S + (((static_cast<size_t>(c) * p.B + b) * p.H + h) * D + r) * D;
+        if (r < D) {
+#pragma unroll 2
+          for (int c8 = 0; c8 < D / 8; ++c8) {
+            const float4 a0 = __ldg(reinterpret_cast<const float4*>(src + c8 * 8));
+            const float4 a1 = __ldg(reinterpret_cast<const float4*>(src + c8 * 8 + 4));
+            const float x[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+            uint32_t hi4[4], lo4[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              hi4[e] = pack_bf16x2(x[2 * e], x[2 * e + 1]);
+              lo4[e] = pack_bf16x2(x[2 * e] - bf16lo_to_f32(hi4[e]), x[2 * e + 1] - bf16hi_to_f32(hi4[e]));
+            }
+            const uint32_t off = (c8 >> 3) * (D * 128) + sw128_offset(r, c8 & 7);
+            sts128(sShi + off, make_uint4(hi4[0], hi4[1], hi4[2], hi4[3]));
+            sts128(sSlo + off, make_uint4(lo4[0], lo4[1], lo4[2], lo4[3]));
           }
         }
-        tmem_st32(trow + kColP + half * 32, pk);
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bSReady);
       }
-      tmem_st_wait();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(bPhiReady);
       m_run = 0.f;            // the linear part enters with reference max 0
-      l_run = dl;
     }
+    const int cbase = wg * 64;    // first score column of this warpgroup
     for (int j = 0; ok && j < nk; ++j) {
       const int buf = j & 1;
       if (!mbar_wait(bSFull(buf), (j >> 1) & 1, ab, kStatusTimeoutSoftmax)) {
@@ -481,44 +528,49 @@ __global__ void __launch_bounds__(attn_threads(ROPE, HYBRID), 1)
         break;
       }
       tc_fence_after();
-      const uint32_t tS = trow + (buf ? kColS1 : kColS0);
+      const uint32_t tS = trow + (buf ? kColS1 : kColS0) + cbase;
       int col_lo = 0, col_hi = kTileN;
       if (p.n_kseg == 0) {
         const int k0 = g.kbeg + j * kTileN;
-        col_lo = lo - k0;
-        col_hi = hi - k0;
+        col_lo = lo - k0 - cbase;
+        col_hi = hi - k0 - cbase;
       } else {
         const KeyTile kt = key_tile(p, g, j);
-        col_hi = kt.valid;
+        col_hi = kt.valid - cbase;
       }
-      const bool masked = col_lo > 0 || col_hi < kTileN;
-      // pass 1: row max over the visible columns (8 independent maxima)
+      const bool masked = col_lo > 0 || col_hi < 64;
+      // pass 1: max over this warpgroup's 64 visible columns
+      uint32_t a[32], bb[32];
+      tmem_ld32(tS, a);
+      tmem_ld32(tS + 32, bb);
+      tmem_ld_wait_dep2(a, bb);
       float mx8[8];
 #pragma unroll
       for (int i = 0; i < 8; ++i) mx8[i] = -INFINITY;
+      if (!masked) {
 #pragma unroll
-      for (int hf = 0; hf < 2; ++hf) {
-        uint32_t a[32], bb[32];
-        tmem_ld32(tS + hf * 64, a);
-        tmem_ld32(tS + hf * 64 + 32, bb);
-        tmem_ld_wait_dep2(a, bb);
-        if (!masked) {
+        for (int c = 0; c < 32; ++c) {
+          mx8[c & 7] = fmaxf(mx8[c & 7], __uint_as_float(a[c]));
+          mx8[c & 7] = fmaxf(mx8[c & 7], __uint_as_float(bb[c]));
+        }
+      } else {
 #pragma unroll
-          for (int c = 0; c < 32; ++c) {
-            mx8[c & 7] = fmaxf(mx8[c & 7], __uint_as_float(a[c]));
-            mx8[c & 7] = fmaxf(mx8[c & 7], __uint_as_float(bb[c]));
-          }
-        } else {
-#pragma unroll
-          for (int c = 0; c < 32; ++c) {
-            const int ca = hf * 64 + c, cb = ca + 32;
-            mx8[c & 7] = fmaxf(mx8[c & 7], (ca >= col_lo && ca < col_hi) ? __uint_as_float(a[c]) : -INFINITY);
-            mx8[c & 7] = fmaxf(mx8[c & 7], (cb >= col_lo && cb < col_hi) ? __uint_as_float(bb[c]) : -INFINITY);
-          }
+        for (int c = 0; c < 32; ++c) {
+          mx8[c & 7] = fmaxf(mx8[c & 7], (c >= col_lo && c < col_hi) ? __uint_as_float(a[c]) : -INFINITY);
+          mx8[c & 7] = fmaxf(mx8[c & 7],
+                             (c + 32 >= col_lo && c + 32 < col_hi) ? __uint_as_float(bb[c]) : -INFINITY);
         }
       }
-      const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
-                             fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+      float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                       fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+      // exchange with the other warpgroup (double-buffered by tile parity)
+      xmax[(buf * 2 + wg) * 128 + r] = mx;
+      asm volatile("bar.sync 1, 256;" ::: "memory");
+      mx = fmaxf(mx, xmax[(buf * 2 + (wg ^ 1)) * 128 + r]);
+      // the S buffer is consumed once both halves have their registers
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bSFree(buf));
       const float m_tile = mx * sl2;
       const float m_new = fmaxf(m_run, m_tile);
       float factor = 1.f;
@@ -529,104 +581,85 @@ __global__ void __launch_bounds__(attn_threads(ROPE, HYBRID), 1)
         resc = true;
       }
       const float m_use = (m_run == -INFINITY) ? 0.f : m_run;
-      // pass 2: P = exp2(s*scale*log2e - m) in bf16, row sum in fp32.  One
-      // pair in four takes the polynomial exp2 on the FMA pipe, the rest the
-      // MUFU ex2; TMEM loads run one 32-column chunk ahead.  P is published
-      // in two halves of 64 keys; before the first half is stored, the
-      // previous P V (or the hybrid linear init) must have completed, since
-      // it reads the P columns and accumulates into O.
+      // pass 2 on the registers of pass 1: P = exp2(s*scale*log2e - m), one
+      // pair in four on the FMA pipe (polynomial), the rest on MUFU ex2
+      uint32_t pk[32];
       float rs4[4] = {0.f, 0.f, 0.f, 0.f};
-      uint32_t cur[32];
-      tmem_ld32(tS, cur);
-      tmem_ld_wait_dep(cur);
 #pragma unroll
-      for (int hf = 0; hf < 2; ++hf) {
-        uint32_t pk[32];
+      for (int hq = 0; hq < 2; ++hq) {
 #pragma unroll
-        for (int qq = 0; qq < 2; ++qq) {
-          const int q4 = hf * 2 + qq;
-          uint32_t nxt[32];
-          if (q4 < 3) tmem_ld32(tS + (q4 + 1) * 32, nxt);
-#pragma unroll
-          for (int c = 0; c < 32; c += 2) {
-            const int col = q4 * 32 + c;
-            const float x0 = fmaf(__uint_as_float(cur[c]), sl2, -m_use);
-            const float x1 = fmaf(__uint_as_float(cur[c + 1]), sl2, -m_use);
-            float p0, p1;
-            if (((c >> 1) & 3) == 3) {
-              p0 = ex2_poly(x0);
-              p1 = ex2_poly(x1);
-            } else {
-              p0 = ex2_approx(x0);
-              p1 = ex2_approx(x1);
-            }
-            if (masked) {
-              p0 = (col >= col_lo && col < col_hi) ? p0 : 0.f;
-              p1 = (col + 1 >= col_lo && col + 1 < col_hi) ? p1 : 0.f;
-            }
-            rs4[(c >> 1) & 3] += p0 + p1;
-            pk[qq * 16 + c / 2] = pack_bf16x2(p0, p1);
+        for (int c = 0; c < 32; c += 2) {
+          const int col = hq * 32 + c;
+          const uint32_t u0 = hq ? bb[c] : a[c], u1 = hq ? bb[c + 1] : a[c + 1];
+          const float x0 = fmaf(__uint_as_float(u0), sl2, -m_use);
+          const float x1 = fmaf(__uint_as_float(u1), sl2, -m_use);
+          float p0, p1;
+          if (((c >> 1) & 3) == 3) {
+            p0 = ex2_poly(x0);
+            p1 = ex2_poly(x1);
+          } else {
+            p0 = ex2_approx(x0);
+            p1 = ex2_approx(x1);
           }
-          if (q4 < 3) {
-            tmem_ld_wait_dep(nxt);
-#pragma unroll
-            for (int c = 0; c < 32; ++c) cur[c] = nxt[c];
+          if (masked) {
+            p0 = (col >= col_lo && col < col_hi) ? p0 : 0.f;
+            p1 = (col + 1 >= col_lo && col + 1 < col_hi) ? p1 : 0.f;
           }
-          if (q4 == 2) {
-            // the last S chunk is in registers: the S buffer may be rewritten
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(bSFree(buf));
-          }
+          rs4[(c >> 1) & 3] += p0 + p1;
+          pk[hq * 16 + c / 2] = pack_bf16x2(p0, p1);
         }
-        if (hf == 0) {
-          const int need = j + (HYBRID ? 1 : 0);   // bPvDone completions required
-          if (pv_phase < need) {
-            if (!mbar_wait(bPvDone, (need - 1) & 1, ab, kStatusTimeoutSoftmax)) {
-              ok = false;
-            }
-            pv_phase = need;
-            tc_fence_after();
-          }
-          const bool o_valid = HYBRID || j > 0;
-          if (__any_sync(0xffffffffu, resc && o_valid)) {
-            const float f = (resc && o_valid) ? factor : 1.f;
-#pragma unroll 1
-            for (int c = 0; c < D / 32; ++c) {
-              uint32_t orr[32];
-              tmem_ld32(trow + kColO + c * 32, orr);
-              tmem_ld_wait_dep(orr);
-#pragma unroll
-              for (int e = 0; e < 32; ++e) orr[e] = __float_as_uint(__uint_as_float(orr[e]) * f);
-              tmem_st32(trow + kColO + c * 32, orr);
-            }
-          }
-        }
-        tmem_st32(trow + kColP + hf * 32, pk);
       }
+      // the previous P V (or the hybrid linear init) reads the P columns and
+      // accumulates into O: it must be complete before either is touched
+      const int need = j + (HYBRID ? 1 : 0);   // bPvDone completions required
+      if (pv_phase < need) {
+        if (!mbar_wait(bPvDone, (need - 1) & 1, ab, kStatusTimeoutSoftmax)) ok = false;
+        pv_phase = need;
+        tc_fence_after();
+      }
+      const bool o_valid = HYBRID || j > 0;
+      if (__any_sync(0xffffffffu, resc && o_valid)) {
+        const float f = (resc && o_valid) ? factor : 1.f;
+#pragma unroll 1
+        for (int c = wg * (D / 64); c < (wg + 1) * (D / 64); ++c) {
+          uint32_t orr[32];
+          tmem_ld32(trow + kColO + c * 32, orr);
+          tmem_ld_wait_dep(orr);
+#pragma unroll
+          for (int e = 0; e < 32; ++e) orr[e] = __float_as_uint(__uint_as_float(orr[e]) * f);
+          tmem_st32(trow + kColO + c * 32, orr);
+        }
+      }
+      tmem_st32(trow + kColP + wg * 32, pk);
       tmem_st_wait();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(bPFull);
       if (!ok) break;
-      const float rs = (rs4[0] + rs4[1]) + (rs4[2] + rs4[3]);
-      l_run = l_run * factor + rs;
+      l_run = l_run * factor + ((rs4[0] + rs4[1]) + (rs4[2] + rs4[3]));
     }
-    // epilogue: O / l -> bf16, lse
+    // epilogue: O / l -> bf16 (each warpgroup writes its half of the
+    // columns), lse from warpgroup 0
     const int need = nk + (HYBRID ? 1 : 0);
     if (ok && need > 0 && pv_phase < need) {
       ok = mbar_wait(bPvDone, (need - 1) & 1, ab, kStatusTimeoutSoftmax);
       tc_fence_after();
     }
+    // row sums through the exchange slot of parity nk & 1: its last reads
+    // (tile nk - 2) finished before the barrier of tile nk - 1
+    float* xl = reinterpret_cast<float*>(smem + C::kOffXchg) + (nk & 1) * 256;   // [2 wg][128]
+    xl[wg * 128 + r] = l_run;
+    asm volatile("bar.sync 1, 256;" ::: "memory");
+    const float l_all = l_run + xl[(wg ^ 1) * 128 + r];
     if (ok) {
-      const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
+      const float inv = l_all > 0.f ? 1.f / l_all : 0.f;
       __nv_bfloat16* orow = p.o + ((static_cast<size_t>(b) * p.Lq + qn) * p.H + h) * D;
 #pragma unroll 1
-      for (int c = 0; c < D / 32; ++c) {
+      for (int c = wg * (D / 64); c < (wg + 1) * (D / 64); ++c) {
         uint32_t orr[32];
         if (need > 0) {
           tmem_ld32(trow + kColO + c * 32, orr);
-          tmem_ld_wait();
+          tmem_ld_wait_dep(orr);
         } else {
 #pragma unroll
           for (int e = 0; e < 32; ++e) orr[e] = 0u;
@@ -641,14 +674,15 @@ __global__ void __launch_bounds__(attn_threads(ROPE, HYBRID), 1)
           for (int e = 0; e < 4; ++e) dst[e] = make_uint4(w[4 * e], w[4 * e + 1], w[4 * e + 2], w[4 * e + 3]);
         }
       }
-      if (p.lse && row_valid) {
-        const float lse = l_run > 0.f ? (m_run + __log2f(l_run)) * 0.69314718055994531f : -INFINITY;
+      if (wg == 0 && p.lse && row_valid) {
+        const float lse = l_all > 0.f ? (m_run + __log2f(l_all)) * 0.69314718055994531f : -INFINITY;
         p.lse[(static_cast<size_t>(b) * p.H + h) * p.Lq + qn] = lse;
       }
     }
-  } else if (warp >= 8) {
+  } else if (warp >= 12) {
     // ------------------------------------------------------ aux warpgroup
-    const int r = threadIdx.x - 256;
+    // RoPE of the Q tile and of every K tile, in shared memory, in place.
+    const int r = threadIdx.x - 384;
     if constexpr (ROPE == kRopeQK) {
       const int Fr = p.rope_Hg * p.rope_Wg;
       bool ok = mbar_wait(bQFull, 0, ab, kStatusTimeoutAux);
@@ -684,31 +718,6 @@ __global__ void __launch_bounds__(attn_threads(ROPE, HYBRID), 1)
         __syncwarp();
         if (lane == 0) mbar_arrive(bKReady(s));
       }
-    } else if constexpr (HYBRID) {
-      // S_c (fp32 [D][D], row a = key feature) -> bf16 hi + lo, MN-major
-      // 128B-swizzled B operand tiles (64-column blocks of D rows).
-      const int c = g.q0 / p.q_seg_len;
-      const float* src = p.hyb_S + (((static_cast<size_t>(c) * p.B + b) * p.H + h) * D + r) * D;
-      if (r < D) {
-#pragma unroll 2
-        for (int c8 = 0; c8 < D / 8; ++c8) {
-          const float4 a0 = __ldg(reinterpret_cast<const float4*>(src + c8 * 8));
-          const float4 a1 = __ldg(reinterpret_cast<const float4*>(src + c8 * 8 + 4));
-          const float x[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
-          uint32_t hi4[4], lo4[4];
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            hi4[e] = pack_bf16x2(x[2 * e], x[2 * e + 1]);
-            lo4[e] = pack_bf16x2(x[2 * e] - bf16lo_to_f32(hi4[e]), x[2 * e + 1] - bf16hi_to_f32(hi4[e]));
-          }
-          const uint32_t off = (c8 >> 3) * (D * 128) + sw128_offset(r, c8 & 7);
-          sts128(sShi + off, make_uint4(hi4[0], hi4[1], hi4[2], hi4[3]));
-          sts128(sSlo + off, make_uint4(lo4[0], lo4[1], lo4[2], lo4[3]));
-        }
-      }
-      fence_proxy_async_smem();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(bSReady);
     }
   }
 

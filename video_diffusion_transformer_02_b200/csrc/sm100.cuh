@@ -20,6 +20,7 @@ enum : uint32_t {
   kStatusTimeoutMma = 2,
   kStatusTimeoutSoftmax = 3,
   kStatusTimeoutAux = 4,
+  kStatusSmemAlign = 5,   // dynamic shared memory not 1024-byte aligned
 };
 // Wall-clock bound of a single wait (nanoseconds of %globaltimer).
 constexpr uint64_t kWaitLimitNs = 2000000000ull;

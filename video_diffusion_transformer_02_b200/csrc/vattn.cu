@@ -222,6 +222,8 @@ vattn_status vattn_check(vattn_stream stream) {
   if (v) {
     const uint32_t zero = 0;
     VATTN_CUDA(cudaMemcpyToSymbol(g_vattn_status, &zero, sizeof(zero)));
+    if (v == vattn::sm100::kStatusSmemAlign)
+      return fail(VATTN_ERR_CUDA, "dynamic shared memory was not 1024-byte aligned; the kernel did not run");
     return fail(VATTN_ERR_TIMEOUT, "a kernel gave up on a bounded wait (code %u)", v);
   }
   return VATTN_OK;
