@@ -45,6 +45,27 @@ constexpr uint32_t kTmemCols = 512;
 // units): stale maxima keep every exp2 argument below it, so fp32 stays
 // far from overflow while most tiles skip the O correction.
 constexpr float kRescaleThreshold = 8.0f;
+// Which of every 8 consecutive score pairs take the FMA-pipe polynomial
+// exp2 instead of MUFU ex2 (bit i set: pair i mod 8).  At head dim 128 the
+// MUFU keeps pace with the tensor core and the polynomial only adds issue
+// pressure; at head dim 64 the MMA work per score halves and a quarter of
+// the exponentials move to the FMA pipe (measured on B200).
+template <int D>
+struct PolyMask {
+  static constexpr uint32_t value = D == 64 ? 0x88u : 0x00u;
+};
+// Packed fp32x2 arithmetic for the scale-and-subtract and the row sums.
+#define VATTN_PACKED_FP32 1
+// Poll back-off (ns) of the waits of the TMA producers and of the MMA thread.
+#ifndef VATTN_SLEEP_PROD
+#define VATTN_SLEEP_PROD 0
+#endif
+#ifndef VATTN_SLEEP_MMA
+#define VATTN_SLEEP_MMA 0
+#endif
+#ifndef VATTN_SLEEP_SOFT
+#define VATTN_SLEEP_SOFT 0
+#endif
 
 enum Mode : int { kFull = 0, kChunkCausal = 1, kSliding = 2 };
 
@@ -322,7 +343,7 @@ __global__ void __launch_bounds__(attn_threads(ROPE, HYBRID), 1)
       int j = 0;
       for (; j < nk; ++j) {
         const int s = j % NS;
-        if (j >= NS && !mbar_wait(bKEmpty(s), ((j / NS) - 1) & 1, ab, kStatusTimeoutProducer)) break;
+        if (j >= NS && !mbar_wait(bKEmpty(s), ((j / NS) - 1) & 1, ab, kStatusTimeoutProducer, VATTN_SLEEP_PROD)) break;
         const KeyTile kt = key_tile(p, g, j);
         const CUtensorMap* m = kt.map ? &tmK2 : &tmK;
         mbar_arrive_expect_tx(bKFull(s), C::kTileBytes);
@@ -347,7 +368,7 @@ __global__ void __launch_bounds__(attn_threads(ROPE, HYBRID), 1)
       int j = 0;
       for (; j < nk; ++j) {
         const int s = j % NS;
-        if (j >= NS && !mbar_wait(bVEmpty(s), ((j / NS) - 1) & 1, ab, kStatusTimeoutProducer)) break;
+        if (j >= NS && !mbar_wait(bVEmpty(s), ((j / NS) - 1) & 1, ab, kStatusTimeoutProducer, VATTN_SLEEP_PROD)) break;
         const KeyTile kt = key_tile(p, g, j);
         const CUtensorMap* m = kt.map ? &tmV2 : &tmV;
         mbar_arrive_expect_tx(bVFull(s), C::kTileBytes);
@@ -386,39 +407,58 @@ __global__ void __launch_bounds__(attn_threads(ROPE, HYBRID), 1)
       if (ok) ok = mbar_wait(ROPE != kRopeNone ? bQReady : bQFull, 0, ab, kStatusTimeoutMma);
       tc_fence_after();
       auto issue_pv = [&](int i) -> bool {
-        if (!mbar_wait(bPFull, i & 1, ab, kStatusTimeoutMma)) return false;
+        if (!mbar_wait(bPFull, i & 1, ab, kStatusTimeoutMma, VATTN_SLEEP_MMA)) return false;
         const int s = i % NS;
-        if (!mbar_wait(bVFull(s), (i / NS) & 1, ab, kStatusTimeoutMma)) return false;
+        if (!mbar_wait(bVFull(s), (i / NS) & 1, ab, kStatusTimeoutMma, VATTN_SLEEP_MMA)) return false;
         tc_fence_after();
-        const uint32_t vb = sV + s * C::kTileBytes;
+        const uint64_t dVs = sdesc_sw128(sV + s * C::kTileBytes, kTileM * 128, 1024);
 #pragma unroll
         for (int kk = 0; kk < kTileN / 16; ++kk)
-          umma_ts(tO, tP + kk * 8, sdesc_sw128(vb + kk * 2048, kTileM * 128, 1024), idPV,
+          umma_ts(tO, tP + kk * 8, dVs + static_cast<uint64_t>(kk * (2048 >> 4)), idPV,
                   (HYBRID || i > 0 || kk > 0) ? 1u : 0u);
         umma_commit(bPvDone);
         umma_commit(bVEmpty(s));
         return true;
       };
-      for (int j = 0; ok && j < nk; ++j) {
-        const int s = j % NS, buf = j & 1;
-        if (!mbar_wait(ROPE == kRopeQK ? bKReady(s) : bKFull(s), (j / NS) & 1, ab, kStatusTimeoutMma)) break;
-        if (j >= 2 && !mbar_wait(bSFree(buf), ((j - 2) >> 1) & 1, ab, kStatusTimeoutMma)) break;
+      // shared-memory descriptors, built once: the start-address field
+      // (address >> 4, 14 bits) is advanced by adding (offset >> 4) to the
+      // low word, which cannot carry past the field (shared memory < 256 KB)
+      const uint64_t dQ = sdesc_sw128(sQ, 16, 1024);
+      const uint64_t dK = sdesc_sw128(sK, 16, 1024);
+      // S = Q K^T for tile t into S buffer t & 1; it needs K tile t and the
+      // buffer's previous tile (t - 2) consumed by the softmax, which is
+      // signalled right after that tile's row max, long before its P.
+      auto issue_qk = [&](int t) -> bool {
+        const int s = t % NS, buf = t & 1;
+        if (!mbar_wait(ROPE == kRopeQK ? bKReady(s) : bKFull(s), (t / NS) & 1, ab, kStatusTimeoutMma,
+                       VATTN_SLEEP_MMA))
+          return false;
+        if (t >= 2 && !mbar_wait(bSFree(buf), ((t - 2) >> 1) & 1, ab, kStatusTimeoutMma, VATTN_SLEEP_MMA))
+          return false;
         tc_fence_after();
-        const uint32_t kb = sK + s * C::kTileBytes;
+        const uint64_t dKs = dK + static_cast<uint64_t>((s * C::kTileBytes) >> 4);
         const uint32_t tS = tmem + (buf ? kColS1 : kColS0);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * (kTileM * 128) + (kk & 3) * 32;
-          umma_ss(tS, sdesc_sw128(sQ + off, 16, 1024), sdesc_sw128(kb + off, 16, 1024), idQK, kk > 0);
+          const uint32_t off = ((kk >> 2) * (kTileM * 128) + (kk & 3) * 32) >> 4;
+          umma_ss(tS, dQ + off, dKs + off, idQK, kk > 0);
         }
         umma_commit(bSFull(buf));
         umma_commit(bKEmpty(s));
-        if (j >= 1 && !issue_pv(j - 1)) {
+        return true;
+      };
+      // issue order: QK(0), QK(1), then per tile j: QK(j + 2), PV(j)
+      for (int t = 0; ok && t < 2 && t < nk; ++t) ok = issue_qk(t);
+      for (int j = 0; ok && j < nk; ++j) {
+        if (j + 2 < nk && !issue_qk(j + 2)) {
+          ok = false;
+          break;
+        }
+        if (!issue_pv(j)) {
           ok = false;
           break;
         }
       }
-      if (ok && nk > 0) issue_pv(nk - 1);
       // all issued MMAs complete before teardown
       umma_commit(bFinal);
       const uint64_t t0 = global_timer_ns();
@@ -523,7 +563,7 @@ __global__ void __launch_bounds__(attn_threads(ROPE, HYBRID), 1)
     const int cbase = wg * 64;    // first score column of this warpgroup
     for (int j = 0; ok && j < nk; ++j) {
       const int buf = j & 1;
-      if (!mbar_wait(bSFull(buf), (j >> 1) & 1, ab, kStatusTimeoutSoftmax)) {
+      if (!mbar_wait(bSFull(buf), (j >> 1) & 1, ab, kStatusTimeoutSoftmax, VATTN_SLEEP_SOFT)) {
         ok = false;
         break;
       }
@@ -549,10 +589,8 @@ __global__ void __launch_bounds__(attn_threads(ROPE, HYBRID), 1)
       for (int i = 0; i < 8; ++i) mx8[i] = -INFINITY;
       if (!masked) {
 #pragma unroll
-        for (int c = 0; c < 32; ++c) {
-          mx8[c & 7] = fmaxf(mx8[c & 7], __uint_as_float(a[c]));
-          mx8[c & 7] = fmaxf(mx8[c & 7], __uint_as_float(bb[c]));
-        }
+        for (int c = 0; c < 32; ++c)
+          mx8[c & 7] = fmax3(mx8[c & 7], __uint_as_float(a[c]), __uint_as_float(bb[c]));
       } else {
 #pragma unroll
         for (int c = 0; c < 32; ++c) {
@@ -581,39 +619,65 @@ __global__ void __launch_bounds__(attn_threads(ROPE, HYBRID), 1)
         resc = true;
       }
       const float m_use = (m_run == -INFINITY) ? 0.f : m_run;
-      // pass 2 on the registers of pass 1: P = exp2(s*scale*log2e - m), one
-      // pair in four on the FMA pipe (polynomial), the rest on MUFU ex2
+      // pass 2 on the registers of pass 1: P = exp2(s*scale*log2e - m) on the
+      // MUFU ex2; scale-and-subtract and the row sum run as packed fp32x2.
+      // Unmasked tiles (all but the edges of a key range) take a loop with
+      // no per-element visibility test.
       uint32_t pk[32];
-      float rs4[4] = {0.f, 0.f, 0.f, 0.f};
+      float rs2[4][2] = {{0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}};
+      const float nm = -m_use;
+      if (!masked) {
 #pragma unroll
-      for (int hq = 0; hq < 2; ++hq) {
+        for (int hq = 0; hq < 2; ++hq) {
 #pragma unroll
-        for (int c = 0; c < 32; c += 2) {
-          const int col = hq * 32 + c;
-          const uint32_t u0 = hq ? bb[c] : a[c], u1 = hq ? bb[c + 1] : a[c + 1];
-          const float x0 = fmaf(__uint_as_float(u0), sl2, -m_use);
-          const float x1 = fmaf(__uint_as_float(u1), sl2, -m_use);
-          float p0, p1;
-          if (((c >> 1) & 3) == 3) {
-            p0 = ex2_poly(x0);
-            p1 = ex2_poly(x1);
-          } else {
-            p0 = ex2_approx(x0);
-            p1 = ex2_approx(x1);
+          for (int c = 0; c < 32; c += 2) {
+            const uint32_t u0 = hq ? bb[c] : a[c], u1 = hq ? bb[c + 1] : a[c + 1];
+            float x0, x1, p0, p1;
+#if VATTN_PACKED_FP32
+            ffma2(x0, x1, __uint_as_float(u0), __uint_as_float(u1), sl2, sl2, nm, nm);
+#else
+            x0 = fmaf(__uint_as_float(u0), sl2, nm);
+            x1 = fmaf(__uint_as_float(u1), sl2, nm);
+#endif
+            if ((PolyMask<D>::value >> ((c >> 1) & 7)) & 1u) {
+              ex2_poly2(p0, p1, x0, x1);
+            } else {
+              p0 = ex2_approx(x0);
+              p1 = ex2_approx(x1);
+            }
+#if VATTN_PACKED_FP32
+            fadd2(rs2[(c >> 1) & 3][0], rs2[(c >> 1) & 3][1], p0, p1);
+#else
+            rs2[(c >> 1) & 3][0] += p0;
+            rs2[(c >> 1) & 3][1] += p1;
+#endif
+            pk[hq * 16 + c / 2] = pack_bf16x2(p0, p1);
           }
-          if (masked) {
+        }
+      } else {
+#pragma unroll
+        for (int hq = 0; hq < 2; ++hq) {
+#pragma unroll
+          for (int c = 0; c < 32; c += 2) {
+            const int col = hq * 32 + c;
+            const uint32_t u0 = hq ? bb[c] : a[c], u1 = hq ? bb[c + 1] : a[c + 1];
+            float p0 = ex2_approx(fmaf(__uint_as_float(u0), sl2, nm));
+            float p1 = ex2_approx(fmaf(__uint_as_float(u1), sl2, nm));
             p0 = (col >= col_lo && col < col_hi) ? p0 : 0.f;
             p1 = (col + 1 >= col_lo && col + 1 < col_hi) ? p1 : 0.f;
+            rs2[(c >> 1) & 3][0] += p0;
+            rs2[(c >> 1) & 3][1] += p1;
+            pk[hq * 16 + c / 2] = pack_bf16x2(p0, p1);
           }
-          rs4[(c >> 1) & 3] += p0 + p1;
-          pk[hq * 16 + c / 2] = pack_bf16x2(p0, p1);
         }
       }
+      const float rs = ((rs2[0][0] + rs2[0][1]) + (rs2[1][0] + rs2[1][1])) +
+                       ((rs2[2][0] + rs2[2][1]) + (rs2[3][0] + rs2[3][1]));
       // the previous P V (or the hybrid linear init) reads the P columns and
       // accumulates into O: it must be complete before either is touched
       const int need = j + (HYBRID ? 1 : 0);   // bPvDone completions required
       if (pv_phase < need) {
-        if (!mbar_wait(bPvDone, (need - 1) & 1, ab, kStatusTimeoutSoftmax)) ok = false;
+        if (!mbar_wait(bPvDone, (need - 1) & 1, ab, kStatusTimeoutSoftmax, VATTN_SLEEP_SOFT)) ok = false;
         pv_phase = need;
         tc_fence_after();
       }
@@ -636,7 +700,7 @@ __global__ void __launch_bounds__(attn_threads(ROPE, HYBRID), 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(bPFull);
       if (!ok) break;
-      l_run = l_run * factor + ((rs4[0] + rs4[1]) + (rs4[2] + rs4[3]));
+      l_run = l_run * factor + rs;
     }
     // epilogue: O / l -> bf16 (each warpgroup writes its half of the
     // columns), lse from warpgroup 0

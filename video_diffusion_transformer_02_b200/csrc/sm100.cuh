@@ -77,12 +77,15 @@ __device__ __forceinline__ void raise_abort(const Abort& ab, uint32_t code) {
 
 // Wait until phase `parity` of `bar` has completed.  Returns false if the
 // CTA aborted or the wait exceeded kWaitLimitNs (then the abort is raised
-// with `code`).
+// with `code`).  sleep_ns > 0 backs off between polls (for threads whose
+// reaction time matters less than the issue slots their polling would take
+// from warps sharing the sub-partition).
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, const Abort& ab,
-                                          uint32_t code) {
+                                          uint32_t code, uint32_t sleep_ns = 0) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_timer_ns();
   for (uint32_t it = 1;; ++it) {
+    if (sleep_ns) __nanosleep(sleep_ns);
     if (mbar_try_wait(bar, parity)) return true;
     if ((it & 63u) == 0u) {
       if (*ab.flag) return false;
@@ -251,6 +254,31 @@ __device__ __forceinline__ void regs_dec() {
   asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
 }
 
+// --------------------------------------------------- packed fp32 / 3-input
+// d = a * b + c on two lanes at once (fma.rn.f32x2).
+__device__ __forceinline__ void ffma2(float& d0, float& d1, float a0, float a1, float b0, float b1, float c0,
+                                      float c1) {
+  asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\tmov.b64 rc, {%6, %7};\n\t"
+      "fma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d0), "=f"(d1)
+      : "f"(a0), "f"(a1), "f"(b0), "f"(b1), "f"(c0), "f"(c1));
+}
+// (d0, d1) += (a0, a1) with add.rn.f32x2.
+__device__ __forceinline__ void fadd2(float& d0, float& d1, float a0, float a1) {
+  asm("{\n\t.reg .b64 ra, rd;\n\t"
+      "mov.b64 rd, {%0, %1};\n\tmov.b64 ra, {%2, %3};\n\t"
+      "add.rn.f32x2 rd, rd, ra;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "+f"(d0), "+f"(d1)
+      : "f"(a0), "f"(a1));
+}
+// max of three fp32 values (one instruction).
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
 // ------------------------------------------------------------ conversions
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   uint32_t r;
@@ -274,6 +302,23 @@ __device__ __forceinline__ float ex2_poly(float x) {
   p = fmaf(p, f, 6.932609677e-01f);
   p = fmaf(p, f, 9.999280572e-01f);
   return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
+}
+
+// Two lanes of ex2_poly with packed fp32x2 arithmetic: the same reduction,
+// polynomial and exponent insertion (exponent added with an integer
+// multiply-add of j * 2^23 onto the polynomial's bits).
+__device__ __forceinline__ void ex2_poly2(float& y0, float& y1, float x0, float x1) {
+  x0 = fmaxf(x0, -126.0f);
+  x1 = fmaxf(x1, -126.0f);
+  float t0, t1, j0, j1, f0, f1, p0, p1;
+  ffma2(t0, t1, x0, x1, 1.0f, 1.0f, 12582912.0f, 12582912.0f);     // x + 1.5*2^23
+  ffma2(j0, j1, t0, t1, 1.0f, 1.0f, -12582912.0f, -12582912.0f);   // round(x)
+  ffma2(f0, f1, j0, j1, -1.0f, -1.0f, x0, x1);                     // x - round(x)
+  ffma2(p0, p1, f0, f1, 5.517166853e-02f, 5.517166853e-02f, 2.426111251e-01f, 2.426111251e-01f);
+  ffma2(p0, p1, p0, p1, f0, f1, 6.932609677e-01f, 6.932609677e-01f);
+  ffma2(p0, p1, p0, p1, f0, f1, 9.999280572e-01f, 9.999280572e-01f);
+  y0 = __int_as_float(__float_as_int(t0) * (1 << 23) + __float_as_int(p0));
+  y1 = __int_as_float(__float_as_int(t1) * (1 << 23) + __float_as_int(p1));
 }
 
 __device__ __forceinline__ float ex2_approx(float x) {
