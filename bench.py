@@ -135,6 +135,24 @@ class ClockSampler:
                 "reasons": sorted(reasons)}
 
 
+# ------------------------------------------------------------ multi-rank
+def reduce_max(value: float, world: int, device=None) -> float:
+    """Max over ranks of a per-rank device time (every rank calls it)."""
+    if world <= 1:
+        return value
+    import torch
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_tflops(flops_per_step: float, steps: int, world: int, max_total_ms: float) -> float:
+    """Whole-job throughput: every rank runs its own replica of the step
+    (weak scaling), so the job does world * steps steps in the slowest
+    rank's time."""
+    return world * flops_per_step * steps / (max_total_ms / 1e3) / 1e12
+
+
 # -------------------------------------------------------------- workloads
 def wan13b_workload(va, torch, device):
     c = si.CONFIGS["wan13b"]
@@ -195,12 +213,9 @@ def run_ours(args, rank, world, device):
     step_ms = [a.elapsed_time(b) for a, b in evs]
     total_ms = float(sum(step_ms))
     rope_ms = _time_events(torch, rope_k_only, args.steps, flush)
-    if world > 1:
-        t = torch.tensor([total_ms], dtype=torch.float64, device=device)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = reduce_max(total_ms, world, device)
     ms_per_step = total_ms / args.steps
-    value = world * w["flops"] * args.steps / (total_ms / 1e3) / 1e12
+    value = job_tflops(w["flops"], args.steps, world, total_ms)
     # two launches per step: the key rotation (HBM pass) and the attention
     # kernel; the attention kernel's duration is the step minus the rotation
     # pass timed alone on the same stream
@@ -231,10 +246,7 @@ def run_ours(args, rank, world, device):
     e1.record(stream)
     torch.cuda.synchronize()
     e2e_ms = e0.elapsed_time(e1) / e_steps
-    if world > 1:
-        t = torch.tensor([e2e_ms], dtype=torch.float64, device=device)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = reduce_max(e2e_ms, world, device)
     h2d = 3 * w["q"].numel() * 2
     d2h = w["o"].numel() * 2
 
@@ -319,6 +331,7 @@ def secondary_measurements(va, torch, device, flush):
     cache = va.KVCache(kr, vr, ids)
     rope = va.Rope(Hg=c["Hg"], Wg=c["Wg"], pairs=c["pairs"], max_pos=64)
     tab = va.rope_table(rope, d, device=device)
+    cache.enable_rope(torch.zeros((cap + 1, 1, F, H, d), dtype=torch.bfloat16, device=device), rope, tab)
     of = torch.empty((1, F, H, d), dtype=torch.bfloat16, device=device)
     frames = [(qd[f].unsqueeze(0), kd[f].unsqueeze(0), vd[f].unsqueeze(0)) for f in range(T)]
 
@@ -338,7 +351,7 @@ def secondary_measurements(va, torch, device, flush):
     app = lambda: cache.append(frames[5][1], frames[5][2], 5)
     app()
     ms_app = _time_events(torch, lambda: [app() for _ in range(16)], 3) / 16
-    app_bytes = 2 * 2 * F * H * d * 2
+    app_bytes = (2 + 3) * F * H * d * 2    # read k, v; write raw k, v and rotated k
     out["stream"] = {"frames_per_s": T / (ms / 1e3), "ms_per_frame": ms / T, "tflops": total_flops / ms * 1e-9,
                      "steady_attention_ms": ms_att,
                      "steady_attention_tflops": 4.0 * d * F * F * H * 5 / ms_att * 1e-9,

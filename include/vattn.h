@@ -168,8 +168,25 @@ vattn_status vattn_attention_stream(vattn_kvcache* cache, const void* q, const v
 /* Copy the host mirror of frame_ids (capacity entries) into host_ids. */
 vattn_status vattn_kvcache_frame_ids(const vattn_kvcache* cache, int32_t* host_ids);
 /* After the caller restored ring and frame_ids contents (checkpoint /
-   resume), set the host mirror to host_ids (capacity entries). */
-vattn_status vattn_kvcache_restore(vattn_kvcache* cache, const int32_t* host_ids);
+   resume), set the host mirror to host_ids (capacity entries); with a
+   rotated-key ring, the restored frames' keys are rotated again on
+   `stream`. */
+vattn_status vattn_kvcache_restore(vattn_kvcache* cache, const int32_t* host_ids, vattn_stream stream);
+/*
+ * Keep a second, rotated copy of the keys so that each frame's keys are
+ * rotated once, at their absolute frame index, instead of once per query
+ * tile that reads them (FlashDecoder applies RoPE with precomputed tables,
+ * "Inference Optimization", Sec. 4.6).  k_ring_rot: caller-owned bf16
+ * [capacity + 1][B][F][Hkv][d]; frame f's rotated keys live in slot
+ * f % (capacity + 1).  From then on vattn_kvcache_append writes the raw copy
+ * and the rotated copy in one pass, and vattn_attention_stream (which must
+ * then be given the same rope and table) rotates the current frame's keys
+ * into the spare slot and reads rotated keys only.  Frames already in the
+ * ring are rotated now, on `stream`.  The raw ring stays the exact input
+ * bytes.
+ */
+vattn_status vattn_kvcache_enable_rope(vattn_kvcache* cache, void* k_ring_rot, const vattn_rope* rope,
+                                       const float* table, vattn_stream stream);
 vattn_status vattn_kvcache_destroy(vattn_kvcache* cache);
 
 /*

@@ -60,6 +60,7 @@ def test_stream_config_sampled_rows(va):
     vr = torch.zeros_like(kr)
     ids = torch.zeros(cap, dtype=torch.int32, device="cuda")
     cache = va.KVCache(kr, vr, ids)
+    cache.enable_rope(torch.zeros((cap + 1, 1, F, H, d), dtype=torch.bfloat16, device="cuda"), rope, tab)
     o = torch.full(qd.shape, float("nan"), dtype=torch.bfloat16, device="cuda")
     for f in range(T):
         sl = slice(f * F, (f + 1) * F)

@@ -16,7 +16,7 @@ def va():
     return va
 
 
-def _run_stream(va, q, k, v, F, H, Hkv, d, cap, wb, rope, tab, check_ring=None):
+def _run_stream(va, q, k, v, F, H, Hkv, d, cap, wb, rope, tab, check_ring=None, rot_ring=False):
     """Frame-by-frame decode through the ring; returns o [B, L, H, d]."""
     import torch
     B, L = q.shape[0], q.shape[1]
@@ -25,6 +25,8 @@ def _run_stream(va, q, k, v, F, H, Hkv, d, cap, wb, rope, tab, check_ring=None):
     vr = torch.zeros_like(kr)
     ids = torch.zeros(cap, dtype=torch.int32, device="cuda")
     cache = va.KVCache(kr, vr, ids)
+    if rot_ring:
+        cache.enable_rope(torch.zeros((cap + 1, B, F, Hkv, d), dtype=torch.bfloat16, device="cuda"), rope, tab)
     qd, kd, vd = to_dev(q), to_dev(k), to_dev(v)
     o = torch.full((B, L, H, d), float("nan"), dtype=torch.bfloat16, device="cuda")
     for f in range(T):
@@ -41,7 +43,8 @@ def _run_stream(va, q, k, v, F, H, Hkv, d, cap, wb, rope, tab, check_ring=None):
     return o
 
 
-def test_stream_small_with_ring_bit_exact(va):
+@pytest.mark.parametrize("rot_ring", [False, True], ids=["k-fused", "k-rotated-ring"])
+def test_stream_small_with_ring_bit_exact(va, rot_ring):
     T, Hg, Wg, H, d, cap, wb = 9, 5, 30, 2, 64, 4, 4     # F = 150: ragged frame tiles
     F = Hg * Wg
     L = T * F
@@ -59,7 +62,7 @@ def test_stream_small_with_ring_bit_exact(va):
         assert np.array_equal(bits_of(vr), ev), "V ring differs after frame %d" % f
         assert list(ids.cpu().numpy()) == list(eids) == cache.host_frame_ids()
 
-    o = _run_stream(va, q, k, v, F, H, H, d, cap, wb, rope, tab, check_ring)
+    o = _run_stream(va, q, k, v, F, H, H, d, cap, wb, rope, tab, check_ring, rot_ring=rot_ring)
     ref, _ = oracle.stream(q, k, v, F, d ** -0.5, wb, rope=dict(Hg=Hg, Wg=Wg, pairs=(12, 10, 10),
                                                                   theta=1e4))
     assert_parity(from_dev(o), ref, "stream")
@@ -142,3 +145,77 @@ def test_hybrid_state_resume(va):
     got = np.concatenate([from_dev(o1), from_dev(o2)], axis=1)
     assert_parity(got, ro, "resumed hybrid")
     assert_parity(S.cpu().numpy(), rS, "resumed S", max_abs=np.inf)
+
+
+def test_rotated_ring_contents(va):
+    # The rotated-key ring holds each frame's keys rotated at its absolute
+    # frame: within one bf16 ulp of the exact rotation.
+    import torch
+    T, Hg, Wg, H, d, cap = 6, 4, 32, 2, 64, 4
+    F = Hg * Wg
+    k = si.normal_bf16(81, (1, T * F, H, d))
+    v = si.normal_bf16(82, (1, T * F, H, d))
+    rope = va.Rope(Hg=Hg, Wg=Wg, pairs=(12, 10, 10), max_pos=64)
+    tab = va.rope_table(rope, d)
+    kr = torch.zeros((cap, 1, F, H, d), dtype=torch.bfloat16, device="cuda")
+    cache = va.KVCache(kr, torch.zeros_like(kr), torch.zeros(cap, dtype=torch.int32, device="cuda"))
+    rot = torch.zeros((cap + 1, 1, F, H, d), dtype=torch.bfloat16, device="cuda")
+    cache.enable_rope(rot, rope, tab)
+    kd, vd = to_dev(k), to_dev(v)
+    for f in range(T):
+        cache.append(kd[:, f * F:(f + 1) * F].contiguous(), vd[:, f * F:(f + 1) * F].contiguous(), f)
+    va.vattn_check()
+    exact = oracle.rope(k, Hg, Wg, (12, 10, 10), 1e4)
+    for f in range(T - cap - 1 + 1, T):
+        got = from_dev(rot[f % (cap + 1)])[0]
+        ref = exact[0, f * F:(f + 1) * F]
+        assert np.all(np.abs(got - ref) <= np.abs(ref) * 2.0 ** -8 + 1e-6), "frame %d" % f
+    cache.close()
+
+
+def test_stream_checkpoint_resume(va):
+    # Decode frames 0..k-1, copy the ring out, restore it into a fresh cache
+    # and continue: outputs and ring contents equal an unsplit run.
+    import torch
+    T, Hg, Wg, H, d, cap, wb, split = 9, 5, 30, 2, 64, 4, 4, 5
+    F = Hg * Wg
+    q = si.normal_bf16(91, (1, T * F, H, d))
+    k = si.normal_bf16(92, (1, T * F, H, d))
+    v = si.normal_bf16(93, (1, T * F, H, d))
+    rope = va.Rope(Hg=Hg, Wg=Wg, pairs=(12, 10, 10), max_pos=64)
+    tab = va.rope_table(rope, d)
+    qd, kd, vd = to_dev(q), to_dev(k), to_dev(v)
+
+    def new_cache():
+        kr = torch.zeros((cap, 1, F, H, d), dtype=torch.bfloat16, device="cuda")
+        c = va.KVCache(kr, torch.zeros_like(kr), torch.zeros(cap, dtype=torch.int32, device="cuda"))
+        c.enable_rope(torch.zeros((cap + 1, 1, F, H, d), dtype=torch.bfloat16, device="cuda"), rope, tab)
+        return c
+
+    def step(c, f):
+        sl = slice(f * F, (f + 1) * F)
+        of = torch.empty((1, F, H, d), dtype=torch.bfloat16, device="cuda")
+        c.attend(qd[:, sl].contiguous(), kd[:, sl].contiguous(), vd[:, sl].contiguous(), of, f, wb,
+                 rope=rope, table=tab)
+        c.append(kd[:, sl].contiguous(), vd[:, sl].contiguous(), f)
+        return of
+
+    a = new_cache()
+    full = [step(a, f) for f in range(T)]
+    b = new_cache()
+    first = [step(b, f) for f in range(split)]
+    saved = (b.k_ring.clone(), b.v_ring.clone(), b.frame_ids.clone(), b.host_frame_ids())
+    b.close()
+    c = new_cache()
+    c.k_ring.copy_(saved[0])
+    c.v_ring.copy_(saved[1])
+    c.frame_ids.copy_(saved[2])
+    c.restore(saved[3])
+    rest = [step(c, f) for f in range(split, T)]
+    va.vattn_check()
+    for f, (x, y) in enumerate(zip(full, first + rest)):
+        assert torch.equal(x, y), "frame %d differs after resume" % f
+    assert torch.equal(a.k_ring, c.k_ring) and torch.equal(a.v_ring, c.v_ring)
+    assert a.host_frame_ids() == c.host_frame_ids()
+    a.close()
+    c.close()

@@ -80,7 +80,8 @@ _kv_append = _sig("vattn_kvcache_append", _I, _P, _P, _P, _I, _P)
 _attention_stream = _sig("vattn_attention_stream", _I, _P, _P, _P, _P, _P, _P, _I, _I, _I, _F, _RP,
                          _P, _P)
 _kv_ids = _sig("vattn_kvcache_frame_ids", _I, _P, _P)
-_kv_restore = _sig("vattn_kvcache_restore", _I, _P, _P)
+_kv_restore = _sig("vattn_kvcache_restore", _I, _P, _P, _P)
+_kv_rope = _sig("vattn_kvcache_enable_rope", _I, _P, _P, _RP, _P, _P)
 _kv_destroy = _sig("vattn_kvcache_destroy", _I, _P)
 _hyb_ws = _sig("vattn_hybrid_workspace_bytes", _S, _I, _I, _I, _I, _I)
 _hybrid = _sig("vattn_hybrid_chunk", _I, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _P, _S, _P)
@@ -223,9 +224,15 @@ class KVCache:
         _ok(_kv_ids(self._h, arr))
         return list(arr)
 
-    def restore(self, host_ids):
+    def restore(self, host_ids, stream=None):
         arr = (ctypes.c_int32 * self.capacity)(*host_ids)
-        _ok(_kv_restore(self._h, arr))
+        _ok(_kv_restore(self._h, arr, _stream(stream)))
+
+    def enable_rope(self, k_ring_rot, rope: Rope, table, stream=None):
+        """Rotated-key ring (bf16 [capacity + 1, B, F, Hkv, d]): keys rotated once per frame."""
+        self.k_ring_rot = k_ring_rot
+        _ok(_kv_rope(self._h, _bf16(k_ring_rot, "k_ring_rot"), ctypes.byref(rope.c()), _ptr(table),
+                     _stream(stream)))
 
     def close(self):
         if getattr(self, "_h", None):

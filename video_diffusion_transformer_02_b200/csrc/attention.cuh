@@ -70,8 +70,10 @@ struct PolyMask {
 enum Mode : int { kFull = 0, kChunkCausal = 1, kSliding = 2 };
 
 struct KeySegment {
-  int map;      // 0: k/v maps, 1: k2/v2 maps
-  int c3_base;  // fourth TMA coordinate = c3_base + batch index
+  int kmap;     // K source: 0 = tmK, 1 = tmK2
+  int kc3;      // K fourth TMA coordinate = kc3 + batch index
+  int vmap;     // V source: 0 = tmV, 1 = tmV2
+  int vc3;      // V fourth TMA coordinate = vc3 + batch index
   int tok0;     // first token of the segment along the token axis
   int n_tok;    // tokens in the segment
   int frame;    // absolute frame index (RoPE t of every key in it)
@@ -172,7 +174,8 @@ __device__ __forceinline__ TileGeom tile_geom(const Params& p, int qt) {
 }
 
 struct KeyTile {
-  int map, c3, k0;    // TMA source: map, 4th coordinate (minus batch), token start
+  int kmap, kc3, vmap, vc3;   // TMA sources and 4th coordinates (minus batch)
+  int k0;             // token start
   int valid;          // keys in this tile that exist (segment mode)
   int frame;          // segment frame (segment mode)
 };
@@ -180,8 +183,8 @@ struct KeyTile {
 __device__ __forceinline__ KeyTile key_tile(const Params& p, const TileGeom& g, int j) {
   KeyTile kt;
   if (p.n_kseg == 0) {
-    kt.map = 0;
-    kt.c3 = 0;
+    kt.kmap = kt.vmap = 0;
+    kt.kc3 = kt.vc3 = 0;
     kt.k0 = g.kbeg + j * kTileN;
     kt.valid = min(kTileN, g.kend - kt.k0);
     kt.frame = 0;
@@ -192,8 +195,10 @@ __device__ __forceinline__ KeyTile key_tile(const Params& p, const TileGeom& g, 
       if (p.kseg[i].tile0 <= j) s = i;
     const KeySegment& sg = p.kseg[s];
     const int t = j - sg.tile0;
-    kt.map = sg.map;
-    kt.c3 = sg.c3_base;
+    kt.kmap = sg.kmap;
+    kt.kc3 = sg.kc3;
+    kt.vmap = sg.vmap;
+    kt.vc3 = sg.vc3;
     kt.k0 = sg.tok0 + t * kTileN;
     kt.valid = min(kTileN, sg.n_tok - t * kTileN);
     kt.frame = sg.frame;
@@ -345,12 +350,12 @@ __global__ void __launch_bounds__(attn_threads(ROPE, HYBRID), 1)
         const int s = j % NS;
         if (j >= NS && !mbar_wait(bKEmpty(s), ((j / NS) - 1) & 1, ab, kStatusTimeoutProducer, VATTN_SLEEP_PROD)) break;
         const KeyTile kt = key_tile(p, g, j);
-        const CUtensorMap* m = kt.map ? &tmK2 : &tmK;
+        const CUtensorMap* m = kt.kmap ? &tmK2 : &tmK;
         mbar_arrive_expect_tx(bKFull(s), C::kTileBytes);
 #pragma unroll
         for (int blk = 0; blk < C::kBlocks; ++blk)
           tma_load_4d(sK + s * C::kTileBytes + blk * (kTileM * 128), m, bKFull(s), blk * 64, kvh, kt.k0,
-                      kt.c3 + b);
+                      kt.kc3 + b);
       }
       // drain: wait until every load issued so far has landed
       for (int i = max(0, j - NS); i < j; ++i) {
@@ -370,12 +375,12 @@ __global__ void __launch_bounds__(attn_threads(ROPE, HYBRID), 1)
         const int s = j % NS;
         if (j >= NS && !mbar_wait(bVEmpty(s), ((j / NS) - 1) & 1, ab, kStatusTimeoutProducer, VATTN_SLEEP_PROD)) break;
         const KeyTile kt = key_tile(p, g, j);
-        const CUtensorMap* m = kt.map ? &tmV2 : &tmV;
+        const CUtensorMap* m = kt.vmap ? &tmV2 : &tmV;
         mbar_arrive_expect_tx(bVFull(s), C::kTileBytes);
 #pragma unroll
         for (int blk = 0; blk < C::kBlocks; ++blk)
           tma_load_4d(sV + s * C::kTileBytes + blk * (kTileM * 128), m, bVFull(s), blk * 64, kvh, kt.k0,
-                      kt.c3 + b);
+                      kt.vc3 + b);
       }
       for (int i = max(0, j - NS); i < j; ++i) {
         const uint64_t t0 = global_timer_ns();

@@ -198,7 +198,51 @@ struct vattn_kvcache {
   int capacity, B, F, Hkv, d;
   std::vector<int32_t> host_ids;
   CUtensorMap map_k, map_v;
+  // optional rotated-key ring: capacity + 1 slots, frame f in slot f % (capacity + 1)
+  void* k_rot = nullptr;
+  vattn_rope rope{};
+  const float* table = nullptr;
+  CUtensorMap map_krot;
 };
+
+namespace {
+size_t frame_bytes(const vattn_kvcache* c) { return static_cast<size_t>(c->B) * c->F * c->Hkv * c->d * 2; }
+
+// Launch the append / rotate pass for one frame.  kr/vr null: rotate only.
+vattn_status launch_append_rope(const vattn_kvcache* c, const void* k, const void* v, void* kr, void* vr,
+                                int32_t* ids, int slot, int frame, cudaStream_t stream) {
+  vattn::kv::AppendRopeParams p{};
+  p.k = static_cast<const uint4*>(k);
+  p.v = static_cast<const uint4*>(v);
+  p.kr = static_cast<uint4*>(kr);
+  p.vr = static_cast<uint4*>(vr);
+  p.krot = reinterpret_cast<uint4*>(static_cast<uint8_t*>(c->k_rot) +
+                                    static_cast<size_t>(frame % (c->capacity + 1)) * frame_bytes(c));
+  p.n16 = static_cast<long long>(frame_bytes(c) / 16);
+  p.ids = ids;
+  p.slot = slot;
+  p.frame = frame;
+  p.F = c->F;
+  p.Hkv = c->Hkv;
+  p.d = c->d;
+  p.Wg = c->rope.Wg;
+  p.pt = c->rope.pairs_t;
+  p.ph = c->rope.pairs_h;
+  p.tab = reinterpret_cast<const float2*>(c->table);
+  int sms = 148, dev;
+  if (current_device(&dev) == VATTN_OK) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const long long want = (p.n16 + 255) / 256;
+  const int blocks = static_cast<int>(want < sms * 8LL ? want : sms * 8LL);
+  vattn::kv::append_rope_kernel<<<blocks, 256, 0, stream>>>(p);
+  VATTN_CUDA(cudaGetLastError());
+  return VATTN_OK;
+}
+
+bool same_rope(const vattn_rope& a, const vattn_rope& b) {
+  return a.Hg == b.Hg && a.Wg == b.Wg && a.pairs_t == b.pairs_t && a.pairs_h == b.pairs_h &&
+         a.pairs_w == b.pairs_w && a.theta == b.theta && a.max_pos == b.max_pos;
+}
+}  // namespace
 
 extern "C" {
 
@@ -421,6 +465,12 @@ vattn_status vattn_kvcache_append(vattn_kvcache* c, const void* k, const void* v
   const long long n16 = bytes / 16;
   uint4* kr = reinterpret_cast<uint4*>(static_cast<uint8_t*>(c->k_ring) + slot * bytes);
   uint4* vr = reinterpret_cast<uint4*>(static_cast<uint8_t*>(c->v_ring) + slot * bytes);
+  if (c->k_rot) {
+    if (frame_idx >= c->rope.max_pos) return fail(VATTN_ERR_INVALID_ARG, "frame index beyond rope max_pos");
+    if (vattn_status st = launch_append_rope(c, k, v, kr, vr, c->frame_ids, slot, frame_idx, stream)) return st;
+    c->host_ids[slot] = frame_idx;
+    return VATTN_OK;
+  }
   int sms = 148, dev;
   if (current_device(&dev) == VATTN_OK) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const long long want = (n16 + 255) / 256;
@@ -470,17 +520,34 @@ vattn_status vattn_attention_stream(vattn_kvcache* c, const void* q, const void*
   p.q_tiles_per_seg = (c->F + 127) / 128;
   p.n_q_tiles = p.q_tiles_per_seg;
   p.reverse_q = 0;
+  // Keys come from the rotated-key ring (rotated once per frame) when the
+  // cache has one and the call rotates; otherwise from the raw ring, rotated
+  // tile by tile in the kernel when rope is given.
+  const bool rot_ring = rope && c->k_rot;
+  if (rot_ring) {
+    if (!same_rope(*rope, c->rope) || table != c->table)
+      return fail(VATTN_ERR_INVALID_ARG, "rope/table differ from those given to vattn_kvcache_enable_rope");
+    // the current frame's rotated keys: slot frame_idx % (capacity + 1),
+    // which holds a frame outside the window
+    if (vattn_status st = launch_append_rope(c, k_cur, v_cur, nullptr, nullptr, nullptr, 0, frame_idx, stream))
+      return st;
+  }
   int n = 0, tiles = 0;
   const int per = (c->F + 127) / 128;
+  const int rcap = c->capacity + 1;
   for (int fr = frame_idx - window_back; fr < frame_idx; ++fr) {
     if (fr < 0) continue;
     const int slot = fr % c->capacity;
     if (c->host_ids[slot] != fr) continue;
-    p.kseg[n] = vattn::attn::KeySegment{0, slot * c->B, 0, c->F, fr, tiles};
+    const int kc3 = rot_ring ? (fr % rcap) * c->B : slot * c->B;
+    p.kseg[n] = vattn::attn::KeySegment{0, kc3, 0, slot * c->B, 0, c->F, fr, tiles};
     tiles += per;
     ++n;
   }
-  p.kseg[n] = vattn::attn::KeySegment{1, 0, 0, c->F, frame_idx, tiles};
+  if (rot_ring)
+    p.kseg[n] = vattn::attn::KeySegment{0, (frame_idx % rcap) * c->B, 1, 0, 0, c->F, frame_idx, tiles};
+  else
+    p.kseg[n] = vattn::attn::KeySegment{1, 0, 1, 0, 0, c->F, frame_idx, tiles};
   ++n;
   p.n_kseg = n;
   fill_rope_params(p, rope, table);
@@ -488,6 +555,8 @@ vattn_status vattn_attention_stream(vattn_kvcache* c, const void* q, const void*
   if (vattn_status st = make_map(&mq, q, c->d, H, c->F, c->B, 128)) return st;
   if (vattn_status st = make_map(&mk2, k_cur, c->d, c->Hkv, c->F, c->B, 128)) return st;
   if (vattn_status st = make_map(&mv2, v_cur, c->d, c->Hkv, c->F, c->B, 128)) return st;
+  if (rot_ring)
+    return dispatch_attention(c->d, vattn::attn::kRopeQ, mq, c->map_krot, c->map_v, c->map_krot, mv2, p, stream);
   return dispatch_attention(c->d, rope ? vattn::attn::kRopeQK : vattn::attn::kRopeNone, mq, c->map_k,
                             c->map_v, mk2, mv2, p, stream);
 }
@@ -498,13 +567,48 @@ vattn_status vattn_kvcache_frame_ids(const vattn_kvcache* c, int32_t* host_ids) 
   return VATTN_OK;
 }
 
-vattn_status vattn_kvcache_restore(vattn_kvcache* c, const int32_t* host_ids) {
+namespace {
+// Rotate every frame present in the raw ring into the rotated-key ring.
+vattn_status rerotate_present(vattn_kvcache* c, cudaStream_t stream) {
+  const size_t bytes = frame_bytes(c);
+  for (int i = 0; i < c->capacity; ++i) {
+    const int fr = c->host_ids[i];
+    if (fr < 0) continue;
+    if (fr >= c->rope.max_pos) return fail(VATTN_ERR_INVALID_ARG, "frame %d beyond rope max_pos", fr);
+    const uint8_t* kraw = static_cast<const uint8_t*>(c->k_ring) + static_cast<size_t>(i) * bytes;
+    const uint8_t* vraw = static_cast<const uint8_t*>(c->v_ring) + static_cast<size_t>(i) * bytes;
+    if (vattn_status st = launch_append_rope(c, kraw, vraw, nullptr, nullptr, nullptr, 0, fr, stream)) return st;
+  }
+  return VATTN_OK;
+}
+}  // namespace
+
+vattn_status vattn_kvcache_restore(vattn_kvcache* c, const int32_t* host_ids, vattn_stream stream) {
   if (!c || !host_ids) return fail(VATTN_ERR_INVALID_ARG, "NULL pointer");
   for (int i = 0; i < c->capacity; ++i)
     if (host_ids[i] >= 0 && host_ids[i] % c->capacity != i)
       return fail(VATTN_ERR_INVALID_ARG, "frame %d cannot sit in slot %d", host_ids[i], i);
   std::memcpy(c->host_ids.data(), host_ids, sizeof(int32_t) * c->capacity);
+  if (c->k_rot) return rerotate_present(c, stream);
   return VATTN_OK;
+}
+
+vattn_status vattn_kvcache_enable_rope(vattn_kvcache* c, void* k_ring_rot, const vattn_rope* rope,
+                                       const float* table, vattn_stream stream) {
+  if (!c || !k_ring_rot || !table) return fail(VATTN_ERR_INVALID_ARG, "NULL pointer");
+  if (!aligned16(k_ring_rot)) return fail(VATTN_ERR_INVALID_ARG, "k_ring_rot must be 16-byte aligned");
+  if (vattn_status st = check_rope(rope, c->d)) return st;
+  if (static_cast<long long>(rope->Hg) * rope->Wg != c->F)
+    return fail(VATTN_ERR_INVALID_ARG, "rope grid Hg*Wg != frame tokens %d", c->F);
+  if (static_cast<long long>(c->capacity + 1) * c->B > 65535)
+    return fail(VATTN_ERR_UNSUPPORTED, "(capacity+1)*B too large");
+  CUtensorMap m;
+  if (vattn_status st = make_map(&m, k_ring_rot, c->d, c->Hkv, c->F, (c->capacity + 1) * c->B, 128)) return st;
+  c->k_rot = k_ring_rot;
+  c->rope = *rope;
+  c->table = table;
+  c->map_krot = m;
+  return rerotate_present(c, stream);
 }
 
 vattn_status vattn_kvcache_destroy(vattn_kvcache* c) {
