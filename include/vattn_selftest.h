@@ -20,6 +20,16 @@
 extern "C" {
 #endif
 vattn_status vattn_selftest_umma(int variant, const void* a, const void* b, float* out, vattn_stream stream);
+
+/*
+ * Timeout reporting check (no counterpart in the pages).  Launches one warp
+ * that waits, with a bound of limit_us microseconds (1..2000000), on a
+ * shared-memory barrier that nothing ever arrives on.  The wait gives up,
+ * records a code in the device status word and the kernel returns normally:
+ * the following vattn_check() reports VATTN_ERR_TIMEOUT and clears the word,
+ * and the context stays usable.  Nothing faults, traps or hangs.
+ */
+vattn_status vattn_selftest_wait_timeout(uint32_t limit_us, vattn_stream stream);
 #ifdef __cplusplus
 }
 #endif

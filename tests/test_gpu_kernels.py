@@ -137,3 +137,23 @@ def test_attention_single_token_and_tiny_lengths(va):
         va.vattn_check()
         ref, _ = oracle.attention(q, k, v, 0.125)
         assert_parity(from_dev(o), ref, "L=%d" % L)
+
+
+def test_bounded_wait_reports_timeout_and_context_survives(va):
+    # A barrier nothing arrives on: the kernel's bounded wait gives up after
+    # 50 ms, the status word reports a timeout, and the next call still works.
+    import torch
+    va.vattn_check()                                   # start from a clear status word
+    va.vattn_selftest_wait_timeout(50000)
+    with pytest.raises(va.VattnError) as e:
+        va.vattn_check()
+    assert e.value.status == va.ERR_TIMEOUT
+    va.vattn_check()                                   # cleared
+    q = si.normal_bf16(75, (1, 200, 1, 64))
+    k = si.normal_bf16(76, (1, 200, 1, 64))
+    v = si.normal_bf16(77, (1, 200, 1, 64))
+    o = torch.empty((1, 200, 1, 64), dtype=torch.bfloat16, device="cuda")
+    va.vattn_attention(to_dev(q), to_dev(k), to_dev(v), o, scale=0.125)
+    va.vattn_check()
+    ref, _ = oracle.attention(q, k, v, 0.125)
+    assert_parity(from_dev(o), ref, "after timeout")

@@ -87,6 +87,7 @@ _hyb_ws = _sig("vattn_hybrid_workspace_bytes", _S, _I, _I, _I, _I, _I)
 _hybrid = _sig("vattn_hybrid_chunk", _I, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _P, _S, _P)
 _hybrid_noalloc = _sig("vattn_hybrid_chunk_noalloc", _I, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _P)
 _selftest = _sig("vattn_selftest_umma", _I, _I, _P, _P, _P, _P)
+_selftest_timeout = _sig("vattn_selftest_wait_timeout", _I, ctypes.c_uint32, _P)
 HYBRID_NOALLOC_MAX_BYTES = 32 << 20
 
 
@@ -296,3 +297,7 @@ def vattn_check(stream=None):
 
 def vattn_selftest_umma(variant, a, b, out, stream=None):
     _ok(_selftest(variant, _bf16(a, "a"), _bf16(b, "b"), _ptr(out), _stream(stream)))
+
+
+def vattn_selftest_wait_timeout(limit_us, stream=None):
+    _ok(_selftest_timeout(limit_us, _stream(stream)))

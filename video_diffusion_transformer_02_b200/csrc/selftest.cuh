@@ -107,5 +107,22 @@ __global__ void __launch_bounds__(128, 1)
   }
 }
 
+// A wait that runs out: thread 0 arms an mbarrier that nothing ever
+// arrives on; every thread's bounded wait gives up after limit_ns, the
+// abort is raised (status word set) and the kernel returns normally.
+__global__ void __launch_bounds__(32, 1) wait_timeout_kernel(uint64_t limit_ns, uint32_t* status) {
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ uint32_t abort_flag;
+  const uint32_t b = smem_addr(&bar);
+  if (threadIdx.x == 0) {
+    mbar_init(b, 1);
+    abort_flag = 0;
+    fence_barrier_init();
+  }
+  __syncwarp();
+  Abort ab{&abort_flag, status};
+  mbar_wait_limit(b, 0, ab, kStatusTimeoutAux, limit_ns);
+}
+
 }  // namespace selftest
 }  // namespace vattn

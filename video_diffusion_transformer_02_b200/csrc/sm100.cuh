@@ -75,6 +75,23 @@ __device__ __forceinline__ void raise_abort(const Abort& ab, uint32_t code) {
   if (ab.status) atomicCAS(ab.status, 0u, code);
 }
 
+// As mbar_wait below, with an explicit time limit (ns) and no back-off.
+__device__ __forceinline__ bool mbar_wait_limit(uint32_t bar, uint32_t parity, const Abort& ab, uint32_t code,
+                                                uint64_t limit_ns) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = global_timer_ns();
+  for (uint32_t it = 1;; ++it) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((it & 63u) == 0u) {
+      if (*ab.flag) return false;
+      if (global_timer_ns() - t0 > limit_ns) {
+        raise_abort(ab, code);
+        return false;
+      }
+    }
+  }
+}
+
 // Wait until phase `parity` of `bar` has completed.  Returns false if the
 // CTA aborted or the wait exceeded kWaitLimitNs (then the abort is raised
 // with `code`).  sleep_ns > 0 backs off between polls (for threads whose

@@ -760,4 +760,15 @@ vattn_status vattn_selftest_umma(int variant, const void* a, const void* b, floa
   return VATTN_OK;
 }
 
+// Not part of the attention interface: drives a bounded wait to its limit
+// to check the timeout reporting path (see include/vattn_selftest.h).
+vattn_status vattn_selftest_wait_timeout(uint32_t limit_us, vattn_stream stream) {
+  if (limit_us == 0 || limit_us > 2000000) return fail(VATTN_ERR_INVALID_ARG, "limit_us must be 1..2000000");
+  uint32_t* status;
+  if (vattn_status st = status_ptr(&status)) return st;
+  vattn::selftest::wait_timeout_kernel<<<1, 32, 0, stream>>>(static_cast<uint64_t>(limit_us) * 1000ull, status);
+  VATTN_CUDA(cudaGetLastError());
+  return VATTN_OK;
+}
+
 }  // extern "C"
