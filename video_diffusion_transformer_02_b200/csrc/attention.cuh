@@ -566,12 +566,13 @@ __global__ void __launch_bounds__(attn_threads(ROPE, HYBRID), 1)
       m_run = 0.f;            // the linear part enters with reference max 0
     }
     const int cbase = wg * 64;    // first score column of this warpgroup
-    for (int j = 0; ok && j < nk; ++j) {
+    // No early exit: after a failed wait (which only happens once the CTA has
+    // aborted, when every later wait fails at once) the remaining tiles run
+    // on garbage, so both warpgroups execute the same row-max barriers and
+    // meet the epilogue barrier exactly once.
+    for (int j = 0; j < nk; ++j) {
       const int buf = j & 1;
-      if (!mbar_wait(bSFull(buf), (j >> 1) & 1, ab, kStatusTimeoutSoftmax, VATTN_SLEEP_SOFT)) {
-        ok = false;
-        break;
-      }
+      if (!mbar_wait(bSFull(buf), (j >> 1) & 1, ab, kStatusTimeoutSoftmax, VATTN_SLEEP_SOFT)) ok = false;
       tc_fence_after();
       const uint32_t tS = trow + (buf ? kColS1 : kColS0) + cbase;
       int col_lo = 0, col_hi = kTileN;
@@ -704,7 +705,6 @@ __global__ void __launch_bounds__(attn_threads(ROPE, HYBRID), 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(bPFull);
-      if (!ok) break;
       l_run = l_run * factor + rs;
     }
     // epilogue: O / l -> bf16 (each warpgroup writes its half of the
@@ -714,6 +714,7 @@ __global__ void __launch_bounds__(attn_threads(ROPE, HYBRID), 1)
       ok = mbar_wait(bPvDone, (need - 1) & 1, ab, kStatusTimeoutSoftmax);
       tc_fence_after();
     }
+    ok = __all_sync(0xffffffffu, ok);   // the epilogue's TMEM loads are warp-collective
     // row sums through the exchange slot of parity nk & 1: its last reads
     // (tile nk - 2) finished before the barrier of tile nk - 1
     float* xl = reinterpret_cast<float*>(smem + C::kOffXchg) + (nk & 1) * 256;   // [2 wg][128]
