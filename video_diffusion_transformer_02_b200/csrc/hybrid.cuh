@@ -129,12 +129,11 @@ __global__ void __launch_bounds__(256, 1)
     const int r = threadIdx.x - 128;   // token row of a tile; later feature column
     float zacc = 0.f;
     bool ok = true;
+    // No early exit (a failed wait only follows an abort): every thread runs
+    // the same number of named-barrier syncs below.
     for (int t = 0; t < nt; ++t) {
       const int s = t % NS;
-      if (!mbar_wait(bFull(s), (t / NS) & 1, ab, kStatusTimeoutAux)) {
-        ok = false;
-        break;
-      }
+      if (!mbar_wait(bFull(s), (t / NS) & 1, ab, kStatusTimeoutAux)) ok = false;
       const uint32_t kb = sK + s * C::kTileBytes;
       const bool valid = c0 + t * kRows + r < c1;   // rows past the chunk end weigh 0
 #pragma unroll 4
@@ -171,6 +170,7 @@ __global__ void __launch_bounds__(256, 1)
       ok = mbar_wait(bDone, 0, ab, kStatusTimeoutAux);
       tc_fence_after();
     }
+    ok = __all_sync(0xffffffffu, ok);   // the TMEM loads below are warp-collective
     if (ok) {
       const uint32_t trow = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
       float* dst = p.wsS + ((((static_cast<size_t>(c) * p.B + b) * p.H + h) * D) + r) * D;
@@ -204,7 +204,10 @@ __global__ void __launch_bounds__(256, 1)
 
 // Exclusive scan over chunks, in place in the workspace, starting from the
 // caller's state; the caller's state leaves as the total.  One float4 per
-// thread and element, coalesced 16-byte loads and stores.
+// thread and element; the loads of up to kScanBatch chunks are issued before
+// their stores (coalesced 16-byte accesses, many in flight).
+constexpr int kScanBatch = 8;
+
 __global__ void __launch_bounds__(256) scan_kernel(float4* __restrict__ wsS, float4* __restrict__ S, long long nS4,
                                                    float4* __restrict__ wsz, float4* __restrict__ z, long long nz4,
                                                    int C) {
@@ -217,15 +220,21 @@ __global__ void __launch_bounds__(256) scan_kernel(float4* __restrict__ wsS, flo
     float4* ws = isS ? wsS : wsz;
     float4* st = isS ? S : z;
     float4 run = st[e];
-    float4 nxt = C > 0 ? ws[e] : make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int c = 0; c < C; ++c) {
-      const float4 d = nxt;
-      if (c + 1 < C) nxt = ws[(c + 1) * n + e];
-      ws[c * n + e] = run;
-      run.x += d.x;
-      run.y += d.y;
-      run.z += d.z;
-      run.w += d.w;
+    for (int c0 = 0; c0 < C; c0 += kScanBatch) {
+      float4 d[kScanBatch];
+#pragma unroll
+      for (int u = 0; u < kScanBatch; ++u)
+        if (c0 + u < C) d[u] = ws[(c0 + u) * n + e];
+#pragma unroll
+      for (int u = 0; u < kScanBatch; ++u) {
+        if (c0 + u < C) {
+          ws[(c0 + u) * n + e] = run;
+          run.x += d[u].x;
+          run.y += d[u].y;
+          run.z += d[u].z;
+          run.w += d[u].w;
+        }
+      }
     }
     st[e] = run;
   }

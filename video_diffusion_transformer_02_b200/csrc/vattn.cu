@@ -188,6 +188,20 @@ void fill_rope_params(vattn::attn::Params& p, const vattn_rope* r, const float* 
   p.rope_maxpos = r->max_pos;
 }
 
+// Rows split evenly over whole waves of 8 blocks per SM; threads cover the
+// chunks of one row (up to 256 per pass).
+template <bool COPY>
+cudaError_t launch_rotate_rows(const vattn::rope::RotParams& p, cudaStream_t stream) {
+  int sms = 148, dev;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int cpt = p.heads * (p.d / 8);
+  const int threads = cpt < 256 ? ((cpt + 31) / 32) * 32 : 256;
+  long long blocks = static_cast<long long>(sms) * 8;
+  if (blocks > p.rows) blocks = p.rows;
+  vattn::rope::rotate_rows_kernel<COPY><<<static_cast<int>(blocks), threads, 0, stream>>>(p);
+  return cudaGetLastError();
+}
+
 }  // namespace
 
 // ============================================================ C interface
@@ -211,30 +225,27 @@ size_t frame_bytes(const vattn_kvcache* c) { return static_cast<size_t>(c->B) * 
 // Launch the append / rotate pass for one frame.  kr/vr null: rotate only.
 vattn_status launch_append_rope(const vattn_kvcache* c, const void* k, const void* v, void* kr, void* vr,
                                 int32_t* ids, int slot, int frame, cudaStream_t stream) {
-  vattn::kv::AppendRopeParams p{};
-  p.k = static_cast<const uint4*>(k);
-  p.v = static_cast<const uint4*>(v);
-  p.kr = static_cast<uint4*>(kr);
-  p.vr = static_cast<uint4*>(vr);
-  p.krot = reinterpret_cast<uint4*>(static_cast<uint8_t*>(c->k_rot) +
-                                    static_cast<size_t>(frame % (c->capacity + 1)) * frame_bytes(c));
-  p.n16 = static_cast<long long>(frame_bytes(c) / 16);
-  p.ids = ids;
-  p.slot = slot;
-  p.frame = frame;
-  p.F = c->F;
-  p.Hkv = c->Hkv;
+  vattn::rope::RotParams p{};
+  p.src = static_cast<const uint4*>(k);
+  p.dst = reinterpret_cast<uint4*>(static_cast<uint8_t*>(c->k_rot) +
+                                   static_cast<size_t>(frame % (c->capacity + 1)) * frame_bytes(c));
+  p.src2 = static_cast<const uint4*>(v);
+  p.raw_dst = static_cast<uint4*>(kr);
+  p.raw_dst2 = static_cast<uint4*>(vr);
+  p.rows = static_cast<long long>(c->B) * c->F;
+  p.L = c->F;
+  p.heads = c->Hkv;
   p.d = c->d;
+  p.frame_offset = frame;
+  p.Hg = c->rope.Hg;
   p.Wg = c->rope.Wg;
   p.pt = c->rope.pairs_t;
   p.ph = c->rope.pairs_h;
   p.tab = reinterpret_cast<const float2*>(c->table);
-  int sms = 148, dev;
-  if (current_device(&dev) == VATTN_OK) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  const long long want = (p.n16 + 255) / 256;
-  const int blocks = static_cast<int>(want < sms * 8LL ? want : sms * 8LL);
-  vattn::kv::append_rope_kernel<<<blocks, 256, 0, stream>>>(p);
-  VATTN_CUDA(cudaGetLastError());
+  p.ids = ids;
+  p.slot = slot;
+  p.frame = frame;
+  VATTN_CUDA(kr ? launch_rotate_rows<true>(p, stream) : launch_rotate_rows<false>(p, stream));
   return VATTN_OK;
 }
 
@@ -305,32 +316,25 @@ vattn_status vattn_rope_qk(const void* q, const void* k, void* q_out, void* k_ou
   const long long F = static_cast<long long>(rope->Hg) * rope->Wg;
   if (frame_offset + (L - 1) / F >= rope->max_pos)
     return fail(VATTN_ERR_INVALID_ARG, "frame index beyond rope max_pos");
-  vattn::rope::QKParams p{};
-  p.src[0] = static_cast<const uint4*>(q);
-  p.dst[0] = static_cast<uint4*>(q_out);
-  p.n16[0] = q ? static_cast<long long>(B) * L * H * d / 8 : 0;
-  p.src[1] = static_cast<const uint4*>(k);
-  p.dst[1] = static_cast<uint4*>(k_out);
-  p.n16[1] = k ? static_cast<long long>(B) * L * Hkv * d / 8 : 0;
-  p.heads[0] = H;
-  p.heads[1] = Hkv;
-  p.L = L;
-  p.d = d;
-  p.Hg = rope->Hg;
-  p.Wg = rope->Wg;
-  p.pt = rope->pairs_t;
-  p.ph = rope->pairs_h;
-  p.frame_offset = frame_offset;
-  p.tab = reinterpret_cast<const float2*>(table);
-  const long long total = p.n16[0] + p.n16[1];
-  if (total == 0) return VATTN_OK;
-  int sms = 148;
-  int dev;
-  if (current_device(&dev) == VATTN_OK) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  const long long want = (total + 255) / 256;
-  const int blocks = static_cast<int>(want < sms * 16LL ? want : sms * 16LL);
-  vattn::rope::rope_qk_kernel<<<blocks, 256, 0, stream>>>(p);
-  VATTN_CUDA(cudaGetLastError());
+  for (int which = 0; which < 2; ++which) {
+    const void* src = which ? k : q;
+    void* dst = which ? k_out : q_out;
+    if (!src) continue;
+    vattn::rope::RotParams p{};
+    p.src = static_cast<const uint4*>(src);
+    p.dst = static_cast<uint4*>(dst);
+    p.rows = static_cast<long long>(B) * L;
+    p.L = L;
+    p.heads = which ? Hkv : H;
+    p.d = d;
+    p.frame_offset = frame_offset;
+    p.Hg = rope->Hg;
+    p.Wg = rope->Wg;
+    p.pt = rope->pairs_t;
+    p.ph = rope->pairs_h;
+    p.tab = reinterpret_cast<const float2*>(table);
+    VATTN_CUDA(launch_rotate_rows<false>(p, stream));
+  }
   return VATTN_OK;
 }
 
@@ -473,8 +477,11 @@ vattn_status vattn_kvcache_append(vattn_kvcache* c, const void* k, const void* v
   }
   int sms = 148, dev;
   if (current_device(&dev) == VATTN_OK) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  const long long want = (n16 + 255) / 256;
-  const int blocks = static_cast<int>(want < sms * 8LL ? want : sms * 8LL);
+  // an equal share for every SM: a multiple of the SM count, each thread
+  // moving kUnroll vectors per tensor and step
+  const long long want = (n16 + 256LL * vattn::kv::kUnroll - 1) / (256LL * vattn::kv::kUnroll);
+  const long long per_sm = (want + sms - 1) / sms;
+  const int blocks = static_cast<int>(sms * (per_sm < 8 ? per_sm : 8));
   vattn::kv::append_kernel<<<blocks, 256, 0, stream>>>(static_cast<const uint4*>(k), static_cast<const uint4*>(v),
                                                        kr, vr, n16, c->frame_ids, slot, frame_idx);
   VATTN_CUDA(cudaGetLastError());
