@@ -178,12 +178,15 @@ vattn_status vattn_kvcache_restore(vattn_kvcache* cache, const int32_t* host_ids
  * tile that reads them (FlashDecoder applies RoPE with precomputed tables,
  * "Inference Optimization", Sec. 4.6).  k_ring_rot: caller-owned bf16
  * [capacity + 1][B][F][Hkv][d]; frame f's rotated keys live in slot
- * f % (capacity + 1).  From then on vattn_kvcache_append writes the raw copy
- * and the rotated copy in one pass, and vattn_attention_stream (which must
- * then be given the same rope and table) rotates the current frame's keys
- * into the spare slot and reads rotated keys only.  Frames already in the
- * ring are rotated now, on `stream`.  The raw ring stays the exact input
- * bytes.
+ * f % (capacity + 1).  From then on vattn_attention_stream (which must then
+ * be given the same rope and table) rotates the current frame's keys into
+ * slot frame_idx % (capacity + 1), outside the window, and reads rotated keys
+ * only; vattn_kvcache_append then copies the raw K and V, and also writes the
+ * rotated copy in the same pass unless the last vattn_attention_stream call
+ * on this cache was for the same frame with the same k pointer (those keys
+ * are in place already; the caller must not change the k buffer's contents
+ * between the two calls).  Frames already in the ring are rotated now, on
+ * `stream`.  The raw ring stays the exact input bytes.
  */
 vattn_status vattn_kvcache_enable_rope(vattn_kvcache* cache, void* k_ring_rot, const vattn_rope* rope,
                                        const float* table, vattn_stream stream);

@@ -37,15 +37,25 @@ struct DeltaCfg {
   static constexpr int kSmemBytes = kOffMisc + 64 + 1024;
 };
 
-// grid (C, H, B), 256 threads: warp 0 TMA, warp 1 TMEM + MMA, warps 4..7
-// feature map / column sums / epilogue.
+// grid (C, H, B), 384 threads: warp 0 TMA, warp 1 TMEM + MMA, warps 4..11
+// feature map, column sums and epilogue.  Feature-map thread t owns the
+// 16-byte chunk t % 16 (eight features) of rows t / 16 + 16 i of every tile,
+// so the column sums of its eight features stay in registers; the eight
+// warps release a stage with one arrive each, with no block-wide barrier
+// per tile, and the column sums are reduced across rows once at the end.
+constexpr int kDeltaThreads = 384;
+constexpr int kPhiThreads = 256;
+
 template <int D>
-__global__ void __launch_bounds__(256, 1)
+__global__ void __launch_bounds__(kDeltaThreads, 1)
     delta_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                  const DeltaParams p) {
   static_assert(D == 128, "state delta supports head_dim 128");
   using C = DeltaCfg<D>;
   constexpr int NS = C::kStages;
+  constexpr int kChunks = D / 8;                       // 16-byte chunks per row
+  constexpr int kRowGroups = kPhiThreads / kChunks;    // rows handled in parallel
+  constexpr int kRowsPerThread = kRows / kRowGroups;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sbase = smem_addr(smem);
@@ -68,7 +78,7 @@ __global__ void __launch_bounds__(256, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < NS; ++s) {
       mbar_init(bFull(s), 1);
-      mbar_init(bPhi(s), 4);
+      mbar_init(bPhi(s), kPhiThreads / 32);
       mbar_init(bEmpty(s), 1);
     }
     mbar_init(bDone, 1);
@@ -126,43 +136,42 @@ __global__ void __launch_bounds__(256, 1)
       }
     }
   } else if (warp >= 4) {
-    const int r = threadIdx.x - 128;   // token row of a tile; later feature column
-    float zacc = 0.f;
+    const int tid = threadIdx.x - 128;
+    const int ch = tid % kChunks, rg = tid / kChunks;
+    // address of this thread's chunk in row rg of a tile; row rg + 16 i adds
+    // 16 i * 128 bytes and keeps the swizzle phase (16 i is a multiple of 8)
+    const uint32_t off0 = (ch >> 3) * (kRows * 128) + sw128_offset(rg, ch & 7);
+    float zacc[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) zacc[e] = 0.f;
     bool ok = true;
-    // No early exit (a failed wait only follows an abort): every thread runs
-    // the same number of named-barrier syncs below.
+    // No early exit (a failed wait only follows an abort): every thread
+    // reaches the reduction barrier below.
     for (int t = 0; t < nt; ++t) {
       const int s = t % NS;
       if (!mbar_wait(bFull(s), (t / NS) & 1, ab, kStatusTimeoutAux)) ok = false;
-      const uint32_t kb = sK + s * C::kTileBytes;
-      const bool valid = c0 + t * kRows + r < c1;   // rows past the chunk end weigh 0
-#pragma unroll 4
-      for (int c16 = 0; c16 < D / 8; ++c16) {
-        const uint32_t addr = kb + (c16 >> 3) * (kRows * 128) + sw128_offset(r, c16 & 7);
-        const uint4 v = lds128(addr);
-        uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+      const uint32_t kb = sK + s * C::kTileBytes + off0;
+      const int row_end = c1 - (c0 + t * kRows);    // rows at or past it belong to the next chunk
+      uint4 v[kRowsPerThread];
+#pragma unroll
+      for (int i = 0; i < kRowsPerThread; ++i) v[i] = lds128(kb + i * (kRowGroups * 128));
+#pragma unroll
+      for (int i = 0; i < kRowsPerThread; ++i) {
+        const bool valid = rg + i * kRowGroups < row_end;
+        uint32_t w4[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           float x0 = bf16lo_to_f32(w4[e]), x1 = bf16hi_to_f32(w4[e]);
           x0 = valid ? (x0 > 0.f ? x0 + 1.f : __expf(x0)) : 0.f;
           x1 = valid ? (x1 > 0.f ? x1 + 1.f : __expf(x1)) : 0.f;
           w4[e] = pack_bf16x2(x0, x1);
+          // z sums the same bf16 values the MMA multiplies
+          zacc[2 * e] += bf16lo_to_f32(w4[e]);
+          zacc[2 * e + 1] += bf16hi_to_f32(w4[e]);
         }
-        sts128(addr, make_uint4(w4[0], w4[1], w4[2], w4[3]));
+        sts128(kb + i * (kRowGroups * 128), make_uint4(w4[0], w4[1], w4[2], w4[3]));
       }
       fence_proxy_async_smem();
-      asm volatile("bar.sync 1, 128;" ::: "memory");
-      // column sums of the (bf16) feature map: thread r owns feature r
-      {
-        const uint32_t colbase = kb + (r >> 6) * (kRows * 128);
-        const uint32_t chunk = (r & 63) >> 3, within = (r & 7) * 2;
-#pragma unroll 8
-        for (int row = 0; row < kRows; ++row) {
-          uint16_t hv;
-          asm volatile("ld.shared.u16 %0, [%1];" : "=h"(hv) : "r"(colbase + sw128_offset(row, chunk) + within));
-          zacc += __uint_as_float(static_cast<uint32_t>(hv) << 16);
-        }
-      }
       __syncwarp();
       if (lane == 0) mbar_arrive(bPhi(s));
     }
@@ -170,27 +179,40 @@ __global__ void __launch_bounds__(256, 1)
       ok = mbar_wait(bDone, 0, ab, kStatusTimeoutAux);
       tc_fence_after();
     }
+    // reduce the column sums over the row groups (stage 0 of K is free now:
+    // every load has landed and every MMA has completed or the kernel aborts)
+    float* red = reinterpret_cast<float*>(smem + C::kOffK);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) red[rg * D + ch * 8 + e] = zacc[e];
+    asm volatile("bar.sync 1, %0;" ::"n"(kPhiThreads) : "memory");
+    if (tid < D) {
+      float zs = 0.f;
+#pragma unroll
+      for (int g = 0; g < kRowGroups; ++g) zs += red[g * D + tid];
+      p.wsz[((static_cast<size_t>(c) * p.B + b) * p.H + h) * D + tid] = zs;
+    }
     ok = __all_sync(0xffffffffu, ok);   // the TMEM loads below are warp-collective
-    if (ok) {
-      const uint32_t trow = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
-      float* dst = p.wsS + ((((static_cast<size_t>(c) * p.B + b) * p.H + h) * D) + r) * D;
+    // S rows from TMEM: warp w reads lanes 32 (w % 4) ..; warps 4..7 take
+    // columns 0..63, warps 8..11 columns 64..127
+    const int r = (warp & 3) * 32 + lane;
+    const int cb = (warp >= 8) ? D / 2 : 0;
+    float* dst = p.wsS + ((((static_cast<size_t>(c) * p.B + b) * p.H + h) * D) + r) * D + cb;
+    const uint32_t trow = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16) + cb;
 #pragma unroll 1
-      for (int q = 0; q < D / 32; ++q) {
-        uint32_t v[32];
-        if (nt > 0) {
-          tmem_ld32(trow + q * 32, v);
-          tmem_ld_wait();
-        } else {
+    for (int q = 0; q < D / 64; ++q) {
+      uint32_t v[32];
+      if (ok && nt > 0) {
+        tmem_ld32(trow + q * 32, v);
+        tmem_ld_wait();
+      } else {
 #pragma unroll
-          for (int e = 0; e < 32; ++e) v[e] = 0u;
-        }
-        float4* d4 = reinterpret_cast<float4*>(dst + q * 32);
-#pragma unroll
-        for (int e = 0; e < 8; ++e)
-          d4[e] = make_float4(__uint_as_float(v[4 * e]), __uint_as_float(v[4 * e + 1]),
-                              __uint_as_float(v[4 * e + 2]), __uint_as_float(v[4 * e + 3]));
+        for (int e = 0; e < 32; ++e) v[e] = 0u;
       }
-      p.wsz[((static_cast<size_t>(c) * p.B + b) * p.H + h) * D + r] = zacc;
+      float4* d4 = reinterpret_cast<float4*>(dst + q * 32);
+#pragma unroll
+      for (int e = 0; e < 8; ++e)
+        d4[e] = make_float4(__uint_as_float(v[4 * e]), __uint_as_float(v[4 * e + 1]),
+                            __uint_as_float(v[4 * e + 2]), __uint_as_float(v[4 * e + 3]));
     }
   }
 
@@ -206,29 +228,30 @@ __global__ void __launch_bounds__(256, 1)
 // caller's state; the caller's state leaves as the total.  One float4 per
 // thread and element; the loads of up to kScanBatch chunks are issued before
 // their stores (coalesced 16-byte accesses, many in flight).
-constexpr int kScanBatch = 8;
+constexpr int kScanBatch = 12;
 
-__global__ void __launch_bounds__(256) scan_kernel(float4* __restrict__ wsS, float4* __restrict__ S, long long nS4,
-                                                   float4* __restrict__ wsz, float4* __restrict__ z, long long nz4,
-                                                   int C) {
+__global__ void __launch_bounds__(256, 2) scan_kernel(float4* __restrict__ wsS, float4* __restrict__ S, long long nS4,
+                                                      float4* __restrict__ wsz, float4* __restrict__ z, long long nz4,
+                                                      int C) {
   const long long total = nS4 + nz4;
   for (long long idx = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; idx < total;
        idx += static_cast<long long>(gridDim.x) * blockDim.x) {
     const bool isS = idx < nS4;
     const long long e = isS ? idx : idx - nS4;
     const long long n = isS ? nS4 : nz4;
-    float4* ws = isS ? wsS : wsz;
-    float4* st = isS ? S : z;
-    float4 run = st[e];
+    float4* col = (isS ? wsS : wsz) + e;   // chunk c's element at col[c * n]
+    float4* st = (isS ? S : z) + e;
+    float4 run = *st;
     for (int c0 = 0; c0 < C; c0 += kScanBatch) {
+      float4* base = col + c0 * n;
       float4 d[kScanBatch];
 #pragma unroll
       for (int u = 0; u < kScanBatch; ++u)
-        if (c0 + u < C) d[u] = ws[(c0 + u) * n + e];
+        if (c0 + u < C) d[u] = base[u * n];
 #pragma unroll
       for (int u = 0; u < kScanBatch; ++u) {
         if (c0 + u < C) {
-          ws[(c0 + u) * n + e] = run;
+          base[u * n] = run;
           run.x += d[u].x;
           run.y += d[u].y;
           run.z += d[u].z;
@@ -236,7 +259,7 @@ __global__ void __launch_bounds__(256) scan_kernel(float4* __restrict__ wsS, flo
         }
       }
     }
-    st[e] = run;
+    *st = run;
   }
 }
 

@@ -61,7 +61,7 @@ struct RotParams {
 };
 
 template <bool COPY>
-__global__ void __launch_bounds__(256) rotate_rows_kernel(const RotParams p) {
+__global__ void __launch_bounds__(512) rotate_rows_kernel(const RotParams p) {
   const int cpt = p.heads * (p.d / 8);                 // chunks per row
   const long long rows_per_block = (p.rows + gridDim.x - 1) / gridDim.x;
   const long long r0 = static_cast<long long>(blockIdx.x) * rows_per_block;

@@ -188,16 +188,22 @@ void fill_rope_params(vattn::attn::Params& p, const vattn_rope* r, const float* 
   p.rope_maxpos = r->max_pos;
 }
 
-// Rows split evenly over whole waves of 8 blocks per SM; threads cover the
-// chunks of one row (up to 256 per pass).
+// Threads cover the chunks of one row in as few equal passes of at most
+// 512 as possible; each block takes 4..16 consecutive rows (about 4 blocks
+// per SM for small tensors, 16 rows per block for large ones), so a thread
+// has several independent rows in flight.
 template <bool COPY>
 cudaError_t launch_rotate_rows(const vattn::rope::RotParams& p, cudaStream_t stream) {
   int sms = 148, dev;
   if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const int cpt = p.heads * (p.d / 8);
-  const int threads = cpt < 256 ? ((cpt + 31) / 32) * 32 : 256;
-  long long blocks = static_cast<long long>(sms) * 8;
+  const int passes = (cpt + 511) / 512;
+  const int threads = (((cpt + passes - 1) / passes + 31) / 32) * 32;
+  long long rpb = p.rows / (4LL * sms);
+  rpb = rpb < 4 ? 4 : (rpb > 16 ? 16 : rpb);
+  long long blocks = (p.rows + rpb - 1) / rpb;
   if (blocks > p.rows) blocks = p.rows;
+  if (blocks > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
   vattn::rope::rotate_rows_kernel<COPY><<<static_cast<int>(blocks), threads, 0, stream>>>(p);
   return cudaGetLastError();
 }
@@ -217,6 +223,10 @@ struct vattn_kvcache {
   vattn_rope rope{};
   const float* table = nullptr;
   CUtensorMap map_krot;
+  // the last vattn_attention_stream call rotated these keys of this frame
+  // into the rotated ring (host-side record; cleared by restore/enable_rope)
+  const void* rotated_k = nullptr;
+  int rotated_frame = -1;
 };
 
 namespace {
@@ -469,19 +479,24 @@ vattn_status vattn_kvcache_append(vattn_kvcache* c, const void* k, const void* v
   const long long n16 = bytes / 16;
   uint4* kr = reinterpret_cast<uint4*>(static_cast<uint8_t*>(c->k_ring) + slot * bytes);
   uint4* vr = reinterpret_cast<uint4*>(static_cast<uint8_t*>(c->v_ring) + slot * bytes);
-  if (c->k_rot) {
+  const bool rotated = c->k_rot && c->rotated_k == k && c->rotated_frame == frame_idx;
+  c->rotated_k = nullptr;
+  c->rotated_frame = -1;
+  if (c->k_rot && !rotated) {
     if (frame_idx >= c->rope.max_pos) return fail(VATTN_ERR_INVALID_ARG, "frame index beyond rope max_pos");
     if (vattn_status st = launch_append_rope(c, k, v, kr, vr, c->frame_ids, slot, frame_idx, stream)) return st;
     c->host_ids[slot] = frame_idx;
     return VATTN_OK;
   }
+  // plain copy (also when the stream call already rotated these keys)
   int sms = 148, dev;
   if (current_device(&dev) == VATTN_OK) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  // an equal share for every SM: a multiple of the SM count, each thread
-  // moving kUnroll vectors per tensor and step
+  // an equal share for every SM: a multiple of the SM count (at most two
+  // blocks per SM, the fastest measured for one frame), each thread moving
+  // kUnroll vectors per tensor and step
   const long long want = (n16 + 256LL * vattn::kv::kUnroll - 1) / (256LL * vattn::kv::kUnroll);
   const long long per_sm = (want + sms - 1) / sms;
-  const int blocks = static_cast<int>(sms * (per_sm < 8 ? per_sm : 8));
+  const int blocks = static_cast<int>(sms * (per_sm < 2 ? per_sm : 2));
   vattn::kv::append_kernel<<<blocks, 256, 0, stream>>>(static_cast<const uint4*>(k), static_cast<const uint4*>(v),
                                                        kr, vr, n16, c->frame_ids, slot, frame_idx);
   VATTN_CUDA(cudaGetLastError());
@@ -538,6 +553,8 @@ vattn_status vattn_attention_stream(vattn_kvcache* c, const void* q, const void*
     // which holds a frame outside the window
     if (vattn_status st = launch_append_rope(c, k_cur, v_cur, nullptr, nullptr, nullptr, 0, frame_idx, stream))
       return st;
+    c->rotated_k = k_cur;
+    c->rotated_frame = frame_idx;
   }
   int n = 0, tiles = 0;
   const int per = (c->F + 127) / 128;
@@ -596,6 +613,8 @@ vattn_status vattn_kvcache_restore(vattn_kvcache* c, const int32_t* host_ids, va
     if (host_ids[i] >= 0 && host_ids[i] % c->capacity != i)
       return fail(VATTN_ERR_INVALID_ARG, "frame %d cannot sit in slot %d", host_ids[i], i);
   std::memcpy(c->host_ids.data(), host_ids, sizeof(int32_t) * c->capacity);
+  c->rotated_k = nullptr;
+  c->rotated_frame = -1;
   if (c->k_rot) return rerotate_present(c, stream);
   return VATTN_OK;
 }
@@ -615,6 +634,8 @@ vattn_status vattn_kvcache_enable_rope(vattn_kvcache* c, void* k_ring_rot, const
   c->rope = *rope;
   c->table = table;
   c->map_krot = m;
+  c->rotated_k = nullptr;
+  c->rotated_frame = -1;
   return rerotate_present(c, stream);
 }
 
@@ -663,7 +684,7 @@ vattn_status vattn_hybrid_chunk(const void* q, const void* k, const void* v, voi
     const int smem = vattn::hyb::DeltaCfg<128>::kSmemBytes;
     if (vattn_status st = ensure_smem(kern, smem, done)) return st;
     vattn::hyb::DeltaParams dp{wsS, wsz, status, B, L, H, chunk_tokens};
-    kern<<<dim3(C, H, B), 256, smem, stream>>>(mk, mv, dp);
+    kern<<<dim3(C, H, B), vattn::hyb::kDeltaThreads, smem, stream>>>(mk, mv, dp);
     VATTN_CUDA(cudaGetLastError());
   }
   // (2) exclusive scan over chunks (+ state out)
@@ -672,7 +693,7 @@ vattn_status vattn_hybrid_chunk(const void* q, const void* k, const void* v, voi
     int sms = 148, dev;
     if (current_device(&dev) == VATTN_OK) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     const long long want = (nS4 + nz4 + 255) / 256;
-    const int blocks = static_cast<int>(want < sms * 8LL ? want : sms * 8LL);
+    const int blocks = static_cast<int>(want < sms * 4LL ? want : sms * 4LL);
     vattn::hyb::scan_kernel<<<blocks, 256, 0, stream>>>(reinterpret_cast<float4*>(wsS), reinterpret_cast<float4*>(S),
                                                         nS4, reinterpret_cast<float4*>(wsz),
                                                         reinterpret_cast<float4*>(z), nz4, C);
