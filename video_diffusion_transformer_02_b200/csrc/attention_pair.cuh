@@ -1,0 +1,494 @@
+// Attention forward for sm_100a, two 128-query tiles (A and B) of one head
+// per CTA.  Same operation, modes, masks and RoPE placement as
+// attn_fwd_kernel (see attention.cuh); what changes is the schedule:
+//
+//   * one softmax warpgroup per query tile, each thread owning a whole
+//     128-key row of S (no row-max exchange between warpgroups);
+//   * the MMA thread alternates between the tiles, so the tensor core works
+//     on one tile's S = Q K^T / O += P V while the other tile's softmax runs
+//     (the FlashAttention-4 ping-pong for Blackwell);
+//   * every K and V tile is loaded into shared memory once for both query
+//     tiles (half the L2 -> shared-memory traffic of one tile per CTA).
+//
+// Warp roles: warp 0 TMA Q_A, Q_B, then K tiles; warp 1 TMEM allocation and
+// tcgen05.mma issue; warp 2 TMA V tiles; warps 4..7 softmax of tile A,
+// warps 8..11 softmax of tile B (thread r owns query row r = TMEM lane r).
+//
+// TMEM columns (512): S_A [0,128), S_B [128,256) fp32; O_A [256,256+D),
+// O_B [384,384+D) fp32.  P_X (bf16 pairs, 64 columns) overwrites the first
+// half of S_X once the softmax holds S_X in registers; the MMA thread issues
+// the next S_X = Q_X K^T only after the P_X V that reads P_X has completed.
+#pragma once
+#include "attention.cuh"
+
+namespace vattn {
+namespace attn {
+
+template <int D>
+struct PairCfg {
+  static constexpr int kTileBytes = kTileM * D * 2;
+  static constexpr int kBlocks = D / 64;
+  static constexpr int kStages = D == 128 ? 2 : 4;
+  static constexpr int kOffQ = 0;                          // Q_A, Q_B
+  static constexpr int kOffK = 2 * kTileBytes;
+  static constexpr int kOffV = kOffK + kStages * kTileBytes;
+  static constexpr int kOffBar = kOffV + kStages * kTileBytes;
+  static constexpr int kNumBars = 4 + 4 * kStages + 6 + 1;
+  static constexpr int kOffMisc = kOffBar + kNumBars * 8;
+  static constexpr int kSmemBytes = kOffMisc + 64;
+};
+
+constexpr int kPairThreads = 384;
+
+// Rows of the two query tiles of pair `pr` and the key tiles they need
+// (the union of both tiles' visible ranges; rows mask what they do not see).
+struct PairGeom {
+  int q0[2], q_end[2];
+  bool hasB;
+  TileGeom tg;   // q0 / q_end span both tiles; kbeg, kend, n_tiles: the union
+};
+
+__device__ __forceinline__ PairGeom pair_geom(const Params& p, int pr) {
+  PairGeom g;
+  const int pps = (p.q_tiles_per_seg + 1) / 2;
+  const int seg = pr / pps;
+  const int t = pr - seg * pps;
+  int e = (seg + 1) * p.q_seg_len;
+  if (e > p.Lq) e = p.Lq;
+  g.q0[0] = seg * p.q_seg_len + 2 * t * kTileM;
+  g.q_end[0] = min(g.q0[0] + kTileM, e);
+  g.q0[1] = g.q0[0] + kTileM;
+  g.q_end[1] = min(g.q0[1] + kTileM, e);
+  g.hasB = g.q0[1] < g.q_end[1];
+  g.tg.q0 = g.q0[0];
+  g.tg.q_end = g.hasB ? g.q_end[1] : g.q_end[0];
+  if (p.n_kseg == 0) {
+    int lo0, hi0, lo1, hi1;
+    key_range(p, g.tg.q0, lo0, hi0);
+    key_range(p, g.tg.q_end - 1, lo1, hi1);
+    g.tg.kbeg = lo0;
+    g.tg.kend = hi1;
+    g.tg.n_tiles = g.tg.kend > g.tg.kbeg ? (g.tg.kend - g.tg.kbeg + kTileN - 1) / kTileN : 0;
+  } else {
+    g.tg.kbeg = g.tg.kend = 0;
+    const KeySegment& last = p.kseg[p.n_kseg - 1];
+    g.tg.n_tiles = last.tile0 + (last.n_tok + kTileN - 1) / kTileN;
+  }
+  return g;
+}
+
+// Keep the 32 registers of r after every earlier volatile statement (the
+// TMEM load wait): later uses cannot be scheduled above it.
+__device__ __forceinline__ void reg_tie32(uint32_t (&r)[32]) {
+  asm volatile("" : VATTN_RW8(0), VATTN_RW8(8), VATTN_RW8(16), VATTN_RW8(24));
+}
+
+template <int D, int ROPE>
+__global__ void __launch_bounds__(kPairThreads, 1)
+    attn_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                     const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmK2,
+                     const __grid_constant__ CUtensorMap tmV2, const Params p) {
+  static_assert(ROPE == kRopeNone || ROPE == kRopeQ, "keys are rotated before this kernel");
+  using C = PairCfg<D>;
+  constexpr int NS = C::kStages;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = smem_raw;
+  const uint32_t sbase = smem_addr(smem);
+  if (sbase & 1023u) {   // 128B-swizzled operand tiles need 1024-byte alignment
+    if (threadIdx.x == 0 && p.status) atomicCAS(p.status, 0u, kStatusSmemAlign);
+    return;
+  }
+  const uint32_t sQ = sbase + C::kOffQ, sK = sbase + C::kOffK, sV = sbase + C::kOffV;
+  const uint32_t bar0 = sbase + C::kOffBar;
+  auto bQFull = [&](int x) { return bar0 + 8 * x; };
+  auto bQReady = [&](int x) { return bar0 + 16 + 8 * x; };
+  auto bKFull = [&](int s) { return bar0 + 32 + 8 * s; };
+  auto bKEmpty = [&](int s) { return bar0 + 32 + 8 * (NS + s); };
+  auto bVFull = [&](int s) { return bar0 + 32 + 8 * (2 * NS + s); };
+  auto bVEmpty = [&](int s) { return bar0 + 32 + 8 * (3 * NS + s); };
+  const uint32_t bx = bar0 + 32 + 32 * NS;
+  auto bSFull = [&](int x) { return bx + 8 * x; };
+  auto bPFull = [&](int x) { return bx + 16 + 8 * x; };
+  auto bPvDone = [&](int x) { return bx + 32 + 8 * x; };
+  const uint32_t bFinal = bx + 48;
+  uint32_t* misc = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
+  volatile uint32_t* tmem_slot = misc;
+  volatile uint32_t* abort_flag = misc + 1;
+  Abort ab{abort_flag, p.status};
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int h = blockIdx.y, b = blockIdx.z;
+  const int kvh = h / (p.H / p.Hkv);
+  const int pr = p.reverse_q ? static_cast<int>(gridDim.x - 1 - blockIdx.x) : static_cast<int>(blockIdx.x);
+  const PairGeom g = pair_geom(p, pr);
+  if (g.q0[0] >= g.q_end[0]) return;   // pair past the end of a short last segment
+  const int nk = g.tg.n_tiles;
+  const bool hasB = g.hasB;
+
+  if (threadIdx.x == 0) {
+    for (int x = 0; x < 2; ++x) {
+      mbar_init(bQFull(x), 1);
+      mbar_init(bQReady(x), 4);
+      mbar_init(bSFull(x), 1);
+      mbar_init(bPFull(x), 4);
+      mbar_init(bPvDone(x), 1);
+    }
+    for (int s = 0; s < NS; ++s) {
+      mbar_init(bKFull(s), 1);
+      mbar_init(bKEmpty(s), 1);
+      mbar_init(bVFull(s), 1);
+      mbar_init(bVEmpty(s), 1);
+    }
+    mbar_init(bFinal, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tmQ);
+    tma_prefetch_desc(&tmK);
+    tma_prefetch_desc(&tmV);
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_addr(const_cast<uint32_t*>(tmem_slot)), kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------ producer: Q_A, Q_B, then K
+    if (lane == 0) {
+      for (int x = 0; x < (hasB ? 2 : 1); ++x) {
+        mbar_arrive_expect_tx(bQFull(x), C::kTileBytes);
+#pragma unroll
+        for (int blk = 0; blk < C::kBlocks; ++blk)
+          tma_load_4d(sQ + x * C::kTileBytes + blk * (kTileM * 128), &tmQ, bQFull(x), blk * 64, h,
+                      x ? g.q0[1] : g.q0[0], b);
+      }
+      int j = 0;
+      for (; j < nk; ++j) {
+        const int s = j % NS;
+        if (j >= NS && !mbar_wait(bKEmpty(s), ((j / NS) - 1) & 1, ab, kStatusTimeoutProducer)) break;
+        const KeyTile kt = key_tile(p, g.tg, j);
+        const CUtensorMap* m = kt.kmap ? &tmK2 : &tmK;
+        mbar_arrive_expect_tx(bKFull(s), C::kTileBytes);
+#pragma unroll
+        for (int blk = 0; blk < C::kBlocks; ++blk)
+          tma_load_4d(sK + s * C::kTileBytes + blk * (kTileM * 128), m, bKFull(s), blk * 64, kvh, kt.k0,
+                      kt.kc3 + b);
+      }
+      // drain: every load issued so far has landed before the CTA exits
+      for (int i = max(0, j - NS); i < j; ++i) {
+        const uint64_t t0 = global_timer_ns();
+        while (!mbar_try_wait(bKFull(i % NS), (i / NS) & 1) && global_timer_ns() - t0 < kWaitLimitNs) {
+        }
+      }
+      for (int x = 0; x < (hasB ? 2 : 1); ++x) {
+        const uint64_t t0 = global_timer_ns();
+        while (!mbar_try_wait(bQFull(x), 0) && global_timer_ns() - t0 < kWaitLimitNs) {
+        }
+      }
+    }
+  } else if (warp == 2) {
+    // ----------------------------------------------------- producer: V
+    if (lane == 0) {
+      int j = 0;
+      for (; j < nk; ++j) {
+        const int s = j % NS;
+        if (j >= NS && !mbar_wait(bVEmpty(s), ((j / NS) - 1) & 1, ab, kStatusTimeoutProducer)) break;
+        const KeyTile kt = key_tile(p, g.tg, j);
+        const CUtensorMap* m = kt.vmap ? &tmV2 : &tmV;
+        mbar_arrive_expect_tx(bVFull(s), C::kTileBytes);
+#pragma unroll
+        for (int blk = 0; blk < C::kBlocks; ++blk)
+          tma_load_4d(sV + s * C::kTileBytes + blk * (kTileM * 128), m, bVFull(s), blk * 64, kvh, kt.k0,
+                      kt.vc3 + b);
+      }
+      for (int i = max(0, j - NS); i < j; ++i) {
+        const uint64_t t0 = global_timer_ns();
+        while (!mbar_try_wait(bVFull(i % NS), (i / NS) & 1) && global_timer_ns() - t0 < kWaitLimitNs) {
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------- MMA
+    if (lane == 0) {
+      constexpr uint32_t idQK = idesc_bf16_f32(kTileM, kTileN, false, false);
+      constexpr uint32_t idPV = idesc_bf16_f32(kTileM, D, false, true);
+      // descriptors built once; the start-address field (address >> 4,
+      // 14 bits) is advanced by adding (offset >> 4), which cannot carry out
+      // of the field (shared memory < 256 KB)
+      const uint64_t dQ = sdesc_sw128(sQ, 16, 1024);
+      const uint64_t dK = sdesc_sw128(sK, 16, 1024);
+      const uint64_t dV = sdesc_sw128(sV, kTileM * 128, 1024);
+      auto issue_qk = [&](int x, int j) {
+        const uint64_t dKs = dK + static_cast<uint64_t>((j % NS) * (C::kTileBytes >> 4));
+        const uint64_t dQx = dQ + static_cast<uint64_t>(x * (C::kTileBytes >> 4));
+        const uint32_t tS = tmem + static_cast<uint32_t>(x * 128);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = ((kk >> 2) * (kTileM * 128) + (kk & 3) * 32) >> 4;
+          umma_ss(tS, dQx + off, dKs + off, idQK, kk > 0);
+        }
+        umma_commit(bSFull(x));
+      };
+      auto issue_pv = [&](int x, int j) {
+        const uint64_t dVs = dV + static_cast<uint64_t>((j % NS) * (C::kTileBytes >> 4));
+        const uint32_t tO = tmem + 256u + static_cast<uint32_t>(x * 128), tP = tmem + static_cast<uint32_t>(x * 128);
+#pragma unroll
+        for (int kk = 0; kk < kTileN / 16; ++kk)
+          umma_ts(tO, tP + kk * 8, dVs + static_cast<uint64_t>(kk * (2048 >> 4)), idPV, (j > 0 || kk > 0) ? 1u : 0u);
+        umma_commit(bPvDone(x));
+      };
+      bool ok = mbar_wait(ROPE == kRopeQ ? bQReady(0) : bQFull(0), 0, ab, kStatusTimeoutMma);
+      if (ok && hasB) ok = mbar_wait(ROPE == kRopeQ ? bQReady(1) : bQFull(1), 0, ab, kStatusTimeoutMma);
+      if (ok && nk > 0) {
+        ok = mbar_wait(bKFull(0), 0, ab, kStatusTimeoutMma);
+        if (ok) {
+          tc_fence_after();
+          issue_qk(0, 0);
+          if (hasB) issue_qk(1, 0);
+          umma_commit(bKEmpty(0));
+        }
+      }
+      for (int j = 0; ok && j < nk; ++j) {
+        const int s = j % NS;
+        const bool more = j + 1 < nk;
+        const int s1 = (j + 1) % NS;
+        // tile A: O_A += P_A V_j, then S_A = Q_A K_{j+1}^T once P_A is read
+        if (!mbar_wait(bPFull(0), j & 1, ab, kStatusTimeoutMma) ||
+            !mbar_wait(bVFull(s), (j / NS) & 1, ab, kStatusTimeoutMma)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        issue_pv(0, j);
+        if (!hasB) umma_commit(bVEmpty(s));
+        if (more) {
+          if (!mbar_wait(bKFull(s1), ((j + 1) / NS) & 1, ab, kStatusTimeoutMma) ||
+              !mbar_wait(bPvDone(0), j & 1, ab, kStatusTimeoutMma)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          issue_qk(0, j + 1);
+          if (!hasB) umma_commit(bKEmpty(s1));
+        }
+        if (hasB) {
+          // tile B: the same, half a period later
+          if (!mbar_wait(bPFull(1), j & 1, ab, kStatusTimeoutMma)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          issue_pv(1, j);
+          umma_commit(bVEmpty(s));
+          if (more) {
+            if (!mbar_wait(bPvDone(1), j & 1, ab, kStatusTimeoutMma)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            issue_qk(1, j + 1);
+            umma_commit(bKEmpty(s1));
+          }
+        }
+      }
+      // all issued MMAs complete before teardown
+      umma_commit(bFinal);
+      const uint64_t t0 = global_timer_ns();
+      while (!mbar_try_wait(bFinal, 0) && global_timer_ns() - t0 < kWaitLimitNs) {
+      }
+    }
+  } else if (warp >= 4 && warp < 12) {
+    // ---------------------------------------------------------- softmax
+    const int x = (warp - 4) >> 2;                   // query tile of this warpgroup
+    if (x == 0 || hasB) {
+      const int r = (threadIdx.x - 128) & 127;       // row of the tile = TMEM lane
+      const uint32_t trow = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
+      const uint32_t tS = trow + static_cast<uint32_t>(x * 128);
+      const uint32_t tO = trow + 256u + static_cast<uint32_t>(x * 128);
+      const int q_end = x ? g.q_end[1] : g.q_end[0];
+      const int qn = (x ? g.q0[1] : g.q0[0]) + r;
+      const bool row_valid = qn < q_end;
+      int lo = 0, hi = 0;
+      if (p.n_kseg == 0) key_range(p, row_valid ? qn : q_end - 1, lo, hi);
+      float m_run = -INFINITY, l_run = 0.f;
+      const float sl2 = p.scale_log2;
+      bool ok = true;
+      if constexpr (ROPE == kRopeQ) {
+        // rotate this thread's query row of Q_x in place, once
+        ok = mbar_wait(bQFull(x), 0, ab, kStatusTimeoutSoftmax);
+        const int Fr = p.rope_Hg * p.rope_Wg;
+        RopePos pos{0, 0, 0};
+        if (row_valid) {
+          const int in = qn % Fr;
+          pos = RopePos{p.qoff + qn / Fr, in / p.rope_Wg, in % p.rope_Wg};
+        }
+        rope_row_inplace<D>(smem + C::kOffQ + x * C::kTileBytes, r, pos, p);
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bQReady(x));
+      }
+      // No early exit: a failed wait only happens after the CTA aborted,
+      // when every later wait fails at once; the warp stays converged for
+      // the warp-collective TMEM accesses.
+      for (int j = 0; j < nk; ++j) {
+        if (!mbar_wait(bSFull(x), j & 1, ab, kStatusTimeoutSoftmax)) ok = false;
+        tc_fence_after();
+        int col_lo = 0, col_hi = kTileN;
+        if (p.n_kseg == 0) {
+          const int k0 = g.tg.kbeg + j * kTileN;
+          col_lo = lo - k0;
+          col_hi = hi - k0;
+        } else {
+          col_hi = key_tile(p, g.tg, j).valid;
+        }
+        const bool masked = col_lo > 0 || col_hi < kTileN;
+        uint32_t s0[32], s1[32], s2[32], s3[32];
+        tmem_ld32(tS, s0);
+        tmem_ld32(tS + 32, s1);
+        tmem_ld32(tS + 64, s2);
+        tmem_ld32(tS + 96, s3);
+        tmem_ld_wait_dep(s0);
+        reg_tie32(s1);
+        reg_tie32(s2);
+        reg_tie32(s3);
+        // row max over the visible columns
+        float mx8[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) mx8[i] = -INFINITY;
+        if (!masked) {
+#pragma unroll
+          for (int c = 0; c < 32; ++c) {
+            mx8[c & 7] = fmax3(mx8[c & 7], __uint_as_float(s0[c]), __uint_as_float(s1[c]));
+            mx8[c & 7] = fmax3(mx8[c & 7], __uint_as_float(s2[c]), __uint_as_float(s3[c]));
+          }
+        } else {
+#pragma unroll
+          for (int c = 0; c < 32; ++c) {
+            const float v0 = (c >= col_lo && c < col_hi) ? __uint_as_float(s0[c]) : -INFINITY;
+            const float v1 = (c + 32 >= col_lo && c + 32 < col_hi) ? __uint_as_float(s1[c]) : -INFINITY;
+            const float v2 = (c + 64 >= col_lo && c + 64 < col_hi) ? __uint_as_float(s2[c]) : -INFINITY;
+            const float v3 = (c + 96 >= col_lo && c + 96 < col_hi) ? __uint_as_float(s3[c]) : -INFINITY;
+            mx8[c & 7] = fmax3(mx8[c & 7], v0, v1);
+            mx8[c & 7] = fmax3(mx8[c & 7], v2, v3);
+          }
+        }
+        const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                               fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+        const float m_new = fmaxf(m_run, mx * sl2);
+        float factor = 1.f;
+        bool resc = false;
+        if (m_new > m_run + kRescaleThreshold) {
+          factor = ex2_approx(m_run - m_new);   // 0 when m_run = -inf
+          m_run = m_new;
+          resc = true;
+        }
+        const float nm = (m_run == -INFINITY) ? 0.f : -m_run;
+        // P = exp2(s * scale * log2e - m) into the first half of S_x, 16
+        // columns (32 keys) at a time; row sums as packed fp32x2
+        float rs2[2][2] = {{0.f, 0.f}, {0.f, 0.f}};
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const uint32_t* sq = q == 0 ? s0 : (q == 1 ? s1 : (q == 2 ? s2 : s3));
+          uint32_t pk[16];
+          if (!masked) {
+#pragma unroll
+            for (int c = 0; c < 32; c += 2) {
+              float x0, x1, p0, p1;
+              ffma2(x0, x1, __uint_as_float(sq[c]), __uint_as_float(sq[c + 1]), sl2, sl2, nm, nm);
+              if ((PolyMask<D>::value >> ((c >> 1) & 7)) & 1u) {
+                ex2_poly2(p0, p1, x0, x1);
+              } else {
+                p0 = ex2_approx(x0);
+                p1 = ex2_approx(x1);
+              }
+              fadd2(rs2[(c >> 1) & 1][0], rs2[(c >> 1) & 1][1], p0, p1);
+              pk[c / 2] = pack_bf16x2(p0, p1);
+            }
+          } else {
+#pragma unroll
+            for (int c = 0; c < 32; c += 2) {
+              const int col = q * 32 + c;
+              float p0 = ex2_approx(fmaf(__uint_as_float(sq[c]), sl2, nm));
+              float p1 = ex2_approx(fmaf(__uint_as_float(sq[c + 1]), sl2, nm));
+              p0 = (col >= col_lo && col < col_hi) ? p0 : 0.f;
+              p1 = (col + 1 >= col_lo && col + 1 < col_hi) ? p1 : 0.f;
+              rs2[(c >> 1) & 1][0] += p0;
+              rs2[(c >> 1) & 1][1] += p1;
+              pk[c / 2] = pack_bf16x2(p0, p1);
+            }
+          }
+          tmem_st16(tS + q * 16, pk);
+        }
+        const float rs = (rs2[0][0] + rs2[0][1]) + (rs2[1][0] + rs2[1][1]);
+        // O_x rescale: the previous P_x V is complete (S_x of this tile was
+        // issued after it), and the next one waits for P_x below
+        if (__any_sync(0xffffffffu, resc && j > 0)) {
+          const float f = (resc && j > 0) ? factor : 1.f;
+#pragma unroll 1
+          for (int c = 0; c < D / 32; ++c) {
+            uint32_t orr[32];
+            tmem_ld32(tO + c * 32, orr);
+            tmem_ld_wait_dep(orr);
+#pragma unroll
+            for (int e = 0; e < 32; ++e) orr[e] = __float_as_uint(__uint_as_float(orr[e]) * f);
+            tmem_st32(tO + c * 32, orr);
+          }
+        }
+        tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bPFull(x));
+        l_run = l_run * factor + rs;
+      }
+      // epilogue: O_x / l -> bf16, lse
+      if (ok && nk > 0) {
+        ok = mbar_wait(bPvDone(x), (nk - 1) & 1, ab, kStatusTimeoutSoftmax);
+        tc_fence_after();
+      }
+      ok = __all_sync(0xffffffffu, ok);   // the TMEM loads below are warp-collective
+      if (ok) {
+        const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
+        __nv_bfloat16* orow = p.o + ((static_cast<size_t>(b) * p.Lq + qn) * p.H + h) * D;
+#pragma unroll 1
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t orr[32];
+          if (nk > 0) {
+            tmem_ld32(tO + c * 32, orr);
+            tmem_ld_wait_dep(orr);
+          } else {
+#pragma unroll
+            for (int e = 0; e < 32; ++e) orr[e] = 0u;
+          }
+          uint32_t w[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e)
+            w[e] = pack_bf16x2(__uint_as_float(orr[2 * e]) * inv, __uint_as_float(orr[2 * e + 1]) * inv);
+          if (row_valid) {
+            uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) dst[e] = make_uint4(w[4 * e], w[4 * e + 1], w[4 * e + 2], w[4 * e + 3]);
+          }
+        }
+        if (p.lse && row_valid) {
+          const float lse = l_run > 0.f ? (m_run + __log2f(l_run)) * 0.69314718055994531f : -INFINITY;
+          p.lse[(static_cast<size_t>(b) * p.H + h) * p.Lq + qn] = lse;
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+}  // namespace attn
+}  // namespace vattn

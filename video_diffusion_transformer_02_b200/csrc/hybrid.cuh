@@ -37,7 +37,7 @@ struct DeltaCfg {
   static constexpr int kSmemBytes = kOffMisc + 64 + 1024;
 };
 
-// grid (C, H, B), 384 threads: warp 0 TMA, warp 1 TMEM + MMA, warps 4..11
+// grid (H, C, B), 384 threads: warp 0 TMA, warp 1 TMEM + MMA, warps 4..11
 // feature map, column sums and epilogue.  Feature-map thread t owns the
 // 16-byte chunk t % 16 (eight features) of rows t / 16 + 16 i of every tile,
 // so the column sums of its eight features stay in registers; the eight
@@ -70,7 +70,7 @@ __global__ void __launch_bounds__(kDeltaThreads, 1)
   Abort ab{abort_flag, p.status};
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int c = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  const int h = blockIdx.x, c = blockIdx.y, b = blockIdx.z;   // heads fastest: CTAs running together read whole token rows
   const int c0 = c * p.chunk;
   const int c1 = min(p.L, c0 + p.chunk);
   const int nt = (c1 - c0 + kRows - 1) / kRows;

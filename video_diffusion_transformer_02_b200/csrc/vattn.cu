@@ -12,6 +12,13 @@
 
 #include "../../include/vattn.h"
 #include "attention.cuh"
+#include "attention_pair.cuh"
+
+// 1: attention with keys already rotated (or without RoPE) runs two query
+// tiles per CTA; 0: one query tile per CTA.
+#ifndef VATTN_PAIR_TILES
+#define VATTN_PAIR_TILES 1
+#endif
 #include "hybrid.cuh"
 #include "kvcache.cuh"
 #include "rope.cuh"
@@ -158,10 +165,41 @@ vattn_status launch_attention(const CUtensorMap& q, const CUtensorMap& k, const 
   return VATTN_OK;
 }
 
+uint64_t g_pair_smem_done[4][1];
+
+// Two query tiles per CTA (attention_pair.cuh): grid = tile pairs x heads x
+// batch.
+template <int D, int ROPE>
+vattn_status launch_pair(const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v, const CUtensorMap& k2,
+                         const CUtensorMap& v2, const vattn::attn::Params& p, cudaStream_t s) {
+  using Cfg = vattn::attn::PairCfg<D>;
+  constexpr int slot = (D == 64 ? 0 : 2) + (ROPE == vattn::attn::kRopeQ ? 1 : 0);
+  auto kern = vattn::attn::attn_pair_kernel<D, ROPE>;
+  vattn_status st = ensure_smem(kern, Cfg::kSmemBytes, g_pair_smem_done[slot]);
+  if (st) return st;
+  const int segs = p.n_q_tiles / p.q_tiles_per_seg;
+  const long long pairs = static_cast<long long>(segs) * ((p.q_tiles_per_seg + 1) / 2);
+  if (pairs > 0x7fffffffLL) return fail(VATTN_ERR_UNSUPPORTED, "too many query tiles");
+  const dim3 grid(static_cast<unsigned>(pairs), p.H, p.B);
+  kern<<<grid, vattn::attn::kPairThreads, Cfg::kSmemBytes, s>>>(q, k, v, k2, v2, p);
+  VATTN_CUDA(cudaGetLastError());
+  return VATTN_OK;
+}
+
 vattn_status dispatch_attention(int d, int rope_mode, const CUtensorMap& q, const CUtensorMap& k,
                                 const CUtensorMap& v, const CUtensorMap& k2, const CUtensorMap& v2,
                                 const vattn::attn::Params& p, cudaStream_t s) {
   using namespace vattn::attn;
+#if VATTN_PAIR_TILES
+  // keys already rotated (or no RoPE): the two-tile kernel
+  if (rope_mode != kRopeQK) {
+    if (d == 64)
+      return rope_mode == kRopeQ ? launch_pair<64, kRopeQ>(q, k, v, k2, v2, p, s)
+                                 : launch_pair<64, kRopeNone>(q, k, v, k2, v2, p, s);
+    return rope_mode == kRopeQ ? launch_pair<128, kRopeQ>(q, k, v, k2, v2, p, s)
+                               : launch_pair<128, kRopeNone>(q, k, v, k2, v2, p, s);
+  }
+#endif
   if (d == 64) {
     if (rope_mode == kRopeQK) return launch_attention<64, kRopeQK, false>(q, k, v, k2, v2, p, s);
     if (rope_mode == kRopeQ) return launch_attention<64, kRopeQ, false>(q, k, v, k2, v2, p, s);
@@ -421,7 +459,7 @@ vattn_status vattn_attention(const void* q, const void* k, const void* v, void* 
   if (vattn_status st = make_map(&mq, q, d, H, Lq, B, 128)) return st;
   if (vattn_status st = make_map(&mk, k, d, Hkv, Lk, B, 128)) return st;
   if (vattn_status st = make_map(&mv, v, d, Hkv, Lk, B, 128)) return st;
-    if (rope && workspace) {
+  if (rope && workspace) {
     // rotate K once into the workspace; the kernel rotates Q tiles itself
     if (vattn_status st = launch_rope_k(k, workspace, B, Lk, Hkv, d, rope, table, k_frame_offset, stream))
       return st;
@@ -684,7 +722,7 @@ vattn_status vattn_hybrid_chunk(const void* q, const void* k, const void* v, voi
     const int smem = vattn::hyb::DeltaCfg<128>::kSmemBytes;
     if (vattn_status st = ensure_smem(kern, smem, done)) return st;
     vattn::hyb::DeltaParams dp{wsS, wsz, status, B, L, H, chunk_tokens};
-    kern<<<dim3(C, H, B), vattn::hyb::kDeltaThreads, smem, stream>>>(mk, mv, dp);
+    kern<<<dim3(H, C, B), vattn::hyb::kDeltaThreads, smem, stream>>>(mk, mv, dp);
     VATTN_CUDA(cudaGetLastError());
   }
   // (2) exclusive scan over chunks (+ state out)
