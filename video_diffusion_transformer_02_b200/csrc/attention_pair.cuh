@@ -2,22 +2,25 @@
 // per CTA.  Same operation, modes, masks and RoPE placement as
 // attn_fwd_kernel (see attention.cuh); what changes is the schedule:
 //
-//   * one softmax warpgroup per query tile, each thread owning a whole
-//     128-key row of S (no row-max exchange between warpgroups);
-//   * the MMA thread alternates between the tiles, so the tensor core works
-//     on one tile's S = Q K^T / O += P V while the other tile's softmax runs
-//     (the FlashAttention-4 ping-pong for Blackwell);
-//   * every K and V tile is loaded into shared memory once for both query
-//     tiles (half the L2 -> shared-memory traffic of one tile per CTA).
+//   * one softmax warpgroup per query tile, each thread owning a whole row
+//     of a score tile (no row-max exchange between warpgroups);
+//   * scores are computed in 64-key sub-tiles, double-buffered in TMEM per
+//     query tile, so S_X(j+1) = Q_X K_{j+1}^T runs on the tensor core while
+//     the softmax of S_X(j) runs, and the MMA thread interleaves both tiles
+//     (FlashAttention-4-style ping-pong on Blackwell);
+//   * every K and V stage (128 keys, two sub-tiles) is loaded into shared
+//     memory once for both query tiles.
 //
-// Warp roles: warp 0 TMA Q_A, Q_B, then K tiles; warp 1 TMEM allocation and
-// tcgen05.mma issue; warp 2 TMA V tiles; warps 4..7 softmax of tile A,
-// warps 8..11 softmax of tile B (thread r owns query row r = TMEM lane r).
+// Warp roles: warp 0 TMA Q_A, Q_B, then K stages; warp 1 TMEM allocation and
+// tcgen05.mma issue for tile A; warp 2 TMA V stages; warp 3 tcgen05.mma issue
+// for tile B; warps 4..7 softmax of tile A, warps 8..11 softmax of tile B
+// (thread r owns query row r = TMEM lane r).
 //
-// TMEM columns (512): S_A [0,128), S_B [128,256) fp32; O_A [256,256+D),
-// O_B [384,384+D) fp32.  P_X (bf16 pairs, 64 columns) overwrites the first
-// half of S_X once the softmax holds S_X in registers; the MMA thread issues
-// the next S_X = Q_X K^T only after the P_X V that reads P_X has completed.
+// TMEM columns (512): S_X buffer b at [128 x + 64 b, +64) fp32 for tiles
+// x = A, B and b = 0, 1; O_A [256, 256+D), O_B [384, 384+D) fp32.  P (bf16
+// pairs, 32 columns) overwrites the first half of its S buffer once the
+// softmax holds the scores in registers; the MMA thread reuses a buffer for
+// sub-tile j+2 only after the P V of sub-tile j has completed.
 #pragma once
 #include "attention.cuh"
 
@@ -33,7 +36,7 @@ struct PairCfg {
   static constexpr int kOffK = 2 * kTileBytes;
   static constexpr int kOffV = kOffK + kStages * kTileBytes;
   static constexpr int kOffBar = kOffV + kStages * kTileBytes;
-  static constexpr int kNumBars = 4 + 4 * kStages + 6 + 1;
+  static constexpr int kNumBars = 4 + 4 * kStages + 12 + 2;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
   static constexpr int kSmemBytes = kOffMisc + 64;
 };
@@ -91,6 +94,8 @@ __global__ void __launch_bounds__(kPairThreads, 1)
   static_assert(ROPE == kRopeNone || ROPE == kRopeQ, "keys are rotated before this kernel");
   using C = PairCfg<D>;
   constexpr int NS = C::kStages;
+  constexpr int kSub = kTileN / 2;                 // keys per score sub-tile
+  constexpr uint32_t kSubBytes = kSub * 128;       // sub-tile offset inside a 64-column block
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = smem_raw;
   const uint32_t sbase = smem_addr(smem);
@@ -107,10 +112,11 @@ __global__ void __launch_bounds__(kPairThreads, 1)
   auto bVFull = [&](int s) { return bar0 + 32 + 8 * (2 * NS + s); };
   auto bVEmpty = [&](int s) { return bar0 + 32 + 8 * (3 * NS + s); };
   const uint32_t bx = bar0 + 32 + 32 * NS;
-  auto bSFull = [&](int x) { return bx + 8 * x; };
-  auto bPFull = [&](int x) { return bx + 16 + 8 * x; };
-  auto bPvDone = [&](int x) { return bx + 32 + 8 * x; };
-  const uint32_t bFinal = bx + 48;
+  auto bSFull = [&](int x, int b) { return bx + 8 * (2 * x + b); };
+  auto bPFull = [&](int x, int b) { return bx + 32 + 8 * (2 * x + b); };
+  auto bPvDone = [&](int x) { return bx + 64 + 8 * x; };
+  auto bODone = [&](int x) { return bx + 80 + 8 * x; };   // last P V of the tile complete
+  auto bFinal = [&](int x) { return bx + 96 + 8 * x; };     // all MMAs of issuer x complete
   uint32_t* misc = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
   volatile uint32_t* tmem_slot = misc;
   volatile uint32_t* abort_flag = misc + 1;
@@ -122,24 +128,30 @@ __global__ void __launch_bounds__(kPairThreads, 1)
   const int pr = p.reverse_q ? static_cast<int>(gridDim.x - 1 - blockIdx.x) : static_cast<int>(blockIdx.x);
   const PairGeom g = pair_geom(p, pr);
   if (g.q0[0] >= g.q_end[0]) return;   // pair past the end of a short last segment
-  const int nk = g.tg.n_tiles;
+  const int nk = g.tg.n_tiles;          // 128-key stages
+  const int ns = 2 * nk;                // 64-key score sub-tiles
   const bool hasB = g.hasB;
 
   if (threadIdx.x == 0) {
     for (int x = 0; x < 2; ++x) {
       mbar_init(bQFull(x), 1);
       mbar_init(bQReady(x), 4);
-      mbar_init(bSFull(x), 1);
-      mbar_init(bPFull(x), 4);
       mbar_init(bPvDone(x), 1);
+      mbar_init(bODone(x), 1);
+      for (int bb = 0; bb < 2; ++bb) {
+        mbar_init(bSFull(x, bb), 1);
+        mbar_init(bPFull(x, bb), 4);
+      }
     }
+    // a stage is released once by the MMA issuer of each query tile
     for (int s = 0; s < NS; ++s) {
       mbar_init(bKFull(s), 1);
-      mbar_init(bKEmpty(s), 1);
+      mbar_init(bKEmpty(s), hasB ? 2 : 1);
       mbar_init(bVFull(s), 1);
-      mbar_init(bVEmpty(s), 1);
+      mbar_init(bVEmpty(s), hasB ? 2 : 1);
     }
-    mbar_init(bFinal, 1);
+    mbar_init(bFinal(0), 1);
+    mbar_init(bFinal(1), 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -212,94 +224,80 @@ __global__ void __launch_bounds__(kPairThreads, 1)
         }
       }
     }
-  } else if (warp == 1) {
+  } else if (warp == 1 || warp == 3) {
     // ------------------------------------------------------------- MMA
-    if (lane == 0) {
-      constexpr uint32_t idQK = idesc_bf16_f32(kTileM, kTileN, false, false);
+    // one issuing thread per query tile: warp 1 for A, warp 3 for B
+    const int x = warp == 1 ? 0 : 1;
+    if (lane == 0 && (x == 0 || hasB)) {
+      constexpr uint32_t idQK = idesc_bf16_f32(kTileM, kSub, false, false);
       constexpr uint32_t idPV = idesc_bf16_f32(kTileM, D, false, true);
-      // descriptors built once; the start-address field (address >> 4,
-      // 14 bits) is advanced by adding (offset >> 4), which cannot carry out
-      // of the field (shared memory < 256 KB)
-      const uint64_t dQ = sdesc_sw128(sQ, 16, 1024);
+      // descriptors built once; a K step or a sub-tile adds a constant to
+      // the start-address field (address >> 4, 14 bits), which cannot carry
+      // out of the field (shared memory < 256 KB)
+      const uint64_t dQx = sdesc_sw128(sQ + x * C::kTileBytes, 16, 1024);
       const uint64_t dK = sdesc_sw128(sK, 16, 1024);
       const uint64_t dV = sdesc_sw128(sV, kTileM * 128, 1024);
-      auto issue_qk = [&](int x, int j) {
-        const uint64_t dKs = dK + static_cast<uint64_t>((j % NS) * (C::kTileBytes >> 4));
-        const uint64_t dQx = dQ + static_cast<uint64_t>(x * (C::kTileBytes >> 4));
-        const uint32_t tS = tmem + static_cast<uint32_t>(x * 128);
+      const uint32_t tSx = tmem + static_cast<uint32_t>(x * 128);
+      const uint32_t tOx = tmem + 256u + static_cast<uint32_t>(x * 128);
+      // start-address step (>> 4) of sub-tile u: stage (u / 2) % NS, half u % 2
+      auto sub_step = [](int u) -> uint64_t {
+        return static_cast<uint64_t>(((u >> 1) & (NS - 1)) * (C::kTileBytes >> 4) + (u & 1) * (kSubBytes >> 4));
+      };
+      // S_x(u) = Q_x K(u)^T into S buffer u & 1
+      auto issue_qk = [&](int u) {
+        const uint64_t dk = dK + sub_step(u);
+        const uint32_t tS = tSx + static_cast<uint32_t>((u & 1) * kSub);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = ((kk >> 2) * (kTileM * 128) + (kk & 3) * 32) >> 4;
-          umma_ss(tS, dQx + off, dKs + off, idQK, kk > 0);
+          umma_ss(tS, dQx + off, dk + off, idQK, kk > 0);
         }
-        umma_commit(bSFull(x));
+        umma_commit(bSFull(x, u & 1));
       };
-      auto issue_pv = [&](int x, int j) {
-        const uint64_t dVs = dV + static_cast<uint64_t>((j % NS) * (C::kTileBytes >> 4));
-        const uint32_t tO = tmem + 256u + static_cast<uint32_t>(x * 128), tP = tmem + static_cast<uint32_t>(x * 128);
+      // O_x += P_x(u) V(u), P_x(u) in the first half of S buffer u & 1
+      auto issue_pv = [&](int u) {
+        const uint64_t dv = dV + sub_step(u);
+        const uint32_t tP = tSx + static_cast<uint32_t>((u & 1) * kSub);
+        const uint32_t acc0 = u > 0 ? 1u : 0u;
 #pragma unroll
-        for (int kk = 0; kk < kTileN / 16; ++kk)
-          umma_ts(tO, tP + kk * 8, dVs + static_cast<uint64_t>(kk * (2048 >> 4)), idPV, (j > 0 || kk > 0) ? 1u : 0u);
+        for (int kk = 0; kk < kSub / 16; ++kk)
+          umma_ts(tOx, tP + kk * 8, dv + static_cast<uint64_t>(kk * (2048 >> 4)), idPV, kk > 0 ? 1u : acc0);
         umma_commit(bPvDone(x));
       };
-      bool ok = mbar_wait(ROPE == kRopeQ ? bQReady(0) : bQFull(0), 0, ab, kStatusTimeoutMma);
-      if (ok && hasB) ok = mbar_wait(ROPE == kRopeQ ? bQReady(1) : bQFull(1), 0, ab, kStatusTimeoutMma);
+      bool ok = mbar_wait(ROPE == kRopeQ ? bQReady(x) : bQFull(x), 0, ab, kStatusTimeoutMma);
       if (ok && nk > 0) {
         ok = mbar_wait(bKFull(0), 0, ab, kStatusTimeoutMma);
         if (ok) {
           tc_fence_after();
-          issue_qk(0, 0);
-          if (hasB) issue_qk(1, 0);
-          umma_commit(bKEmpty(0));
+          issue_qk(0);
         }
       }
-      for (int j = 0; ok && j < nk; ++j) {
-        const int s = j % NS;
-        const bool more = j + 1 < nk;
-        const int s1 = (j + 1) % NS;
-        // tile A: O_A += P_A V_j, then S_A = Q_A K_{j+1}^T once P_A is read
-        if (!mbar_wait(bPFull(0), j & 1, ab, kStatusTimeoutMma) ||
-            !mbar_wait(bVFull(s), (j / NS) & 1, ab, kStatusTimeoutMma)) {
-          ok = false;
-          break;
+      // per sub-tile u: S_x(u + 1) into the buffer that P_x(u - 1) V released,
+      // then O_x += P_x(u) V(u) once the softmax has published P_x(u); the
+      // tensor core computes the next scores while the softmax works
+      for (int u = 0; ok && u < ns; ++u) {
+        const int un = u + 1;
+        if (un < ns) {
+          const int stn = (un >> 1) & (NS - 1);
+          // a stage is waited for at its first sub-tile only
+          if (!(un & 1) && !mbar_wait(bKFull(stn), ((un >> 1) / NS) & 1, ab, kStatusTimeoutMma)) break;
+          if (u > 0 && !mbar_wait(bPvDone(x), (u - 1) & 1, ab, kStatusTimeoutMma)) break;
+          tc_fence_after();
+          issue_qk(un);
+          if (un & 1) umma_commit(bKEmpty(stn));   // both sub-tiles of the stage issued
         }
+        const int st = (u >> 1) & (NS - 1);
+        if (!(u & 1) && !mbar_wait(bVFull(st), ((u >> 1) / NS) & 1, ab, kStatusTimeoutMma)) break;
+        if (!mbar_wait(bPFull(x, u & 1), (u >> 1) & 1, ab, kStatusTimeoutMma)) break;
         tc_fence_after();
-        issue_pv(0, j);
-        if (!hasB) umma_commit(bVEmpty(s));
-        if (more) {
-          if (!mbar_wait(bKFull(s1), ((j + 1) / NS) & 1, ab, kStatusTimeoutMma) ||
-              !mbar_wait(bPvDone(0), j & 1, ab, kStatusTimeoutMma)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          issue_qk(0, j + 1);
-          if (!hasB) umma_commit(bKEmpty(s1));
-        }
-        if (hasB) {
-          // tile B: the same, half a period later
-          if (!mbar_wait(bPFull(1), j & 1, ab, kStatusTimeoutMma)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          issue_pv(1, j);
-          umma_commit(bVEmpty(s));
-          if (more) {
-            if (!mbar_wait(bPvDone(1), j & 1, ab, kStatusTimeoutMma)) {
-              ok = false;
-              break;
-            }
-            tc_fence_after();
-            issue_qk(1, j + 1);
-            umma_commit(bKEmpty(s1));
-          }
-        }
+        issue_pv(u);
+        if (u == ns - 1) umma_commit(bODone(x));
+        if (u & 1) umma_commit(bVEmpty(st));
       }
       // all issued MMAs complete before teardown
-      umma_commit(bFinal);
+      umma_commit(bFinal(x));
       const uint64_t t0 = global_timer_ns();
-      while (!mbar_try_wait(bFinal, 0) && global_timer_ns() - t0 < kWaitLimitNs) {
+      while (!mbar_try_wait(bFinal(x), 0) && global_timer_ns() - t0 < kWaitLimitNs) {
       }
     }
   } else if (warp >= 4 && warp < 12) {
@@ -308,7 +306,6 @@ __global__ void __launch_bounds__(kPairThreads, 1)
     if (x == 0 || hasB) {
       const int r = (threadIdx.x - 128) & 127;       // row of the tile = TMEM lane
       const uint32_t trow = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
-      const uint32_t tS = trow + static_cast<uint32_t>(x * 128);
       const uint32_t tO = trow + 256u + static_cast<uint32_t>(x * 128);
       const int q_end = x ? g.q_end[1] : g.q_end[0];
       const int qn = (x ? g.q0[1] : g.q0[0]) + r;
@@ -318,6 +315,7 @@ __global__ void __launch_bounds__(kPairThreads, 1)
       float m_run = -INFINITY, l_run = 0.f;
       const float sl2 = p.scale_log2;
       bool ok = true;
+      int pv_seen = 0;   // completions of bPvDone(x) known to this thread
       if constexpr (ROPE == kRopeQ) {
         // rotate this thread's query row of Q_x in place, once
         ok = mbar_wait(bQFull(x), 0, ab, kStatusTimeoutSoftmax);
@@ -335,46 +333,39 @@ __global__ void __launch_bounds__(kPairThreads, 1)
       // No early exit: a failed wait only happens after the CTA aborted,
       // when every later wait fails at once; the warp stays converged for
       // the warp-collective TMEM accesses.
-      for (int j = 0; j < nk; ++j) {
-        if (!mbar_wait(bSFull(x), j & 1, ab, kStatusTimeoutSoftmax)) ok = false;
+      for (int u = 0; u < ns; ++u) {
+        const int bb = u & 1;
+        if (!mbar_wait(bSFull(x, bb), (u >> 1) & 1, ab, kStatusTimeoutSoftmax)) ok = false;
         tc_fence_after();
-        int col_lo = 0, col_hi = kTileN;
+        const uint32_t tS = trow + static_cast<uint32_t>(x * 128 + bb * kSub);
+        int col_lo = 0, col_hi = kSub;
         if (p.n_kseg == 0) {
-          const int k0 = g.tg.kbeg + j * kTileN;
+          const int k0 = g.tg.kbeg + u * kSub;
           col_lo = lo - k0;
           col_hi = hi - k0;
         } else {
-          col_hi = key_tile(p, g.tg, j).valid;
+          col_hi = key_tile(p, g.tg, u >> 1).valid - bb * kSub;
         }
-        const bool masked = col_lo > 0 || col_hi < kTileN;
-        uint32_t s0[32], s1[32], s2[32], s3[32];
+        const bool masked = col_lo > 0 || col_hi < kSub;
+        uint32_t s0[32], s1[32];
         tmem_ld32(tS, s0);
         tmem_ld32(tS + 32, s1);
-        tmem_ld32(tS + 64, s2);
-        tmem_ld32(tS + 96, s3);
         tmem_ld_wait_dep(s0);
         reg_tie32(s1);
-        reg_tie32(s2);
-        reg_tie32(s3);
         // row max over the visible columns
         float mx8[8];
 #pragma unroll
         for (int i = 0; i < 8; ++i) mx8[i] = -INFINITY;
         if (!masked) {
 #pragma unroll
-          for (int c = 0; c < 32; ++c) {
+          for (int c = 0; c < 32; ++c)
             mx8[c & 7] = fmax3(mx8[c & 7], __uint_as_float(s0[c]), __uint_as_float(s1[c]));
-            mx8[c & 7] = fmax3(mx8[c & 7], __uint_as_float(s2[c]), __uint_as_float(s3[c]));
-          }
         } else {
 #pragma unroll
           for (int c = 0; c < 32; ++c) {
             const float v0 = (c >= col_lo && c < col_hi) ? __uint_as_float(s0[c]) : -INFINITY;
             const float v1 = (c + 32 >= col_lo && c + 32 < col_hi) ? __uint_as_float(s1[c]) : -INFINITY;
-            const float v2 = (c + 64 >= col_lo && c + 64 < col_hi) ? __uint_as_float(s2[c]) : -INFINITY;
-            const float v3 = (c + 96 >= col_lo && c + 96 < col_hi) ? __uint_as_float(s3[c]) : -INFINITY;
             mx8[c & 7] = fmax3(mx8[c & 7], v0, v1);
-            mx8[c & 7] = fmax3(mx8[c & 7], v2, v3);
           }
         }
         const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
@@ -388,12 +379,12 @@ __global__ void __launch_bounds__(kPairThreads, 1)
           resc = true;
         }
         const float nm = (m_run == -INFINITY) ? 0.f : -m_run;
-        // P = exp2(s * scale * log2e - m) into the first half of S_x, 16
-        // columns (32 keys) at a time; row sums as packed fp32x2
+        // P = exp2(s * scale * log2e - m) into the first half of the S
+        // buffer, 16 columns (32 keys) at a time; row sums as packed fp32x2
         float rs2[2][2] = {{0.f, 0.f}, {0.f, 0.f}};
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const uint32_t* sq = q == 0 ? s0 : (q == 1 ? s1 : (q == 2 ? s2 : s3));
+        for (int q = 0; q < 2; ++q) {
+          const uint32_t* sq = q == 0 ? s0 : s1;
           uint32_t pk[16];
           if (!masked) {
 #pragma unroll
@@ -425,10 +416,15 @@ __global__ void __launch_bounds__(kPairThreads, 1)
           tmem_st16(tS + q * 16, pk);
         }
         const float rs = (rs2[0][0] + rs2[0][1]) + (rs2[1][0] + rs2[1][1]);
-        // O_x rescale: the previous P_x V is complete (S_x of this tile was
-        // issued after it), and the next one waits for P_x below
-        if (__any_sync(0xffffffffu, resc && j > 0)) {
-          const float f = (resc && j > 0) ? factor : 1.f;
+        // O_x rescale: wait until the P V of the previous sub-tile (which
+        // accumulates into O_x) has completed; the next one waits for P below
+        if (__any_sync(0xffffffffu, resc && u > 0)) {
+          if (pv_seen < u) {
+            if (!mbar_wait(bPvDone(x), (u - 1) & 1, ab, kStatusTimeoutSoftmax)) ok = false;
+            pv_seen = u;
+            tc_fence_after();
+          }
+          const float f = (resc && u > 0) ? factor : 1.f;
 #pragma unroll 1
           for (int c = 0; c < D / 32; ++c) {
             uint32_t orr[32];
@@ -442,12 +438,14 @@ __global__ void __launch_bounds__(kPairThreads, 1)
         tmem_st_wait();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(bPFull(x));
+        if (lane == 0) mbar_arrive(bPFull(x, bb));
         l_run = l_run * factor + rs;
       }
       // epilogue: O_x / l -> bf16, lse
-      if (ok && nk > 0) {
-        ok = mbar_wait(bPvDone(x), (nk - 1) & 1, ab, kStatusTimeoutSoftmax);
+      if (ok && ns > 0) {
+        // bPvDone may still be two completions short here; bODone completes
+        // exactly once, after the last P V of this tile
+        ok = mbar_wait(bODone(x), 0, ab, kStatusTimeoutSoftmax);
         tc_fence_after();
       }
       ok = __all_sync(0xffffffffu, ok);   // the TMEM loads below are warp-collective
@@ -457,7 +455,7 @@ __global__ void __launch_bounds__(kPairThreads, 1)
 #pragma unroll 1
         for (int c = 0; c < D / 32; ++c) {
           uint32_t orr[32];
-          if (nk > 0) {
+          if (ns > 0) {
             tmem_ld32(tO + c * 32, orr);
             tmem_ld_wait_dep(orr);
           } else {
