@@ -38,6 +38,7 @@ import seeded_inputs as si  # noqa: E402
 METRIC = "attention TFLOPS (mask-adjusted) & % of B200 BF16 peak; streaming frames/s"
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 KERNEL_SOURCES = ["video_diffusion_transformer_02_b200/csrc/attention.cuh",
+                  "video_diffusion_transformer_02_b200/csrc/attention_pair.cuh",
                   "video_diffusion_transformer_02_b200/csrc/sm100.cuh"]
 
 
@@ -271,7 +272,7 @@ def run_ours(args, rank, world, device):
         roofline={"bound": "tensor", "achieved": achieved, "peak": pk["bf16_tflops"],
                   "unit": "TFLOP/s", "frac": achieved / pk["bf16_tflops"],
                   "frac_of_sustained": achieved / pk.get("bf16_tflops_sustained", pk["bf16_tflops"]),
-                  "peak_source": src + " (burst bf16 GEMM)", "kernel": "attn_fwd_kernel<128,rope-q,0>",
+                  "peak_source": src + " (burst bf16 GEMM)", "kernel": "attn_pair_kernel<128,rope-q>",
                   "kernel_ms": kernel_ms, "rope_k_ms": rope_ms, "traffic": recorded_traffic()},
         cpu_baseline=cpu,
         e2e={"value": w["flops"] / (e2e_ms / 1e3) / 1e12 * world, "unit": "TFLOP/s",

@@ -265,6 +265,11 @@ __global__ void __launch_bounds__(kPairThreads, 1)
         umma_commit(bPvDone(x));
       };
       bool ok = mbar_wait(ROPE == kRopeQ ? bQReady(x) : bQFull(x), 0, ab, kStatusTimeoutMma);
+      // tile B starts once tile A has published its first P, so the two
+      // softmax warpgroups work half a period apart (measured faster than
+      // starting both together: their exponentials and TMEM traffic then
+      // overlap the other tile's MMAs instead of each other)
+      if (x == 1 && ok && nk > 0) ok = mbar_wait(bPFull(0, 0), 0, ab, kStatusTimeoutMma);
       if (ok && nk > 0) {
         ok = mbar_wait(bKFull(0), 0, ab, kStatusTimeoutMma);
         if (ok) {
