@@ -62,7 +62,7 @@ def kernel_hash() -> str:
 def recorded_traffic():
     """DRAM bytes per launch of the attention kernel from the committed ncu
     summary, if it was taken on the current kernel source (else None)."""
-    p = os.path.join(ROOT, "profiles", "attn_fwd_traffic.txt")
+    p = os.path.join(ROOT, "profiles", "attn_pair_traffic.txt")
     if not os.path.exists(p):
         return None
     vals = {}
