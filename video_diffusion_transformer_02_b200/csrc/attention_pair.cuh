@@ -36,7 +36,7 @@ struct PairCfg {
   static constexpr int kOffK = 2 * kTileBytes;
   static constexpr int kOffV = kOffK + kStages * kTileBytes;
   static constexpr int kOffBar = kOffV + kStages * kTileBytes;
-  static constexpr int kNumBars = 4 + 4 * kStages + 12 + 2;
+  static constexpr int kNumBars = 4 + 4 * kStages + 12 + 2 + 5;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
   static constexpr int kSmemBytes = kOffMisc + 64;
 };
@@ -86,12 +86,13 @@ __device__ __forceinline__ void reg_tie32(uint32_t (&r)[32]) {
   asm volatile("" : VATTN_RW8(0), VATTN_RW8(8), VATTN_RW8(16), VATTN_RW8(24));
 }
 
-template <int D, int ROPE>
+template <int D, int ROPE, bool HYB>
 __global__ void __launch_bounds__(kPairThreads, 1)
     attn_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                      const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmK2,
                      const __grid_constant__ CUtensorMap tmV2, const Params p) {
   static_assert(ROPE == kRopeNone || ROPE == kRopeQ, "keys are rotated before this kernel");
+  static_assert(!HYB || (D == 128 && ROPE == kRopeNone), "hybrid: head dim 128, no RoPE");
   using C = PairCfg<D>;
   constexpr int NS = C::kStages;
   constexpr int kSub = kTileN / 2;                 // keys per score sub-tile
@@ -117,6 +118,10 @@ __global__ void __launch_bounds__(kPairThreads, 1)
   auto bPvDone = [&](int x) { return bx + 64 + 8 * x; };
   auto bODone = [&](int x) { return bx + 80 + 8 * x; };   // last P V of the tile complete
   auto bFinal = [&](int x) { return bx + 96 + 8 * x; };     // all MMAs of issuer x complete
+  // hybrid read-out: phi(Q_x) in place of Q_x, S_c (bf16 hi / lo) in the K stages, phi(Q_x) S_c
+  auto bPhiReady = [&](int x) { return bx + 112 + 8 * x; };
+  const uint32_t bScReady = bx + 128;
+  auto bLinDone = [&](int x) { return bx + 136 + 8 * x; };
   uint32_t* misc = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
   volatile uint32_t* tmem_slot = misc;
   volatile uint32_t* abort_flag = misc + 1;
@@ -152,6 +157,11 @@ __global__ void __launch_bounds__(kPairThreads, 1)
     }
     mbar_init(bFinal(0), 1);
     mbar_init(bFinal(1), 1);
+    mbar_init(bPhiReady(0), 4);
+    mbar_init(bPhiReady(1), 4);
+    mbar_init(bScReady, hasB ? 8 : 4);
+    mbar_init(bLinDone(0), 1);
+    mbar_init(bLinDone(1), 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -280,7 +290,8 @@ __global__ void __launch_bounds__(kPairThreads, 1)
       // per sub-tile u: S_x(u + 1) into the buffer that P_x(u - 1) V released,
       // then O_x += P_x(u) V(u) once the softmax has published P_x(u); the
       // tensor core computes the next scores while the softmax works
-      for (int u = 0; ok && u < ns; ++u) {
+      int u = 0;
+      for (; ok && u < ns; ++u) {
         const int un = u + 1;
         if (un < ns) {
           const int stn = (un >> 1) & (NS - 1);
@@ -298,6 +309,28 @@ __global__ void __launch_bounds__(kPairThreads, 1)
         issue_pv(u);
         if (u == ns - 1) umma_commit(bODone(x));
         if (u & 1) umma_commit(bVEmpty(st));
+      }
+      if constexpr (HYB) {
+        // linear read-out phi(Q_x) S_c into the S buffers of tile x (free
+        // after the last P V): A = phi(Q_x) K-major in place of Q_x, B = S_c
+        // split into bf16 hi and lo parts, MN-major, in the K stages
+        if (ok && u == ns && mbar_wait(bPhiReady(x), 0, ab, kStatusTimeoutMma) &&
+            mbar_wait(bScReady, 0, ab, kStatusTimeoutMma)) {
+          tc_fence_after();
+          const uint64_t dHi = sdesc_sw128(sK, D * 128, 1024);
+          const uint64_t dLo = sdesc_sw128(sK + D * D * 2, D * 128, 1024);
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t off = ((kk >> 2) * (kTileM * 128) + (kk & 3) * 32) >> 4;
+            umma_ss(tSx, dQx + off, dHi + static_cast<uint64_t>(kk * (2048 >> 4)), idPV, kk > 0);
+          }
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t off = ((kk >> 2) * (kTileM * 128) + (kk & 3) * 32) >> 4;
+            umma_ss(tSx, dQx + off, dLo + static_cast<uint64_t>(kk * (2048 >> 4)), idPV, 1u);
+          }
+          umma_commit(bLinDone(x));
+        }
       }
       // all issued MMAs complete before teardown
       umma_commit(bFinal(x));
@@ -446,6 +479,76 @@ __global__ void __launch_bounds__(kPairThreads, 1)
         if (lane == 0) mbar_arrive(bPFull(x, bb));
         l_run = l_run * factor + rs;
       }
+      float dl = 0.f;   // hybrid: phi(q_r) . z_c
+      if constexpr (HYB) {
+        // the Q tiles and the K / V stages are free once both tiles' last
+        // P V (and so every MMA reading them) has completed
+        bool okh = ok && ns > 0 && mbar_wait(bODone(0), 0, ab, kStatusTimeoutSoftmax) &&
+                   (!hasB || mbar_wait(bODone(1), 0, ab, kStatusTimeoutSoftmax));
+        tc_fence_after();
+        const int c = g.q0[0] / p.q_seg_len;   // the pair's chunk
+        // phi(q_r) = elu(q_r) + 1 in place of row r of Q_x (bf16), and phi(q_r) . z_c in fp32
+        const float* zc = p.hyb_z + ((static_cast<size_t>(c) * p.B + b) * p.H + h) * D;
+        const uint32_t qrow = sQ + static_cast<uint32_t>(x * C::kTileBytes);
+#pragma unroll 1
+        for (int blk = 0; blk < D / 64; ++blk) {
+#pragma unroll 2
+          for (int c8 = 0; c8 < 8; ++c8) {
+            const uint32_t addr = qrow + blk * (kTileM * 128) + sw128_offset(r, c8);
+            const uint4 v = lds128(addr);
+            const float4 z0 = __ldg(reinterpret_cast<const float4*>(zc + blk * 64 + c8 * 8));
+            const float4 z1 = __ldg(reinterpret_cast<const float4*>(zc + blk * 64 + c8 * 8 + 4));
+            const float zz[8] = {z0.x, z0.y, z0.z, z0.w, z1.x, z1.y, z1.z, z1.w};
+            uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              float x0 = bf16lo_to_f32(w4[e]), x1 = bf16hi_to_f32(w4[e]);
+              x0 = x0 > 0.f ? x0 + 1.f : __expf(x0);
+              x1 = x1 > 0.f ? x1 + 1.f : __expf(x1);
+              dl = fmaf(x0, zz[2 * e], dl);
+              dl = fmaf(x1, zz[2 * e + 1], dl);
+              w4[e] = pack_bf16x2(x0, x1);
+            }
+            sts128(addr, make_uint4(w4[0], w4[1], w4[2], w4[3]));
+          }
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bPhiReady(x));
+        // S_c (fp32 [D][D], row a = key feature) -> bf16 hi + lo, MN-major
+        // 128B-swizzled B operand tiles (64-column blocks of D rows) in the K
+        // stages; with two tiles, warpgroup x converts rows [64 x, 64 x + 64),
+        // thread r the column half r / 64
+        {
+          const int a = hasB ? x * 64 + (r & 63) : r;
+          const int h0 = hasB ? (r >> 6) : 0, h1 = hasB ? h0 + 1 : 2;
+          const float* src = p.hyb_S + (((static_cast<size_t>(c) * p.B + b) * p.H + h) * D + a) * D;
+#pragma unroll 1
+          for (int half = h0; half < h1; ++half) {
+#pragma unroll 2
+            for (int c8 = 0; c8 < 8; ++c8) {
+              const float4 a0 = __ldg(reinterpret_cast<const float4*>(src + half * 64 + c8 * 8));
+              const float4 a1 = __ldg(reinterpret_cast<const float4*>(src + half * 64 + c8 * 8 + 4));
+              const float xs[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+              uint32_t hi4[4], lo4[4];
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                hi4[e] = pack_bf16x2(xs[2 * e], xs[2 * e + 1]);
+                lo4[e] = pack_bf16x2(xs[2 * e] - bf16lo_to_f32(hi4[e]), xs[2 * e + 1] - bf16hi_to_f32(hi4[e]));
+              }
+              const uint32_t off = half * (D * 128) + sw128_offset(a, c8);
+              sts128(sK + off, make_uint4(hi4[0], hi4[1], hi4[2], hi4[3]));
+              sts128(sK + D * D * 2 + off, make_uint4(lo4[0], lo4[1], lo4[2], lo4[3]));
+            }
+          }
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bScReady);
+        okh = okh && mbar_wait(bLinDone(x), 0, ab, kStatusTimeoutSoftmax);
+        tc_fence_after();
+        ok = okh;
+      }
       // epilogue: O_x / l -> bf16, lse
       if (ok && ns > 0) {
         // bPvDone may still be two completions short here; bODone completes
@@ -455,7 +558,13 @@ __global__ void __launch_bounds__(kPairThreads, 1)
       }
       ok = __all_sync(0xffffffffu, ok);   // the TMEM loads below are warp-collective
       if (ok) {
-        const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
+        // hybrid: o = (2^m O + lin) / (2^m l + phi(q).z) with O, l relative
+        // to the softmax's reference max m; scaled by 2^-m when m > 0, so
+        // neither factor overflows
+        const float as = (HYB && m_run <= 0.f) ? ex2_approx(m_run) : 1.f;   // 0 when m = -inf
+        const float fl = HYB ? (m_run > 0.f ? ex2_approx(-m_run) : 1.f) : 0.f;
+        const float den = as * l_run + fl * dl;
+        const float inv = den > 0.f ? 1.f / den : 0.f;
         __nv_bfloat16* orow = p.o + ((static_cast<size_t>(b) * p.Lq + qn) * p.H + h) * D;
 #pragma unroll 1
         for (int c = 0; c < D / 32; ++c) {
@@ -463,6 +572,14 @@ __global__ void __launch_bounds__(kPairThreads, 1)
           if (ns > 0) {
             tmem_ld32(tO + c * 32, orr);
             tmem_ld_wait_dep(orr);
+            if constexpr (HYB) {
+              uint32_t lin[32];
+              tmem_ld32(trow + static_cast<uint32_t>(x * 128 + c * 32), lin);
+              tmem_ld_wait_dep(lin);
+#pragma unroll
+              for (int e = 0; e < 32; ++e)
+                orr[e] = __float_as_uint(fmaf(fl, __uint_as_float(lin[e]), as * __uint_as_float(orr[e])));
+            }
           } else {
 #pragma unroll
             for (int e = 0; e < 32; ++e) orr[e] = 0u;

@@ -165,16 +165,16 @@ vattn_status launch_attention(const CUtensorMap& q, const CUtensorMap& k, const 
   return VATTN_OK;
 }
 
-uint64_t g_pair_smem_done[4][1];
+uint64_t g_pair_smem_done[5][1];
 
 // Two query tiles per CTA (attention_pair.cuh): grid = tile pairs x heads x
 // batch.
-template <int D, int ROPE>
+template <int D, int ROPE, bool HYB = false>
 vattn_status launch_pair(const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v, const CUtensorMap& k2,
                          const CUtensorMap& v2, const vattn::attn::Params& p, cudaStream_t s) {
   using Cfg = vattn::attn::PairCfg<D>;
-  constexpr int slot = (D == 64 ? 0 : 2) + (ROPE == vattn::attn::kRopeQ ? 1 : 0);
-  auto kern = vattn::attn::attn_pair_kernel<D, ROPE>;
+  constexpr int slot = HYB ? 4 : (D == 64 ? 0 : 2) + (ROPE == vattn::attn::kRopeQ ? 1 : 0);
+  auto kern = vattn::attn::attn_pair_kernel<D, ROPE, HYB>;
   vattn_status st = ensure_smem(kern, Cfg::kSmemBytes, g_pair_smem_done[slot]);
   if (st) return st;
   const int segs = p.n_q_tiles / p.q_tiles_per_seg;
@@ -758,7 +758,11 @@ vattn_status vattn_hybrid_chunk(const void* q, const void* k, const void* v, voi
   p.n_q_tiles = C * p.q_tiles_per_seg;
   p.hyb_S = wsS;
   p.hyb_z = wsz;
+#if VATTN_PAIR_TILES
+  return launch_pair<128, vattn::attn::kRopeNone, true>(mq, mk, mv, mk, mv, p, stream);
+#else
   return launch_attention<128, vattn::attn::kRopeNone, true>(mq, mk, mv, mk, mv, p, stream);
+#endif
 }
 
 // ------------------------------------------------- hybrid without workspace
