@@ -114,7 +114,7 @@ vattn_status get_encode(PFN_cuTensorMapEncodeTiled_v12000* fn) {
 // bf16 tensor [n3][n2][n1][d] (d innermost) as a 4-D TMA map whose box is
 // 64 channels x 1 x `rows` x 1, 128-byte swizzle, zero fill out of range.
 vattn_status make_map(CUtensorMap* m, const void* base, int d, int n1, int n2, int n3, int rows) {
-  PFN_cuTensorMapEncodeTiled_v12000 enc;
+  PFN_cuTensorMapEncodeTiled_v12000 enc = nullptr;
   vattn_status st = get_encode(&enc);
   if (st) return st;
   const cuuint64_t dims[4] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(n1),
@@ -165,6 +165,7 @@ vattn_status launch_attention(const CUtensorMap& q, const CUtensorMap& k, const 
   return VATTN_OK;
 }
 
+#if VATTN_PAIR_TILES
 uint64_t g_pair_smem_done[5][1];
 
 // Two query tiles per CTA (attention_pair.cuh): grid = tile pairs x heads x
@@ -185,6 +186,8 @@ vattn_status launch_pair(const CUtensorMap& q, const CUtensorMap& k, const CUten
   VATTN_CUDA(cudaGetLastError());
   return VATTN_OK;
 }
+
+#endif
 
 vattn_status dispatch_attention(int d, int rope_mode, const CUtensorMap& q, const CUtensorMap& k,
                                 const CUtensorMap& v, const CUtensorMap& k2, const CUtensorMap& v2,
