@@ -289,12 +289,7 @@ def run_ours(args, rank, world, device):
         metric=METRIC, value=value, unit="TFLOP/s", n_gpus=world, steps=args.steps,
         warmup=args.warmup, ms_per_step=ms_per_step, higher_is_better=True, scaling="weak",
         vs_baseline=None, dtype="bf16", data="synthetic",
-        config={"workload": "wan13b full bidirectional attention + fused 3D-RoPE "
-                            "(B=1, H=12, d=128, grid 21x30x52 = 32760 tokens, pairs t22/h21/w21, "
-                            "theta 1e4)",
-                "mask_adjusted_flops_per_step": w["flops"],
-                "l2": "flushed before every timed step (256 MiB write); inputs 300 MB > L2",
-                "parallelism": "replicas x%d" % world},
+        config=workload_config(w["flops"], world),
         roofline={"bound": "tensor", "achieved": achieved, "peak": pk["bf16_tflops"],
                   "unit": "TFLOP/s", "frac": achieved / pk["bf16_tflops"],
                   "frac_of_sustained": achieved / pk.get("bf16_tflops_sustained", pk["bf16_tflops"]),
@@ -448,6 +443,15 @@ def cpu_baseline(w, rows=2048):
                       "fp64 with 3D-RoPE; TFLOP/s of mask-adjusted work" % len(rows_arr)}
 
 
+def workload_config(flops, world):
+    """The benchmarked workload, named the same way by both arms."""
+    return {"workload": "wan13b full bidirectional attention + fused 3D-RoPE "
+                        "(B=1, H=12, d=128, grid 21x30x52 = 32760 tokens, pairs t22/h21/w21, theta 1e4)",
+            "mask_adjusted_flops_per_step": flops,
+            "l2": "flushed before every timed step (256 MiB write); inputs 300 MB > L2",
+            "parallelism": "replicas x%d" % world}
+
+
 def run_reference(args, rank, world):
     """The oracle timed on the host as the reference arm (rank 0 only)."""
     if rank != 0:
@@ -477,8 +481,7 @@ def run_reference(args, rank, world):
     return dict(metric=METRIC, value=val, unit="TFLOP/s", n_gpus=world, steps=args.steps,
                 warmup=args.warmup, ms_per_step=dt / args.steps * 1e3, higher_is_better=True,
                 scaling="weak", vs_baseline=None, dtype="f64", data="synthetic", impl="reference",
-                config={"workload": "wan13b full bidirectional attention + 3D-RoPE (B=1, H=12, d=128, "
-                                    "32760 tokens); bounded row sample per step"},
+                config=workload_config(4.0 * d * L * L * c["H"], world),
                 cpu_baseline={"value": val, "unit": "TFLOP/s", "cores": oracle.num_threads(),
                               "kind": "oracle", "sample": sample},
                 e2e={"value": val, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0})
