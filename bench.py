@@ -428,7 +428,7 @@ def secondary_measurements(va, torch, device, flush):
     return out
 
 
-def cpu_baseline(w, rows=2048):
+def cpu_baseline(w, rows=20480):
     """The fp64 oracle, as it stands, on a bounded sample of the workload."""
     import oracle
     rows_arr = si.sample_rows(0xBA5E, rows, w["B"], 2, w["L"])
@@ -495,7 +495,7 @@ def main():
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--no-secondary", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--cpu-rows", type=int, default=2048)
+    ap.add_argument("--cpu-rows", type=int, default=20480)
     ap.add_argument("--ref-rows", type=int, default=512)
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3) if args.impl == "ours" else args.warmup
