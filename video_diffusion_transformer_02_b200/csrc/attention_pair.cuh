@@ -6,10 +6,16 @@
 //     of a score tile (no row-max exchange between warpgroups);
 //   * scores are computed in 64-key sub-tiles, double-buffered in TMEM per
 //     query tile, so S_X(j+1) = Q_X K_{j+1}^T runs on the tensor core while
-//     the softmax of S_X(j) runs, and the MMA thread interleaves both tiles
-//     (FlashAttention-4-style ping-pong on Blackwell);
+//     the softmax of S_X(j) runs; each tile has its own MMA-issuing thread
+//     and tile B starts half a period after tile A (a ping-pong of the two
+//     softmax warpgroups, as in FlashAttention-4 on Blackwell);
 //   * every K and V stage (128 keys, two sub-tiles) is loaded into shared
 //     memory once for both query tiles.
+//
+// The HYB instantiation adds MobileWan's linear read-out after the chunk's
+// softmax part: phi(Q) replaces Q in shared memory, S_c (bf16 hi + lo) fills
+// the freed K stages, phi(Q) S_c runs into the freed S buffers, and the
+// epilogue joins both parts in one normalisation.
 //
 // Warp roles: warp 0 TMA Q_A, Q_B, then K stages; warp 1 TMEM allocation and
 // tcgen05.mma issue for tile A; warp 2 TMA V stages; warp 3 tcgen05.mma issue
@@ -19,7 +25,7 @@
 // TMEM columns (512): S_X buffer b at [128 x + 64 b, +64) fp32 for tiles
 // x = A, B and b = 0, 1; O_A [256, 256+D), O_B [384, 384+D) fp32.  P (bf16
 // pairs, 32 columns) overwrites the first half of its S buffer once the
-// softmax holds the scores in registers; the MMA thread reuses a buffer for
+// softmax holds the scores in registers; an issuer reuses a buffer for
 // sub-tile j+2 only after the P V of sub-tile j has completed.
 #pragma once
 #include "attention.cuh"
