@@ -41,7 +41,7 @@ typedef struct CUstream_st* vattn_stream;
 typedef enum {
   VATTN_OK = 0,
   VATTN_ERR_INVALID_ARG = 1, /* a pointer, size or option is invalid          */
-  VATTN_ERR_UNSUPPORTED = 2, /* valid, but not a shape this build supports    */
+  VATTN_ERR_UNSUPPORTED = 2, /* valid, but not a shape the library supports   */
   VATTN_ERR_CUDA = 3,        /* a CUDA runtime/driver call failed             */
   VATTN_ERR_TIMEOUT = 4      /* a kernel gave up on a bounded internal wait   */
 } vattn_status;
