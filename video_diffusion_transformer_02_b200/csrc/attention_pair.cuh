@@ -7,8 +7,8 @@
 //   * scores are computed in 64-key sub-tiles, double-buffered in TMEM per
 //     query tile, so S_X(j+1) = Q_X K_{j+1}^T runs on the tensor core while
 //     the softmax of S_X(j) runs; each tile has its own MMA-issuing thread
-//     and tile B starts half a period after tile A (a ping-pong of the two
-//     softmax warpgroups, as in FlashAttention-4 on Blackwell);
+//     and tile B starts after tile A's first P (two softmax warpgroups
+//     sharing the tensor core, as in FlashAttention-4 on Blackwell);
 //   * every K and V stage (128 keys, two sub-tiles) is loaded into shared
 //     memory once for both query tiles.
 //
@@ -282,9 +282,8 @@ __global__ void __launch_bounds__(kPairThreads, 1)
       };
       bool ok = mbar_wait(ROPE == kRopeQ ? bQReady(x) : bQFull(x), 0, ab, kStatusTimeoutMma);
       // tile B starts once tile A has published its first P, so the two
-      // softmax warpgroups work half a period apart (measured faster than
-      // starting both together: their exponentials and TMEM traffic then
-      // overlap the other tile's MMAs instead of each other)
+      // softmax warpgroups do not start in lockstep (measured 2-3 % faster
+      // than starting both together)
       if (x == 1 && ok && nk > 0) ok = mbar_wait(bPFull(0, 0), 0, ab, kStatusTimeoutMma);
       if (ok && nk > 0) {
         ok = mbar_wait(bKFull(0), 0, ab, kStatusTimeoutMma);
