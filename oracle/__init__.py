@@ -1,3 +1,3 @@
 """fp64 CPU oracle (test infrastructure only; see oracle.py)."""
-from .oracle import (attention, build, hybrid_parallel, hybrid_recurrent, num_threads,  # noqa: F401
-                     ring_model, rope, stream)
+from .oracle import (attention, build, hybrid2_parallel, hybrid2_recurrent, hybrid_parallel,  # noqa: F401
+                     hybrid_recurrent, merge, num_threads, ring_model, rope, stream)

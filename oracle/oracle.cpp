@@ -268,18 +268,33 @@ int oracle_attention(const uint16_t* q, const uint16_t* k, const uint16_t* v,
 
 // Streaming decode (FlashDecoder Sec. 3.3): frame f's F query tokens attend
 // to all tokens of frames max(0, f - wb) .. f, taken from the full key and
-// value sequences of n_frames frames, keys rotated at their own absolute
-// frame index.  Keys are gathered per frame (the frame-by-frame processing
-// order), not masked.  rows: (b, h, i) triples over the whole sequence
-// (i = f * F + token); o [n_rows][d], lse [n_rows].
+// value sequences of n_frames frames.  Keys are gathered per frame (the
+// frame-by-frame processing order), not masked.  rows: (b, h, i) triples
+// over the whole sequence (i = f * F + token); o [n_rows][d], lse [n_rows].
+//
+// RoPE positions (rope_cfg given): a stream frame holds r = F / (Hg*Wg)
+// latent frames of Hg x Wg tokens (r = 1 for the backbone; r = r_t for the
+// temporal-refinement layers, which see r_t * L_frm tokens per step,
+// FlashDecoder "Complexity Analysis", Sec. 3.3).  Token n of stream frame
+// fr sits at t = r * (fr - base) + n / (Hg*Wg), h = (n / Wg) % Hg,
+// w = n % Wg, where base = 0 (absolute frame index) or, with
+// window_relative, base = max(0, f - wb), the first frame of the query's
+// window (positions relative to the current window, "Long Video Decoding",
+// Sec. 4.3).
 int oracle_stream(const uint16_t* q, const uint16_t* k, const uint16_t* v,
                   int B, int n_frames, int F, int H, int Hkv, int d, double scale, int wb,
                   const int* rope_cfg, double theta,
-                  const int32_t* rows, long n_rows, double* o, double* lse) {
+                  const int32_t* rows, long n_rows, double* o, double* lse, int window_relative) {
   if (H % Hkv) return 1;
   const bool use_rope = rope_cfg != nullptr;
   Rope r{};
-  if (use_rope) r = Rope{rope_cfg[0], rope_cfg[1], rope_cfg[2], rope_cfg[3], rope_cfg[4], theta};
+  long sub = 1;   // latent frames per stream frame
+  if (use_rope) {
+    r = Rope{rope_cfg[0], rope_cfg[1], rope_cfg[2], rope_cfg[3], rope_cfg[4], theta};
+    const long fr_tokens = static_cast<long>(r.Hg) * r.Wg;
+    if (F % fr_tokens) return 1;
+    sub = F / fr_tokens;
+  }
   const long L = static_cast<long>(n_frames) * F;
   const int group = H / Hkv;
 #pragma omp parallel
@@ -292,6 +307,7 @@ int oracle_stream(const uint16_t* q, const uint16_t* k, const uint16_t* v,
       const long i = rows[3 * s + 2];
       const long f = i / F;
       const long f0 = std::max(0L, f - wb);
+      const long base = window_relative ? f0 : 0;
       const long nk = (f - f0 + 1) * F;
       K.assign(nk * d, 0.0);
       V.assign(nk * d, 0.0);
@@ -303,7 +319,7 @@ int oracle_stream(const uint16_t* q, const uint16_t* k, const uint16_t* v,
           load_vec(v, L, Hkv, d, b, fr * F + tkn, h / group, &V[j * d]);
           if (use_rope) {
             long t, hh, w;
-            token_position(tkn, fr, r, &t, &hh, &w);
+            token_position(tkn, sub * (fr - base), r, &t, &hh, &w);
             rope_rotate(&K[j * d], d, r, t, hh, w);
           }
         }
@@ -311,7 +327,7 @@ int oracle_stream(const uint16_t* q, const uint16_t* k, const uint16_t* v,
       load_vec(q, L, H, d, b, i, h, qv.data());
       if (use_rope) {
         long t, hh, w;
-        token_position(i % F, f, r, &t, &hh, &w);
+        token_position(i % F, sub * (f - base), r, &t, &hh, &w);
         rope_rotate(qv.data(), d, r, t, hh, w);
       }
       attend_row(qv.data(), K.data(), V.data(), nk, d, scale, mask, o + s * d, lse + s);
@@ -454,6 +470,183 @@ int oracle_hybrid_recurrent(const uint16_t* q, const uint16_t* k, const uint16_t
         std::copy(z.begin(), z.end(), z_io + bh * d);
       }
     }
+  }
+  return 0;
+}
+
+// ---------------------------------------------------------------------------
+// Hybrid chunk attention, general form: the feature map of the MobileWan page
+// variant and softmax chunks that overlap the previous chunk (MobileWan
+// review, axiom ledger / App. A.3.1: learnable polynomial feature maps of
+// degree 3 for phi_q and phi_k; chunk overlap T_o).
+//   fmap 0: phi(x) = elu(x) + 1 (coef unused);
+//   fmap 1: phi_q(x) = a0 + a1 x + a2 x^2 + a3 x^3 with (a0..a3) =
+//           coef[(0 * H + h) * 4 ..], phi_k likewise with coef[(1 * H + h) * 4 ..]
+//           (one polynomial per head and map; coefficients are caller data).
+// With overlap ov >= 0 tokens, the softmax part of chunk c covers keys
+// [max(0, c * ct - ov), min(L, (c + 1) * ct)) -- the chunk plus the last ov
+// tokens before it -- and the linear part the keys j < c * ct - ov (plus the
+// incoming state); every key before the end of the query's chunk is counted
+// once.  The overlap reaches back inside this call only (chunk 0 has none);
+// the outgoing state covers all L tokens.  ov = 0 is the form above.
+// ---------------------------------------------------------------------------
+static inline double feature(int fmap, const double* a, double x) {
+  if (fmap == 0) return x > 0.0 ? x + 1.0 : std::exp(x);
+  return a[0] + x * (a[1] + x * (a[2] + x * a[3]));
+}
+
+// Parallel form: rows (b, h, i); o [n_rows][d]; S0/z0 nullable as above.
+int oracle_hybrid2_parallel(const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                            int B, int L, int H, int d, int chunk_tokens, int overlap, double scale,
+                            int fmap, const double* coef, const double* S0, const double* z0,
+                            const int32_t* rows, long n_rows, double* o) {
+  if (chunk_tokens <= 0 || overlap < 0 || (fmap == 1 && !coef) || fmap < 0 || fmap > 1) return 1;
+#pragma omp parallel
+  {
+    std::vector<double> qv(d), pq(d), kv(d), vv(d), num(d);
+#pragma omp for schedule(dynamic, 1)
+    for (long s = 0; s < n_rows; ++s) {
+      const int b = rows[3 * s], h = rows[3 * s + 1];
+      const long i = rows[3 * s + 2];
+      const double* aq = fmap == 1 ? coef + (0L * H + h) * 4 : nullptr;
+      const double* ak = fmap == 1 ? coef + (1L * H + h) * 4 : nullptr;
+      const long c = i / chunk_tokens;
+      const long w0 = std::max(0L, c * chunk_tokens - overlap);      // softmax window start
+      const long w1 = std::min<long>(L, (c + 1) * chunk_tokens);     // and end
+      load_vec(q, L, H, d, b, i, h, qv.data());
+      for (int x = 0; x < d; ++x) pq[x] = feature(fmap, aq, qv[x]);
+      std::fill(num.begin(), num.end(), 0.0);
+      double den = 0.0;
+      if (S0) {
+        const double* Sb = S0 + (static_cast<long>(b) * H + h) * d * d;
+        const double* zb = z0 + (static_cast<long>(b) * H + h) * d;
+        for (int a = 0; a < d; ++a) {
+          den += pq[a] * zb[a];
+          for (int e = 0; e < d; ++e) num[e] += pq[a] * Sb[a * d + e];
+        }
+      }
+      for (long j = 0; j < w0; ++j) {           // before the window: linear
+        load_vec(k, L, H, d, b, j, h, kv.data());
+        load_vec(v, L, H, d, b, j, h, vv.data());
+        double w = 0.0;
+        for (int x = 0; x < d; ++x) w += pq[x] * feature(fmap, ak, kv[x]);
+        den += w;
+        for (int x = 0; x < d; ++x) num[x] += w * vv[x];
+      }
+      for (long j = w0; j < w1; ++j) {          // the window: softmax weights
+        load_vec(k, L, H, d, b, j, h, kv.data());
+        load_vec(v, L, H, d, b, j, h, vv.data());
+        double acc = 0.0;
+        for (int x = 0; x < d; ++x) acc += qv[x] * kv[x];
+        const double w = std::exp(scale * acc);
+        den += w;
+        for (int x = 0; x < d; ++x) num[x] += w * vv[x];
+      }
+      for (int x = 0; x < d; ++x) o[s * d + x] = num[x] / den;
+    }
+  }
+  return 0;
+}
+
+// Recurrent form: per (b, h) the state (S, z) is advanced in chunk order;
+// chunk c's queries read the state of keys j < c * ct - ov, then the keys
+// [c * ct - ov, (c + 1) * ct - ov) are folded in; after the last chunk the
+// remaining keys are folded so that the outgoing state covers all L tokens.
+int oracle_hybrid2_recurrent(const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                             int B, int L, int H, int d, int chunk_tokens, int overlap, double scale,
+                             int fmap, const double* coef, double* S_io, double* z_io,
+                             const char* row_mask, double* o) {
+  if (chunk_tokens <= 0 || overlap < 0 || (fmap == 1 && !coef) || fmap < 0 || fmap > 1) return 1;
+  const long n_chunks = (L + chunk_tokens - 1) / chunk_tokens;
+  const long BH = static_cast<long>(B) * H;
+#pragma omp parallel
+  {
+    std::vector<double> S(static_cast<size_t>(d) * d), z(d), qv(d), pq(d), kv(d), vv(d), num(d);
+#pragma omp for schedule(dynamic, 1)
+    for (long bh = 0; bh < BH; ++bh) {
+      const int b = static_cast<int>(bh / H), h = static_cast<int>(bh % H);
+      const double* aq = fmap == 1 ? coef + (0L * H + h) * 4 : nullptr;
+      const double* ak = fmap == 1 ? coef + (1L * H + h) * 4 : nullptr;
+      if (S_io) {
+        std::copy(S_io + bh * d * d, S_io + (bh + 1) * d * d, S.begin());
+        std::copy(z_io + bh * d, z_io + (bh + 1) * d, z.begin());
+      } else {
+        std::fill(S.begin(), S.end(), 0.0);
+        std::fill(z.begin(), z.end(), 0.0);
+      }
+      long folded = 0;   // keys [0, folded) are in the state
+      auto fold_to = [&](long end) {
+        for (; folded < end; ++folded) {
+          load_vec(k, L, H, d, b, folded, h, kv.data());
+          load_vec(v, L, H, d, b, folded, h, vv.data());
+          for (int a = 0; a < d; ++a) {
+            const double pk = feature(fmap, ak, kv[a]);
+            z[a] += pk;
+            for (int e = 0; e < d; ++e) S[a * d + e] += pk * vv[e];
+          }
+        }
+      };
+      for (long c = 0; c < n_chunks; ++c) {
+        const long w0 = std::max(0L, c * chunk_tokens - overlap);
+        const long w1 = std::min<long>(L, (c + 1) * chunk_tokens);
+        fold_to(w0);
+        for (long i = c * chunk_tokens; i < w1; ++i) {
+          if (row_mask && !row_mask[bh * L + i]) continue;
+          load_vec(q, L, H, d, b, i, h, qv.data());
+          for (int x = 0; x < d; ++x) pq[x] = feature(fmap, aq, qv[x]);
+          double den = 0.0;
+          std::fill(num.begin(), num.end(), 0.0);
+          for (int a = 0; a < d; ++a) {
+            den += pq[a] * z[a];
+            for (int e = 0; e < d; ++e) num[e] += pq[a] * S[a * d + e];
+          }
+          for (long j = w0; j < w1; ++j) {
+            load_vec(k, L, H, d, b, j, h, kv.data());
+            load_vec(v, L, H, d, b, j, h, vv.data());
+            double acc = 0.0;
+            for (int x = 0; x < d; ++x) acc += qv[x] * kv[x];
+            const double w = std::exp(scale * acc);
+            den += w;
+            for (int x = 0; x < d; ++x) num[x] += w * vv[x];
+          }
+          double* orow = o + ((static_cast<long>(b) * L + i) * H + h) * d;
+          for (int x = 0; x < d; ++x) orow[x] = num[x] / den;
+        }
+      }
+      fold_to(L);
+      if (S_io) {
+        std::copy(S.begin(), S.end(), S_io + bh * d * d);
+        std::copy(z.begin(), z.end(), z_io + bh * d);
+      }
+    }
+  }
+  return 0;
+}
+
+// Exact combination of R partial attentions of the same rows over disjoint
+// key sets (the join of Ring attention's key shards, ReGenVC "Unified
+// sequence parallelism", Sec. 3.5): the softmax over the union of the key
+// sets, written through each part's log-sum-exp.
+//   o_parts [R][n][d], lse_parts [R][n] (natural log; -inf = no key) ->
+//   o [n][d], lse [n].
+int oracle_merge(const double* o_parts, const double* lse_parts, int R, long n, int d, double* o, double* lse) {
+  if (R < 1) return 1;
+  for (long i = 0; i < n; ++i) {
+    double m = -std::numeric_limits<double>::infinity();
+    for (int r = 0; r < R; ++r) m = std::max(m, lse_parts[r * n + i]);
+    for (int c = 0; c < d; ++c) o[i * d + c] = 0.0;
+    if (m == -std::numeric_limits<double>::infinity()) {
+      lse[i] = m;
+      continue;
+    }
+    double wsum = 0.0;
+    for (int r = 0; r < R; ++r) {
+      const double w = std::exp(lse_parts[r * n + i] - m);
+      wsum += w;
+      for (int c = 0; c < d; ++c) o[i * d + c] += w * o_parts[(r * n + i) * d + c];
+    }
+    for (int c = 0; c < d; ++c) o[i * d + c] /= wsum;
+    lse[i] = m + std::log(wsum);
   }
   return 0;
 }

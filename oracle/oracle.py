@@ -44,11 +44,15 @@ def lib():
         _lib.oracle_rope.argtypes = [P, P, i, i, i, i, i, i, i, i, i, d, i]
         _lib.oracle_attention.argtypes = [P, P, P, i, i, i, i, i, i, d, i, i, i, i, i, i, i,
                                           P, d, P, l, P, P]
-        _lib.oracle_stream.argtypes = [P, P, P, i, i, i, i, i, i, d, i, P, d, P, l, P, P]
+        _lib.oracle_stream.argtypes = [P, P, P, i, i, i, i, i, i, d, i, P, d, P, l, P, P, i]
         _lib.oracle_hybrid_parallel.argtypes = [P, P, P, i, i, i, i, i, d, P, P, P, l, P]
         _lib.oracle_hybrid_recurrent.argtypes = [P, P, P, i, i, i, i, i, d, P, P, P, P]
+        _lib.oracle_hybrid2_parallel.argtypes = [P, P, P, i, i, i, i, i, i, d, i, P, P, P, P, l, P]
+        _lib.oracle_hybrid2_recurrent.argtypes = [P, P, P, i, i, i, i, i, i, d, i, P, P, P, P, P]
+        _lib.oracle_merge.argtypes = [P, P, i, l, i, P, P]
         for f in ("oracle_rope", "oracle_attention", "oracle_stream",
-                  "oracle_hybrid_parallel", "oracle_hybrid_recurrent", "oracle_num_threads"):
+                  "oracle_hybrid_parallel", "oracle_hybrid_recurrent", "oracle_hybrid2_parallel",
+                  "oracle_hybrid2_recurrent", "oracle_merge", "oracle_num_threads"):
             getattr(_lib, f).restype = ctypes.c_int
     return _lib
 
@@ -113,11 +117,14 @@ def attention(q, k, v, scale, mode="full", F=0, chunk=1, wb=0, wf=0,
     return o, lse
 
 
-def stream(q, k, v, F, scale, wb, rope=None, rows=None):
+def stream(q, k, v, F, scale, wb, rope=None, rows=None, window_relative=False):
     """Frame-by-frame streaming attention over a whole sequence of frames.
 
     q/k/v: [B, n_frames * F, H, d].  Returns o [n, d], lse [n] for rows
-    (b, h, i); rows=None evaluates every row (o [B, L, H, d]).
+    (b, h, i); rows=None evaluates every row (o [B, L, H, d]).  With rope, a
+    stream frame of F tokens holds F / (Hg * Wg) latent frames; RoPE t counts
+    latent frames from 0 (absolute) or from the first frame of the query's
+    window (window_relative).
     """
     q, k, v = _bits(q), _bits(k), _bits(v)
     B, L, H, d = q.shape
@@ -132,7 +139,7 @@ def stream(q, k, v, F, scale, wb, rope=None, rows=None):
     lse = np.empty((n,))
     cfg, theta, _ = _rope_args(rope)
     rc = lib().oracle_stream(_ptr(q), _ptr(k), _ptr(v), B, L // F, F, H, Hkv, d, float(scale), wb,
-                             _ptr(cfg), theta, _ptr(rows), n, _ptr(o), _ptr(lse))
+                             _ptr(cfg), theta, _ptr(rows), n, _ptr(o), _ptr(lse), int(bool(window_relative)))
     assert rc == 0
     if full:
         return o.reshape(B, L, H, d), lse.reshape(B, L, H).transpose(0, 2, 1)
@@ -192,3 +199,59 @@ def hybrid_recurrent(q, k, v, chunk_tokens, scale, S=None, z=None, row_mask=None
                                        float(scale), _ptr(S_io), _ptr(z_io), _ptr(m), _ptr(o))
     assert rc == 0
     return o, S_io, z_io
+
+
+def _coef(fmap, coef, H):
+    if fmap == "elu":
+        return 0, None
+    c = np.ascontiguousarray(coef, dtype=np.float64)
+    assert c.shape == (2, H, 4), "coef: [2 (q, k), H, 4] polynomial coefficients a0..a3"
+    return 1, c
+
+
+def hybrid2_parallel(q, k, v, chunk_tokens, scale, rows, overlap=0, fmap="elu", coef=None, S0=None, z0=None):
+    """General hybrid chunk attention (polynomial feature map, chunk
+    overlap), parallel form, for rows (b, h, i) -> o [n, d]."""
+    q, k, v = _bits(q), _bits(k), _bits(v)
+    B, L, H, d = q.shape
+    fm, c = _coef(fmap, coef, H)
+    rows = np.ascontiguousarray(rows, dtype=np.int32)
+    o = np.empty((rows.shape[0], d))
+    S0 = None if S0 is None else np.ascontiguousarray(S0, dtype=np.float64)
+    z0 = None if z0 is None else np.ascontiguousarray(z0, dtype=np.float64)
+    rc = lib().oracle_hybrid2_parallel(_ptr(q), _ptr(k), _ptr(v), B, L, H, d, chunk_tokens, overlap,
+                                       float(scale), fm, _ptr(c), _ptr(S0), _ptr(z0), _ptr(rows),
+                                       rows.shape[0], _ptr(o))
+    assert rc == 0
+    return o
+
+
+def hybrid2_recurrent(q, k, v, chunk_tokens, scale, overlap=0, fmap="elu", coef=None, S=None, z=None,
+                      row_mask=None):
+    """General hybrid chunk attention, recurrent form.  Returns
+    (o [B, L, H, d], S_out [B, H, d, d], z_out [B, H, d])."""
+    q, k, v = _bits(q), _bits(k), _bits(v)
+    B, L, H, d = q.shape
+    fm, c = _coef(fmap, coef, H)
+    S_io = np.zeros((B, H, d, d)) if S is None else np.array(S, dtype=np.float64, copy=True)
+    z_io = np.zeros((B, H, d)) if z is None else np.array(z, dtype=np.float64, copy=True)
+    o = np.full((B, L, H, d), np.nan)
+    m = None if row_mask is None else np.ascontiguousarray(row_mask, dtype=np.int8)
+    rc = lib().oracle_hybrid2_recurrent(_ptr(q), _ptr(k), _ptr(v), B, L, H, d, chunk_tokens, overlap,
+                                        float(scale), fm, _ptr(c), _ptr(S_io), _ptr(z_io), _ptr(m), _ptr(o))
+    assert rc == 0
+    return o, S_io, z_io
+
+
+def merge(o_parts, lse_parts):
+    """Combination of R partial attentions over disjoint key sets:
+    o_parts [R, n, d], lse_parts [R, n] (float64) -> (o [n, d], lse [n])."""
+    o_parts = np.ascontiguousarray(o_parts, dtype=np.float64)
+    lse_parts = np.ascontiguousarray(lse_parts, dtype=np.float64)
+    R, n, d = o_parts.shape
+    assert lse_parts.shape == (R, n)
+    o = np.empty((n, d))
+    lse = np.empty((n,))
+    rc = lib().oracle_merge(_ptr(o_parts), _ptr(lse_parts), R, n, d, _ptr(o), _ptr(lse))
+    assert rc == 0
+    return o, lse

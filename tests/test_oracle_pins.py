@@ -355,3 +355,150 @@ def test_hybrid_state_resume():
     op = oracle.hybrid_parallel(q[:, 24:], k[:, 24:], v[:, 24:], ct, 0.25, rows, S0=S1, z0=z1)
     ref = np.stack([o2[0, i, h] for _, h, i in rows])
     assert np.max(np.abs(op - ref) / (np.abs(ref) + 1e-30)) < 1e-10
+
+
+# ------------------------------------------- window-relative RoPE positions
+@pytest.mark.parametrize("sub", [1, 2])
+def test_stream_window_relative_positions(sub):
+    # FlashDecoder "Long Video Decoding" (Sec. 4.3): positions relative to the
+    # current window.  (a) By RoPE's relative property the attention equals
+    # the absolute-position one (to rounding); (b) a query frame's rows equal
+    # plain attention over its window's tokens with the query at latent frame
+    # sub * (f - f0) and the keys from latent frame 0, evaluated by
+    # oracle_attention (a separate code path); (c) frames before the window
+    # fills (f < wb) are unchanged bit for bit.  sub = latent frames per
+    # stream frame (2: a temporal-refinement step of r_t = 2 frames).
+    T, Hg, Wg, H, d, wb = 7, 3, 4, 2, 64, 2
+    F = sub * Hg * Wg
+    L = T * F
+    q = si.normal_bf16(111, (1, L, H, d))
+    k = si.normal_bf16(112, (1, L, H, d))
+    v = si.normal_bf16(113, (1, L, H, d))
+    rope = dict(Hg=Hg, Wg=Wg, pairs=(12, 10, 10), theta=1e4)
+    o_abs, l_abs = oracle.stream(q, k, v, F, 1 / 8, wb, rope=rope)
+    o_rel, l_rel = oracle.stream(q, k, v, F, 1 / 8, wb, rope=rope, window_relative=True)
+    assert np.max(np.abs(o_rel - o_abs)) < 1e-12 and np.max(np.abs(l_rel - l_abs)) < 1e-12
+    assert np.array_equal(o_rel[:, :wb * F], o_abs[:, :wb * F])
+    for f in range(T):
+        f0 = max(0, f - wb)
+        qf = q[:, f * F:(f + 1) * F]
+        kw, vw = k[:, f0 * F:(f + 1) * F], v[:, f0 * F:(f + 1) * F]
+        ow, lw = oracle.attention(qf, kw, vw, 1 / 8, rope=rope, q_frame_offset=sub * (f - f0), k_frame_offset=0)
+        assert np.array_equal(ow, o_rel[:, f * F:(f + 1) * F]), "frame %d" % f
+
+
+# ------------------------------------------------ hybrid, general form
+POLY = np.array([[[0.7, 0.3, 0.2, 0.05]], [[1.0, 0.5, 0.25, 1.0 / 24.0]]])   # [q/k][H=1][a0..a3]
+
+
+def test_hybrid2_elu_no_overlap_reproduces_the_hybrid():
+    q, k, v = _hyb_inputs()
+    S0 = si.normal_f64(31, 2 * 16 * 16).reshape(1, 2, 16, 16)
+    z0 = np.abs(si.normal_f64(32, 2 * 16)).reshape(1, 2, 16) + 1.0
+    o1, S1, z1 = oracle.hybrid_recurrent(q, k, v, 12, 0.25, S=S0, z=z0)
+    o2, S2, z2 = oracle.hybrid2_recurrent(q, k, v, 12, 0.25, S=S0, z=z0)
+    assert np.max(np.abs(o1 - o2)) < 1e-12
+    assert np.max(np.abs(S1 - S2)) < 1e-10 and np.max(np.abs(z1 - z2)) < 1e-10
+    rows = _all_rows(1, 2, 40)
+    p1 = oracle.hybrid_parallel(q, k, v, 12, 0.25, rows, S0=S0, z0=z0)
+    p2 = oracle.hybrid2_parallel(q, k, v, 12, 0.25, rows, S0=S0, z0=z0)
+    assert np.max(np.abs(p1 - p2)) < 1e-12
+
+
+@pytest.mark.parametrize("fmap,overlap", [("elu", 5), ("poly", 0), ("poly", 7), ("poly", 30)])
+def test_hybrid2_recurrent_equals_parallel(fmap, overlap):
+    q, k, v = _hyb_inputs()
+    coef = np.concatenate([POLY, POLY * 0.9], axis=1)        # H = 2
+    S0 = np.abs(si.normal_f64(33, 2 * 16 * 16)).reshape(1, 2, 16, 16)
+    z0 = np.abs(si.normal_f64(34, 2 * 16)).reshape(1, 2, 16) + 1.0
+    o_rec, _, _ = oracle.hybrid2_recurrent(q, k, v, 12, 0.25, overlap=overlap, fmap=fmap, coef=coef, S=S0, z=z0)
+    rows = _all_rows(1, 2, 40)
+    o_par = oracle.hybrid2_parallel(q, k, v, 12, 0.25, rows, overlap=overlap, fmap=fmap, coef=coef, S0=S0, z0=z0)
+    ref = np.stack([o_rec[0, i, h] for _, h, i in rows])
+    assert np.max(np.abs(o_par - ref) / (np.abs(ref) + 1e-30)) < 1e-10
+
+
+# phi_k(x) = 1 + x/2 + x^2/4 + x^3/24, by hand: phi_k(2) = 1 + 1 + 1 + 1/3,
+# phi_k(-1) = 1 - 1/2 + 1/4 - 1/24, phi_k(0) = 1; phi_q(0) = a0 = 0.7.
+@pytest.mark.parametrize("x,phix", [(2.0, 10.0 / 3.0), (-1.0, 17.0 / 24.0), (0.0, 1.0)])
+@pytest.mark.parametrize("overlap", [0, 3, 7, 9])
+def test_hybrid2_closed_form_polynomial_and_overlap(x, phix, overlap):
+    # q = 0: softmax weights are exp(0) = 1; phi_q(0) = 0.7 on every channel,
+    # so a key with every entry x weighs 0.7 * d * phi_k(x) in the linear
+    # part.  With the softmax window [w0, w1) = [max(0, c ct - ov), end of
+    # chunk c):  o_i = (sum_{window} v + lam sum_{j < w0} v) / (|window| + lam w0).
+    L, H, d, ct = 30, 1, 8, 7
+    q = bf16(np.zeros((1, L, H, d)))
+    k = bf16(np.full((1, L, H, d), x))
+    v = si.normal_bf16(6, (1, L, H, d))
+    V = si.bf16_bits_to_f64(v)[0, :, 0]
+    o, S, z = oracle.hybrid2_recurrent(q, k, v, ct, 0.5, overlap=overlap, fmap="poly", coef=POLY)
+    lam = 0.7 * d * phix
+    for i in range(L):
+        c = i // ct
+        w0, w1 = max(0, c * ct - overlap), min(L, (c + 1) * ct)
+        num = V[w0:w1].sum(0) + lam * V[:w0].sum(0)
+        den = (w1 - w0) + lam * w0
+        assert np.max(np.abs(o[0, i, 0] - num / den)) < 1e-13, (i, w0, w1)
+    assert np.allclose(z[0, 0], np.full(d, L * phix), rtol=1e-13)
+    assert np.allclose(S[0, 0], phix * np.tile(V.sum(0), (d, 1)), rtol=1e-12, atol=1e-12)
+
+
+def test_hybrid2_limits():
+    q, k, v = _hyb_inputs()
+    coef = np.concatenate([POLY, POLY], axis=1)
+    # one chunk covering everything: pure softmax whatever the feature map
+    o, _, _ = oracle.hybrid2_recurrent(q, k, v, 40, 0.25, overlap=3, fmap="poly", coef=coef)
+    ref, _ = oracle.attention(q, k, v, 0.25)
+    assert np.max(np.abs(o - ref)) < 1e-12
+    # an overlap reaching back to token 0 leaves no linear part: every query
+    # sees all keys up to the end of its chunk (chunk-causal softmax)
+    o, _, _ = oracle.hybrid2_recurrent(q, k, v, 12, 0.25, overlap=40, fmap="poly", coef=coef)
+    ref, _ = oracle.attention(q, k, v, 0.25, mode="chunk_causal", F=12, chunk=1)
+    assert np.max(np.abs(o - ref)) < 1e-12
+    # chunk-0 rows are the local softmax of chunk 0 for any overlap
+    o, _, _ = oracle.hybrid2_recurrent(q, k, v, 12, 0.25, overlap=5, fmap="poly", coef=coef)
+    ref, _ = oracle.attention(q, k, v, 0.25, mode="sliding", F=12, wb=0, wf=0)
+    assert np.max(np.abs(o[:, :12] - ref[:, :12])) < 1e-12
+
+
+def test_hybrid2_state_resume_polynomial():
+    # Without overlap, two calls carrying (S, z) equal one call (RNN view).
+    q, k, v = _hyb_inputs()
+    coef = np.concatenate([POLY, POLY], axis=1)
+    o, S, z = oracle.hybrid2_recurrent(q, k, v, 8, 0.25, fmap="poly", coef=coef)
+    o1, S1, z1 = oracle.hybrid2_recurrent(q[:, :16], k[:, :16], v[:, :16], 8, 0.25, fmap="poly", coef=coef)
+    o2, S2, z2 = oracle.hybrid2_recurrent(q[:, 16:], k[:, 16:], v[:, 16:], 8, 0.25, fmap="poly", coef=coef,
+                                          S=S1, z=z1)
+    assert np.max(np.abs(np.concatenate([o1, o2], axis=1) - o)) < 1e-12
+    assert np.max(np.abs(S2 - S)) < 1e-10 and np.max(np.abs(z2 - z)) < 1e-10
+
+
+# --------------------------------------------------------------------- merge
+def test_merge_of_key_shards_is_attention_over_all_keys():
+    # Ring attention's join (ReGenVC Sec. 3.5): partial attentions over
+    # disjoint key shards, combined through their log-sum-exp, equal one
+    # attention over all keys.
+    L, H, d, R = 48, 2, 16, 3
+    q = si.normal_bf16(121, (1, L, H, d))
+    k = si.normal_bf16(122, (1, L, H, d))
+    v = si.normal_bf16(123, (1, L, H, d))
+    ref, lref = oracle.attention(q, k, v, 0.25)
+    cuts = [0, 10, 31, 48]
+    parts = [oracle.attention(q, k[:, a:b], v[:, a:b], 0.25) for a, b in zip(cuts, cuts[1:])]
+    o_p = np.stack([p[0].transpose(0, 2, 1, 3).reshape(-1, d) for p in parts])   # [R, (b h i), d]
+    l_p = np.stack([p[1].reshape(-1) for p in parts])                              # [R, (b h i)]
+    o, lse = oracle.merge(o_p, l_p)
+    assert np.max(np.abs(o - ref.transpose(0, 2, 1, 3).reshape(-1, d))) < 1e-12
+    assert np.max(np.abs(lse - lref.reshape(-1))) < 1e-12
+
+
+def test_merge_closed_form_and_empty_part():
+    # weights e^0 : e^{ln 3} = 1 : 3; a part with lse = -inf has weight 0.
+    o_p = np.array([[[1.0, 0.0]], [[0.0, 1.0]], [[5.0, 5.0]]])
+    l_p = np.array([[0.0], [math.log(3.0)], [-np.inf]])
+    o, lse = oracle.merge(o_p, l_p)
+    assert np.allclose(o, [[0.25, 0.75]], rtol=0, atol=1e-15)
+    assert abs(lse[0] - math.log(4.0)) < 1e-15
+    o, lse = oracle.merge(o_p[2:], l_p[2:])
+    assert np.array_equal(o, [[0.0, 0.0]]) and lse[0] == -np.inf
