@@ -304,8 +304,14 @@ def run_ours(args, rank, world, device):
 
 
 def _time_events(torch, fn, n, flush=None):
+    """Mean ms of n runs of fn, each bracketed by CUDA events on the current
+    stream (L2 flushed before each run, outside the events, when given)."""
+    return statistics.mean(_event_list(torch, fn, n, flush))
+
+
+def _event_list(torch, fn, n, flush=None):
     s = torch.cuda.current_stream()
-    tot = 0.0
+    out = []
     for _ in range(n):
         if flush is not None:
             flush.zero_()
@@ -314,13 +320,54 @@ def _time_events(torch, fn, n, flush=None):
         fn()
         b.record(s)
         torch.cuda.synchronize()
-        tot += a.elapsed_time(b)
-    return tot / n
+        out.append(a.elapsed_time(b))
+    return out
+
+
+REPS = 20   # timed repetitions of every secondary figure (median reported)
+
+
+def _measure(torch, fn, reps=REPS, flush=None, per_call=1):
+    """Median of `reps` event-timed runs of fn (after one untimed run), with
+    the nvidia-smi clock record of the timed runs.  per_call: calls of the
+    measured operation inside one run of fn (the figure is per call)."""
+    fn()
+    torch.cuda.synchronize()
+    sampler = ClockSampler(torch.cuda.current_device())
+    sampler.start()
+    ms = _event_list(torch, fn, reps, flush)
+    clocks = sampler.stop()
+    ms = [m / per_call for m in ms]
+    return {"median_ms": statistics.median(ms), "min_ms": min(ms), "max_ms": max(ms), "reps": reps,
+            "clocks": clocks}
+
+
+def _graph(torch, calls):
+    """A CUDA graph replaying `calls` (a list of callables) back to back."""
+    g = torch.cuda.CUDAGraph()
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        calls[0]()
+        with torch.cuda.graph(g, stream=side):
+            for c in calls:
+                c()
+    torch.cuda.current_stream().wait_stream(side)
+    torch.cuda.synchronize()
+    return g
+
+
+def _hbm(pk, nbytes, m):
+    gbs = nbytes / (m["median_ms"] / 1e3) / 1e9
+    return {"bytes": nbytes, "us": m["median_ms"] * 1e3, "gbs": gbs, "frac_of_hbm": gbs / pk["hbm_gbs"]}
 
 
 def secondary_measurements(va, torch, device, flush):
-    """The other configurations, briefly: 14B full / chunk-causal TFLOPS,
-    streaming frames/s and append GB/s, hybrid time and scan bandwidth."""
+    """The other configurations: 14B full / chunk-causal TFLOPS, streaming
+    frames/s and its fraction of the tensor-peak ceiling, the KV append, the
+    hybrid call and its state delta and scan kernels (GB/s, fraction of HBM).
+    Every figure is the median of REPS event-timed runs with its own clock
+    record."""
     out = {}
     dev = lambda x: torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).to(device)
     pk, _ = peaks()
@@ -338,10 +385,10 @@ def secondary_measurements(va, torch, device, flush):
     for name, mode, frac in (("wan14b_full", "full", 1.0), ("wan14b_chunk", "chunk_causal", 28 / 49)):
         fn = lambda: va.vattn_attention(qd, kd, vd, o, scale=d ** -0.5, mode=mode, tokens_per_frame=F,
                                         chunk_frames=c["chunk_frames"], rope=rope, table=tab, workspace=ws14)
-        fn()
-        ms = _time_events(torch, fn, 3)
+        m = _measure(torch, fn)          # inputs 2.3 GB: far larger than L2
         flops = 4.0 * d * L * L * H * frac
-        out[name] = {"ms": ms, "tflops": flops / ms * 1e-9, "frac_of_peak": flops / ms * 1e-9 / pk["bf16_tflops"]}
+        tf = flops / m["median_ms"] * 1e-9
+        out[name] = dict(m, tflops=tf, frac_of_peak=tf / pk["bf16_tflops"], mask_adjusted_flops=flops)
     del qd, kd, vd, o, ws14
     # streaming decode: 32 frames, ring of 4, window 4
     c = si.CONFIGS["stream"]
@@ -365,46 +412,46 @@ def secondary_measurements(va, torch, device, flush):
             cache.attend(qf, kf, vf, of, f, c["window_back"], rope=rope, table=tab)
             cache.append(kf, vf, f)
 
-    stream_all()
-    ms = _time_events(torch, stream_all, 3)
-    total_flops = 4.0 * d * F * F * H * sum(min(f, c["window_back"]) + 1 for f in range(T))
+    m = _measure(torch, stream_all)
+    pairs_frames = sum(min(f, c["window_back"]) + 1 for f in range(T))   # (q-frame, k-frame) pairs: 150
+    total_flops = 4.0 * d * F * F * H * pairs_frames
+    tf = total_flops / m["median_ms"] * 1e-9
+    fps = T / (m["median_ms"] / 1e3)
+    # ceiling: the whole 32-frame stream's mask-adjusted FLOPs at the
+    # measured bf16 peak; frames/s over the ceiling = TFLOP/s over the peak
+    ceiling_fps = T / (total_flops / (pk["bf16_tflops"] * 1e12))
+    steady_flops = 4.0 * d * F * F * H * (c["window_back"] + 1)
+    stream = dict(m, frames_per_s=fps, ms_per_frame=m["median_ms"] / T, tflops=tf,
+                  frac_of_ceiling=fps / ceiling_fps, ceiling_frames_per_s=ceiling_fps,
+                  ceiling_steady_frames_per_s=pk["bf16_tflops"] * 1e12 / steady_flops,
+                  ceiling_formula="frames/s at the measured bf16 peak = T * peak / (4 d F^2 H * 150); "
+                                  "150 = visible (query frame, key frame) pairs of the 32-frame stream")
     steady = lambda: cache.attend(frames[10][0], frames[10][1], frames[10][2], of, T - 1,
                                   c["window_back"], rope=rope, table=tab)
-    steady()
-    ms_att = _time_events(torch, steady, 10)
-    # KV append, timed as 16 appends of distinct frames (inputs 134 MB, more
-    # than L2) replayed from a CUDA graph.  In the streaming loop the append
-    # after attend is a plain copy (the attend call already rotated the
-    # frame's keys): read k, v; write raw k, v.  An append without a
-    # preceding attend also writes the rotated keys.
-    def graph_appends(cch):
-        g = torch.cuda.CUDAGraph()
-        side = torch.cuda.Stream()
-        side.wait_stream(torch.cuda.current_stream())
-        with torch.cuda.stream(side):
-            cch.append(frames[0][1], frames[0][2], 0)
-            with torch.cuda.graph(g, stream=side):
-                for f in range(16):
-                    cch.append(frames[f][1], frames[f][2], f)
-        torch.cuda.current_stream().wait_stream(side)
-        ms_ = _time_events(torch, g.replay, 5) / 16
-        del g
-        return ms_
-
+    ms_ = _measure(torch, steady)
+    stream["steady_attention"] = dict(ms_, tflops=steady_flops / ms_["median_ms"] * 1e-9,
+                                      frac_of_peak=steady_flops / ms_["median_ms"] * 1e-9 / pk["bf16_tflops"])
+    # KV append of one frame: a single launch after an L2 flush, and 16
+    # appends of distinct frames (inputs 134 MB, more than L2) replayed from
+    # a CUDA graph.  In the streaming loop the append after attend is a
+    # plain copy (the attend call already rotated the frame's keys): read k,
+    # v; write raw k, v.  An append without a preceding attend also writes
+    # the rotated keys.
+    app_bytes = 4 * F * H * d * 2
+    rot_bytes = 5 * F * H * d * 2
     plain = va.KVCache(torch.zeros_like(kr), torch.zeros_like(vr), torch.zeros_like(ids))
-    ms_app = graph_appends(plain)
+    one = _measure(torch, lambda: plain.append(frames[3][1], frames[3][2], 3), flush=flush)
+    g = _graph(torch, [lambda f=f: plain.append(frames[f][1], frames[f][2], f) for f in range(16)])
+    batch = _measure(torch, g.replay, per_call=16)
+    del g
     plain.close()
-    ms_app_rot = graph_appends(cache)
-    app_bytes = 4 * F * H * d * 2          # read k, v; write raw k, v
-    rot_bytes = 5 * F * H * d * 2          # and the rotated k
-    out["stream"] = {"frames_per_s": T / (ms / 1e3), "ms_per_frame": ms / T, "tflops": total_flops / ms * 1e-9,
-                     "steady_attention_ms": ms_att,
-                     "steady_attention_tflops": 4.0 * d * F * F * H * 5 / ms_att * 1e-9,
-                     "append_us": ms_app * 1e3, "append_gbs": app_bytes / (ms_app / 1e3) / 1e9,
-                     "append_frac_of_hbm": app_bytes / (ms_app / 1e3) / 1e9 / pk["hbm_gbs"],
-                     "append_rotated_us": ms_app_rot * 1e3,
-                     "append_rotated_gbs": rot_bytes / (ms_app_rot / 1e3) / 1e9,
-                     "append_rotated_frac_of_hbm": rot_bytes / (ms_app_rot / 1e3) / 1e9 / pk["hbm_gbs"]}
+    g = _graph(torch, [lambda f=f: cache.append(frames[f][1], frames[f][2], f) for f in range(16)])
+    batch_rot = _measure(torch, g.replay, per_call=16)
+    del g
+    stream["append"] = {"single_launch": _hbm(pk, app_bytes, one), "graph16": _hbm(pk, app_bytes, batch),
+                        "rotated_graph16": _hbm(pk, rot_bytes, batch_rot),
+                        "clocks": batch["clocks"]}
+    out["stream"] = stream
     cache.close()
     del qd, kd, vd, kr, vr
     # hybrid chunk attention
@@ -416,14 +463,39 @@ def secondary_measurements(va, torch, device, flush):
     o = torch.empty_like(qd)
     S = torch.zeros((1, H, d, d), dtype=torch.float32, device=device)
     z = torch.zeros((1, H, d), dtype=torch.float32, device=device)
-    ws = torch.empty(va.vattn_hybrid_workspace_bytes(1, L, H, d, ct), dtype=torch.uint8, device=device)
+    wsb = va.vattn_hybrid_workspace_bytes(1, L, H, d, ct)
+    ws = torch.empty(wsb, dtype=torch.uint8, device=device)
     fn = lambda: va.vattn_hybrid_chunk(qd, kd, vd, o, S, z, ct, workspace=ws)
-    fn()
-    ms = _time_events(torch, fn, 5)
+    m = _measure(torch, fn)
     n_ch = (L + ct - 1) // ct
     intra = sum(min(ct, L - i * ct) ** 2 for i in range(n_ch))
-    flops = 4.0 * d * intra * H + (4.0 * d * d + 4.0 * d) * L * H * 2
-    out["hybrid"] = {"ms": ms, "tflops": flops / ms * 1e-9}
+    # softmax part: 4 d per (query, key) pair in the same chunk; state: the
+    # build phi(k) v^T + sum phi(k) (2 d^2 + 2 d per key, as multiply-adds)
+    # and the read-out phi(q)^T S + phi(q) . z (2 d^2 + 2 d per query)
+    flops = 4.0 * d * intra * H + (2.0 * d * d + 2.0 * d) * L * H * 2
+    tf = flops / m["median_ms"] * 1e-9
+    hyb = dict(m, tflops=tf, frac_of_peak=tf / pk["bf16_tflops"], mask_adjusted_flops=flops,
+               flop_formula="4 d sum_c |c|^2 H + (2 d^2 + 2 d) L H (keys) + (2 d^2 + 2 d) L H (queries)")
+    # state delta: reads K and V, writes the per-chunk deltas
+    delta_bytes = 2 * L * H * d * 2 + wsb
+    kd2, vd2 = kd.clone(), vd.clone()      # a second input set: 2 x 149 MB > L2
+    one = _measure(torch, lambda: va.vattn_hybrid_delta(kd, vd, ct, ws), flush=flush)
+    g = _graph(torch, [lambda i=i: va.vattn_hybrid_delta(kd if i % 2 == 0 else kd2, vd if i % 2 == 0 else vd2,
+                                                          ct, ws) for i in range(16)])
+    batch = _measure(torch, g.replay, per_call=16)
+    del g
+    hyb["delta"] = {"single_launch": _hbm(pk, delta_bytes, one), "graph16": _hbm(pk, delta_bytes, batch)}
+    # scan: reads and writes the workspace (in place) and the state in/out;
+    # the graph cycles over 12 workspaces (209 MB, more than L2)
+    scan_bytes = 2 * wsb + 2 * (S.numel() + z.numel()) * 4
+    va.vattn_hybrid_delta(kd, vd, ct, ws)
+    one = _measure(torch, lambda: va.vattn_hybrid_scan(S, z, L, ct, ws), flush=flush)
+    wss = [torch.zeros(wsb, dtype=torch.uint8, device=device) for _ in range(12)]
+    g = _graph(torch, [lambda i=i: va.vattn_hybrid_scan(S, z, L, ct, wss[i % 12]) for i in range(16)])
+    batch = _measure(torch, g.replay, per_call=16)
+    del g, wss
+    hyb["scan"] = {"single_launch": _hbm(pk, scan_bytes, one), "graph16": _hbm(pk, scan_bytes, batch)}
+    out["hybrid"] = hyb
     va.vattn_check()
     return out
 

@@ -133,6 +133,25 @@ vattn_status vattn_attention(const void* q, const void* k, const void* v, void* 
 size_t vattn_attention_workspace_bytes(int B, int Lk, int Hkv, int d, const vattn_rope* rope);
 
 /*
+ * Exact combination of R partial attentions of the same queries over
+ * disjoint key sets (the join of Ring attention's key shards in unified
+ * sequence parallelism, ReGenVC "Unified sequence parallelism", Sec. 3.5;
+ * numerically equivalent to one attention over all keys up to reduction
+ * order):
+ *   o = sum_r e^{lse_r - M} o_r / sum_r e^{lse_r - M},  M = max_r lse_r,
+ *   lse = M + ln sum_r e^{lse_r - M}.
+ *   o_parts bf16 [R][B][L][H][d] and lse_parts fp32 [R][B][H][L]: the o and
+ *   lse outputs of R vattn_attention calls (one per key shard), stacked;
+ *   o bf16 [B][L][H][d]; lse (nullable) fp32 [B][H][L].  A part whose keys
+ *   were all invisible to a row (lse = -inf) has weight 0; a row with no
+ *   visible key in any part gets o = 0, lse = -inf.  1 <= R <= 64; d a
+ *   multiple of 8; o_parts and o 16-byte aligned.  One HBM pass (16-byte
+ *   vectors), asynchronous on `stream`.
+ */
+vattn_status vattn_attention_merge(const void* o_parts, const float* lse_parts, int R, void* o, float* lse, int B,
+                                   int L, int H, int d, vattn_stream stream);
+
+/*
  * Rolling KV cache of a fixed number of frames (FlashDecoder "Streaming with
  * Rolling KV Cache", Sec. 3.3; constant memory regardless of video length,
  * "Long Video Decoding", Sec. 4.3).  Storage is caller-owned device memory:
@@ -216,6 +235,26 @@ vattn_status vattn_hybrid_chunk(const void* q, const void* k, const void* v, voi
                                 float* z, int B, int L, int H, int d, int chunk_tokens,
                                 float scale, void* workspace, size_t workspace_bytes,
                                 vattn_stream stream);
+
+/*
+ * The state part of vattn_hybrid_chunk as two separate calls, for callers
+ * that advance the recurrent state without computing outputs (MobileWan's
+ * RNN form of causal linear attention: S_{c+1} = S_c + phi(K_c)^T V_c,
+ * z_{c+1} = z_c + sum phi(k)).  Same workspace and layouts as
+ * vattn_hybrid_chunk:
+ *  - vattn_hybrid_delta writes, for every chunk c of k/v ([B][L][H][d]
+ *    bf16), dS_c = phi(K_c)^T V_c (fp32 [C][B][H][d][d]) and
+ *    dz_c = sum phi(k) (fp32 [C][B][H][d]) into the workspace (tensor-core
+ *    MMA, one pass over K and V);
+ *  - vattn_hybrid_scan then replaces them in place by the exclusive prefix
+ *    S_c = S_in + sum_{c' < c} dS_c' (same for z) and leaves S, z (in/out)
+ *    as the state after the last chunk (one pass of coalesced 16-byte
+ *    loads and stores).
+ */
+vattn_status vattn_hybrid_delta(const void* k, const void* v, int B, int L, int H, int d, int chunk_tokens,
+                                void* workspace, size_t workspace_bytes, vattn_stream stream);
+vattn_status vattn_hybrid_scan(float* S, float* z, int B, int L, int H, int d, int chunk_tokens, void* workspace,
+                               size_t workspace_bytes, vattn_stream stream);
 
 /*
  * vattn_hybrid_chunk without a caller workspace.  The pages have no

@@ -30,6 +30,36 @@ vattn_status vattn_selftest_umma(int variant, const void* a, const void* b, floa
  * and the context stays usable.  Nothing faults, traps or hangs.
  */
 vattn_status vattn_selftest_wait_timeout(uint32_t limit_us, vattn_stream stream);
+
+/*
+ * The same check inside the two-tile attention kernel (no counterpart in the
+ * pages).  One full-attention call without RoPE (B = 1, Hkv = H, scale
+ * 1/sqrt(d)) on q, k, v, o bf16 [1][L][H][d] (device, 16-byte aligned),
+ * L >= 256, with every wait bounded by limit_us microseconds (1..2000000)
+ * instead of two seconds, and with the first softmax warp of each CTA's
+ * first query tile withholding its arrival for score sub-tile 1.  That
+ * tile's MMA issuer waits for it until the bound runs out, raises the CTA's
+ * abort and records a code in the status word; every other role leaves its
+ * loop, waits (bounded) for its copies and MMAs in flight, the CTA frees its
+ * TMEM and returns.  The following vattn_check() reports VATTN_ERR_TIMEOUT;
+ * o is left partly unwritten.  Nothing faults, traps or hangs.
+ */
+vattn_status vattn_selftest_attention_timeout(const void* q, const void* k, const void* v, void* o, int L,
+                                              int H, int d, uint32_t limit_us, vattn_stream stream);
+
+/*
+ * The softmax exponentials, element by element (no counterpart in the
+ * pages; checks the exp2 the kernels use):
+ *   variant 0: y[i] = 2^x[i] by the FMA-pipe polynomial (Cody-Waite
+ *              reduction, degree-3 minimax, relative error < 7.6e-5 for
+ *              x >= -125; arguments below -125 give a value in
+ *              [0, 2^-124]);
+ *   variant 1: the same on pairs (x[2i], x[2i+1]) in packed fp32x2 form
+ *              (n even);
+ *   variant 2: y[i] = ex2.approx.ftz(x[i]) (MUFU).
+ * x, y: device fp32 [n].
+ */
+vattn_status vattn_selftest_ex2(int variant, const float* x, float* y, int n, vattn_stream stream);
 #ifdef __cplusplus
 }
 #endif

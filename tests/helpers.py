@@ -42,3 +42,46 @@ def assert_parity(got, ref, what="", max_abs=MAX_ABS, rel_l2=REL_L2):
 def gather_rows(o, rows):
     """o [B, L, H, d] (numpy) at rows (b, h, i) -> [n, d]."""
     return np.stack([o[b, i, h] for b, h, i in rows])
+
+
+# ------------------------------------------------------------ guard regions
+# Every output, ring and state buffer a GPU test hands to the library sits
+# inside a larger allocation whose first and last GUARD_BYTES hold a fixed
+# byte pattern; check_guards() after a call proves that nothing was written
+# past either end of the buffer.
+GUARD_BYTES = 4096
+GUARD_BYTE = 0xA5
+
+
+class Guarded:
+    """A contiguous tensor of `shape`/`dtype` with guard regions around it."""
+
+    def __init__(self, shape, dtype, fill=0.0, device="cuda"):
+        import torch
+        itemsize = torch.empty((), dtype=dtype).element_size()
+        self.g = GUARD_BYTES // itemsize
+        n = int(np.prod(shape)) if len(shape) else 1
+        self.buf = torch.empty(n + 2 * self.g, dtype=dtype, device=device)
+        self.buf.view(torch.uint8).fill_(GUARD_BYTE)
+        self.t = self.buf[self.g:self.g + n].view(shape)
+        if fill is not None:
+            self.t.fill_(fill)
+
+    def check(self, what=""):
+        import torch
+        raw = self.buf.view(torch.uint8)
+        nb = self.g * self.buf.element_size()
+        head, tail = raw[:nb], raw[raw.numel() - nb:]
+        bad_head = int((head != GUARD_BYTE).sum())
+        bad_tail = int((tail != GUARD_BYTE).sum())
+        assert bad_head == 0 and bad_tail == 0, (
+            "%s: %d guard bytes before and %d after the buffer were overwritten" % (what, bad_head, bad_tail))
+
+
+def guarded(shape, dtype, fill=0.0, device="cuda"):
+    return Guarded(tuple(shape), dtype, fill, device)
+
+
+def check_guards(*gs, what=""):
+    for g in gs:
+        g.check(what)

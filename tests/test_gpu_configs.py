@@ -7,7 +7,7 @@ import pytest
 
 import oracle
 import seeded_inputs as si
-from helpers import assert_parity, from_dev, gather_rows, to_dev
+from helpers import assert_parity, check_guards, from_dev, gather_rows, guarded, to_dev
 
 pytestmark = pytest.mark.gpu
 N_ROWS = 4096
@@ -33,11 +33,13 @@ def test_large_attention_sampled_rows(va, name, mode):
     (q, k, v), (qd, kd, vd) = _dev_qkv(name)
     rope = va.Rope(Hg=Hg, Wg=Wg, pairs=c["pairs"], max_pos=max(T, Hg, Wg), theta=c["theta"])
     tab = va.rope_table(rope, d)
-    o = torch.full(qd.shape, float("nan"), dtype=torch.bfloat16, device="cuda")
+    go = guarded(qd.shape, torch.bfloat16, float("nan"))
+    o = go.t
     chunk = c.get("chunk_frames", 1)
     va.vattn_attention(qd, kd, vd, o, scale=d ** -0.5, mode=mode, tokens_per_frame=F,
                        chunk_frames=chunk, rope=rope, table=tab)
     va.vattn_check()
+    check_guards(go, what="%s %s o" % (name, mode))
     period = F * chunk if mode == "chunk_causal" else F
     rows = si.sample_rows(0x5EED0000 + 16 * c["index"] + 7, N_ROWS, 1, H, L,
                           forced=si.boundary_tokens(L, period))
@@ -56,11 +58,11 @@ def test_stream_config_sampled_rows(va):
     (q, k, v), (qd, kd, vd) = _dev_qkv("stream")
     rope = va.Rope(Hg=Hg, Wg=Wg, pairs=c["pairs"], max_pos=64, theta=c["theta"])
     tab = va.rope_table(rope, d)
-    kr = torch.zeros((cap, 1, F, H, d), dtype=torch.bfloat16, device="cuda")
-    vr = torch.zeros_like(kr)
-    ids = torch.zeros(cap, dtype=torch.int32, device="cuda")
+    gk, gv = guarded((cap, 1, F, H, d), torch.bfloat16), guarded((cap, 1, F, H, d), torch.bfloat16)
+    gi, gr = guarded((cap,), torch.int32, 0), guarded((cap + 1, 1, F, H, d), torch.bfloat16)
+    kr, vr, ids = gk.t, gv.t, gi.t
     cache = va.KVCache(kr, vr, ids)
-    cache.enable_rope(torch.zeros((cap + 1, 1, F, H, d), dtype=torch.bfloat16, device="cuda"), rope, tab)
+    cache.enable_rope(gr.t, rope, tab)
     o = torch.full(qd.shape, float("nan"), dtype=torch.bfloat16, device="cuda")
     for f in range(T):
         sl = slice(f * F, (f + 1) * F)
@@ -70,6 +72,7 @@ def test_stream_config_sampled_rows(va):
         cache.append(kf, vf, f)
         o[:, sl] = of
     va.vattn_check()
+    check_guards(gk, gv, gi, gr, what="stream config ring")
     # ring holds frames 28..31 bit for bit
     kb = k.reshape(T, F, H, d)
     for slot in range(cap):
@@ -90,11 +93,12 @@ def test_hybrid_config(va):
     T, Hg, Wg, H, d = c["T"], c["Hg"], c["Wg"], c["H"], c["d"]
     L, ct = T * Hg * Wg, c["chunk_frames"] * Hg * Wg
     (q, k, v), (qd, kd, vd) = _dev_qkv("hybrid")
-    S = torch.zeros((1, H, d, d), dtype=torch.float32, device="cuda")
-    z = torch.zeros((1, H, d), dtype=torch.float32, device="cuda")
-    o = torch.full(qd.shape, float("nan"), dtype=torch.bfloat16, device="cuda")
+    gS, gz = guarded((1, H, d, d), torch.float32), guarded((1, H, d), torch.float32)
+    go = guarded(qd.shape, torch.bfloat16, float("nan"))
+    S, z, o = gS.t, gz.t, go.t
     va.vattn_hybrid_chunk(qd, kd, vd, o, S, z, ct, scale=d ** -0.5)
     va.vattn_check()
+    check_guards(gS, gz, go, what="hybrid config o / S / z")
     rows = si.sample_rows(0x5EED0000 + 16 * 3 + 7, N_ROWS, 1, H, L, forced=si.boundary_tokens(L, ct))
     mask = np.zeros((1, H, L), dtype=bool)
     mask[rows[:, 0], rows[:, 1], rows[:, 2]] = True

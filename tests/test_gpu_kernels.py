@@ -6,7 +6,7 @@ import pytest
 
 import oracle
 import seeded_inputs as si
-from helpers import assert_parity, bits_of, errors, from_dev, gather_rows, to_dev
+from helpers import assert_parity, bits_of, check_guards, errors, from_dev, gather_rows, guarded, to_dev
 
 pytestmark = pytest.mark.gpu
 LSE_TOL = 1e-2
@@ -82,8 +82,9 @@ def _attention_case(va, B, T, Hg, Wg, H, Hkv, d, mode, kw, use_rope, seed=0, qof
     k = si.normal_bf16(11 + seed, (B, L, Hkv, d))
     v = si.normal_bf16(12 + seed, (B, L, Hkv, d))
     scale = d ** -0.5
-    o = torch.full((B, L, H, d), float("nan"), dtype=torch.bfloat16, device="cuda")
-    lse = torch.full((B, H, L), float("nan"), dtype=torch.float32, device="cuda")
+    og = guarded((B, L, H, d), torch.bfloat16, float("nan"))
+    lg = guarded((B, H, L), torch.float32, float("nan"))
+    o, lse = og.t, lg.t
     rope = tab = None
     orope = None
     pairs = (12, 10, 10) if d == 64 else (22, 21, 21)
@@ -97,6 +98,7 @@ def _attention_case(va, B, T, Hg, Wg, H, Hkv, d, mode, kw, use_rope, seed=0, qof
                        q_frame_offset=qoff, k_frame_offset=koff, rope=rope, table=tab,
                        fuse_k_rope=fuse_k)
     va.vattn_check()
+    check_guards(og, lg, what="attention o / lse")
     ro, rl = oracle.attention(q, k, v, scale, mode=mode, F=F, chunk=kw.get("chunk", 1),
                               wb=kw.get("wb", 0), wf=kw.get("wf", 0), q_frame_offset=qoff,
                               k_frame_offset=koff, rope=orope)
@@ -157,3 +159,60 @@ def test_bounded_wait_reports_timeout_and_context_survives(va):
     va.vattn_check()
     ref, _ = oracle.attention(q, k, v, 0.125)
     assert_parity(from_dev(o), ref, "after timeout")
+
+
+def test_bounded_wait_in_the_attention_kernel(va):
+    # The real two-tile kernel with one softmax arrival withheld and a 5 ms
+    # wait bound: tile A's MMA issuer gives up, the CTA tears down (drains its
+    # copies and MMAs, frees TMEM) and returns; the status word reports a
+    # timeout, and the next normal call on the same context is correct.
+    import torch
+    va.vattn_check()
+    for d in (64, 128):
+        L, H = 512, 2
+        q = si.normal_bf16(80, (1, L, H, d))
+        k = si.normal_bf16(81, (1, L, H, d))
+        v = si.normal_bf16(82, (1, L, H, d))
+        qd, kd, vd = to_dev(q), to_dev(k), to_dev(v)
+        o = torch.zeros((1, L, H, d), dtype=torch.bfloat16, device="cuda")
+        va.vattn_selftest_attention_timeout(qd, kd, vd, o, 5000)
+        with pytest.raises(va.VattnError) as e:
+            va.vattn_check()
+        assert e.value.status == va.ERR_TIMEOUT
+        va.vattn_check()                               # cleared
+        og = guarded((1, L, H, d), torch.bfloat16, float("nan"))
+        va.vattn_attention(qd, kd, vd, og.t, scale=d ** -0.5)
+        va.vattn_check()
+        check_guards(og, what="attention after timeout")
+        ref, _ = oracle.attention(q, k, v, d ** -0.5)
+        assert_parity(from_dev(og.t), ref, "attention after an aborted launch (d=%d)" % d)
+
+
+def test_exp2_functions_against_fp64(va):
+    # The softmax's exponentials over the whole range they see (arguments
+    # are <= 8 after the running-max subtraction, far below it for masked
+    # or stale entries): the FMA-pipe polynomial within its stated relative
+    # bound for x >= -125 and a value in [0, 2^-124] below, the packed form
+    # equal to the scalar one bit for bit, MUFU ex2 within 2^-20 relative.  (The Remez fit's bound is 7.48e-5 in exact arithmetic; the
+    # fp32 evaluation of the polynomial adds at most a few 1e-7.)
+    import torch
+    x = np.concatenate([np.linspace(-130.0, 64.0, 400001), np.arange(-130, 64, dtype=np.float64),
+                        np.arange(-130, 64, dtype=np.float64) + 0.5,
+                        si.normal_f64(0xE2, 100000) * 8.0]).astype(np.float32)
+    x = x[: len(x) // 2 * 2]
+    xd = torch.from_numpy(x).cuda()
+    ys = {}
+    for variant in (0, 1, 2):
+        y = torch.full_like(xd, float("nan"))
+        va.vattn_selftest_ex2(variant, xd, y)
+        va.vattn_check()
+        ys[variant] = y.cpu().numpy()
+    exact = np.exp2(x.astype(np.float64))
+    inr = x >= -125.0
+    rel = np.abs(ys[0][inr] - exact[inr]) / exact[inr]
+    assert rel.max() <= 7.6e-5, "polynomial exp2: max relative error %.3e" % rel.max()
+    low = ys[0][~inr].astype(np.float64)
+    assert np.all((low >= 0.0) & (low <= 2.0 ** -124)), "arguments below -125 give a value in [0, 2^-124]"
+    assert np.array_equal(ys[0].view(np.uint32), ys[1].view(np.uint32)), "packed and scalar forms differ"
+    relm = np.abs(ys[2][inr] - exact[inr]) / exact[inr]
+    assert relm.max() <= 2.0 ** -20, "ex2.approx: max relative error %.3e" % relm.max()

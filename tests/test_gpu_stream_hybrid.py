@@ -5,7 +5,7 @@ import pytest
 
 import oracle
 import seeded_inputs as si
-from helpers import assert_parity, bits_of, from_dev, gather_rows, to_dev
+from helpers import assert_parity, bits_of, check_guards, from_dev, gather_rows, guarded, to_dev
 
 pytestmark = pytest.mark.gpu
 
@@ -21,23 +21,30 @@ def _run_stream(va, q, k, v, F, H, Hkv, d, cap, wb, rope, tab, check_ring=None, 
     import torch
     B, L = q.shape[0], q.shape[1]
     T = L // F
-    kr = torch.zeros((cap, B, F, Hkv, d), dtype=torch.bfloat16, device="cuda")
-    vr = torch.zeros_like(kr)
-    ids = torch.zeros(cap, dtype=torch.int32, device="cuda")
+    g_k = guarded((cap, B, F, Hkv, d), torch.bfloat16)
+    g_v = guarded((cap, B, F, Hkv, d), torch.bfloat16)
+    g_ids = guarded((cap,), torch.int32, 0)
+    kr, vr, ids = g_k.t, g_v.t, g_ids.t
+    guards = [g_k, g_v, g_ids]
     cache = va.KVCache(kr, vr, ids)
     if rot_ring:
-        cache.enable_rope(torch.zeros((cap + 1, B, F, Hkv, d), dtype=torch.bfloat16, device="cuda"), rope, tab)
+        g_rot = guarded((cap + 1, B, F, Hkv, d), torch.bfloat16)
+        guards.append(g_rot)
+        cache.enable_rope(g_rot.t, rope, tab)
     qd, kd, vd = to_dev(q), to_dev(k), to_dev(v)
     o = torch.full((B, L, H, d), float("nan"), dtype=torch.bfloat16, device="cuda")
+    g_o = guarded((B, F, H, d), torch.bfloat16, float("nan"))
+    guards.append(g_o)
     for f in range(T):
         sl = slice(f * F, (f + 1) * F)
         qf, kf, vf = qd[:, sl].contiguous(), kd[:, sl].contiguous(), vd[:, sl].contiguous()
-        of = torch.empty((B, F, H, d), dtype=torch.bfloat16, device="cuda")
+        of = g_o.t
         cache.attend(qf, kf, vf, of, f, wb, scale=d ** -0.5, rope=rope, table=tab)
         cache.append(kf, vf, f)
         o[:, sl] = of
         if check_ring is not None:
             check_ring(f, kr, vr, ids, cache)
+        check_guards(*guards, what="stream frame %d" % f)
     va.vattn_check()
     cache.close()
     return o
@@ -94,11 +101,12 @@ def test_hybrid_parity_all_rows(va, L, chunk):
     q = si.normal_bf16(51, (1, L, H, d))
     k = si.normal_bf16(52, (1, L, H, d))
     v = si.normal_bf16(53, (1, L, H, d))
-    S = torch.zeros((1, H, d, d), dtype=torch.float32, device="cuda")
-    z = torch.zeros((1, H, d), dtype=torch.float32, device="cuda")
-    o = torch.full((1, L, H, d), float("nan"), dtype=torch.bfloat16, device="cuda")
+    gS, gz = guarded((1, H, d, d), torch.float32), guarded((1, H, d), torch.float32)
+    go = guarded((1, L, H, d), torch.bfloat16, float("nan"))
+    S, z, o = gS.t, gz.t, go.t
     va.vattn_hybrid_chunk(to_dev(q), to_dev(k), to_dev(v), o, S, z, chunk, scale=d ** -0.5)
     va.vattn_check()
+    check_guards(gS, gz, go, what="hybrid o / S / z")
     ro, rS, rz = oracle.hybrid_recurrent(q, k, v, chunk, d ** -0.5)
     assert_parity(from_dev(o), ro, "hybrid o")
     assert_parity(S.cpu().numpy(), rS, "hybrid S", max_abs=np.inf)

@@ -75,6 +75,7 @@ _rope_qk = _sig("vattn_rope_qk", _I, _P, _P, _P, _P, _I, _I, _I, _I, _I, _RP, _P
 _attention = _sig("vattn_attention", _I, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _I, _I, _I,
                   _I, _I, _I, _I, _RP, _P, _P, _S, _P)
 _attn_ws = _sig("vattn_attention_workspace_bytes", _S, _I, _I, _I, _I, _RP)
+_merge = _sig("vattn_attention_merge", _I, _P, _P, _I, _P, _P, _I, _I, _I, _I, _P)
 _kv_init = _sig("vattn_kvcache_init", _I, ctypes.POINTER(_P), _P, _P, _P, _I, _I, _I, _I, _I, _P)
 _kv_append = _sig("vattn_kvcache_append", _I, _P, _P, _P, _I, _P)
 _attention_stream = _sig("vattn_attention_stream", _I, _P, _P, _P, _P, _P, _P, _I, _I, _I, _F, _RP,
@@ -85,9 +86,14 @@ _kv_rope = _sig("vattn_kvcache_enable_rope", _I, _P, _P, _RP, _P, _P)
 _kv_destroy = _sig("vattn_kvcache_destroy", _I, _P)
 _hyb_ws = _sig("vattn_hybrid_workspace_bytes", _S, _I, _I, _I, _I, _I)
 _hybrid = _sig("vattn_hybrid_chunk", _I, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _P, _S, _P)
+_hybrid_delta = _sig("vattn_hybrid_delta", _I, _P, _P, _I, _I, _I, _I, _I, _P, _S, _P)
+_hybrid_scan = _sig("vattn_hybrid_scan", _I, _P, _P, _I, _I, _I, _I, _I, _P, _S, _P)
 _hybrid_noalloc = _sig("vattn_hybrid_chunk_noalloc", _I, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _P)
 _selftest = _sig("vattn_selftest_umma", _I, _I, _P, _P, _P, _P)
 _selftest_timeout = _sig("vattn_selftest_wait_timeout", _I, ctypes.c_uint32, _P)
+_selftest_attn_timeout = _sig("vattn_selftest_attention_timeout", _I, _P, _P, _P, _P, _I, _I, _I,
+                              ctypes.c_uint32, _P)
+_selftest_ex2 = _sig("vattn_selftest_ex2", _I, _I, _P, _P, _I, _P)
 HYBRID_NOALLOC_MAX_BYTES = 32 << 20
 
 
@@ -104,9 +110,9 @@ def _ok(status: int):
         raise VattnError(status, last_error())
 
 
-def _stream(stream=None) -> int:
+def _stream(stream=None, device=None) -> int:
     if stream is None:
-        stream = torch.cuda.current_stream()
+        stream = torch.cuda.current_stream(device)
     return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
 
 
@@ -126,6 +132,55 @@ def _bf16(t, name):
     return _ptr(t)
 
 
+# Argument checks of the wrappers.  They run before any pointer is taken or
+# anything is launched: a tensor whose shape or dtype disagrees with the
+# call would otherwise be read or written past its end by the kernels, and
+# the library runs on the device of the first tensor, so every tensor must
+# live there.
+def _expect(t, name, shape, dtype):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError("%s must be a torch tensor" % name)
+    if t.dtype != dtype:
+        raise TypeError("%s must be %s (got %s)" % (name, dtype, t.dtype))
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError("%s must have shape %s (got %s)" % (name, tuple(shape), tuple(t.shape)))
+    if not t.is_contiguous():
+        raise ValueError("%s must be contiguous" % name)
+
+
+def _min_bytes(t, name, nbytes):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError("%s must be a torch tensor" % name)
+    if not t.is_contiguous():
+        raise ValueError("%s must be contiguous" % name)
+    have = t.numel() * t.element_size()
+    if have < nbytes:
+        raise ValueError("%s holds %d bytes, %d needed" % (name, have, nbytes))
+
+
+def _rank(t, name, n):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError("%s must be a torch tensor" % name)
+    if t.dim() != n:
+        raise ValueError("%s must have %d dimensions (got shape %s)" % (name, n, tuple(t.shape)))
+
+
+def _device(*named):
+    """The common CUDA device of the given (name, tensor) pairs (None entries
+    are skipped); raises if one is not on CUDA or they differ."""
+    dev = None
+    for name, t in named:
+        if t is None:
+            continue
+        if not t.is_cuda:
+            raise ValueError("%s must be on a CUDA device (got %s)" % (name, t.device))
+        if dev is None:
+            dev = t.device
+        elif t.device != dev:
+            raise ValueError("%s is on %s, the other tensors on %s" % (name, t.device, dev))
+    return dev
+
+
 def _rope_c(rope):
     if rope is None:
         return None
@@ -138,7 +193,15 @@ def vattn_rope_table_bytes(rope: Rope, d: int) -> int:
 
 
 def vattn_rope_table_build(rope: Rope, d: int, table: torch.Tensor, stream=None):
-    _ok(_table_build(ctypes.byref(rope.c()), d, _ptr(table), _stream(stream)))
+    n = vattn_rope_table_bytes(rope, d)
+    if n == 0:
+        raise VattnError(ERR_INVALID_ARG, last_error())
+    if table.dtype != torch.float32:
+        raise TypeError("table must be float32")
+    _min_bytes(table, "table", n)
+    dev = _device(("table", table))
+    with torch.cuda.device(dev):
+        _ok(_table_build(ctypes.byref(rope.c()), d, _ptr(table), _stream(stream, dev)))
 
 
 def rope_table(rope: Rope, d: int, device="cuda") -> torch.Tensor:
@@ -152,14 +215,28 @@ def rope_table(rope: Rope, d: int, device="cuda") -> torch.Tensor:
 
 
 def vattn_rope_qk(q, k, q_out, k_out, rope: Rope, table, frame_offset=0, stream=None):
+    """3D-RoPE of q [B, L, H, d] into q_out and of k [B, L, Hkv, d] into k_out
+    (either pair may be None)."""
+    if (q is None) != (q_out is None) or (k is None) != (k_out is None):
+        raise ValueError("q/q_out and k/k_out go together")
     ref = q if q is not None else k
-    B, L = ref.shape[0], ref.shape[1]
-    d = ref.shape[3]
+    if ref is None:
+        raise ValueError("q or k must be given")
+    _rank(ref, "q" if q is not None else "k", 4)
+    B, L, _, d = ref.shape
     H = q.shape[2] if q is not None else 1
     Hkv = k.shape[2] if k is not None else 1
-    _ok(_rope_qk(_bf16(q, "q") if q is not None else None, _bf16(k, "k") if k is not None else None,
-                 _ptr(q_out), _ptr(k_out), B, L, H, Hkv, d, _rope_c(rope), _ptr(table),
-                 frame_offset, _stream(stream)))
+    if q is not None:
+        _expect(q, "q", (B, L, H, d), torch.bfloat16)
+        _expect(q_out, "q_out", (B, L, H, d), torch.bfloat16)
+    if k is not None:
+        _expect(k, "k", (B, L, Hkv, d), torch.bfloat16)
+        _expect(k_out, "k_out", (B, L, Hkv, d), torch.bfloat16)
+    _expect(table, "table", None, torch.float32)
+    dev = _device(("q", q), ("k", k), ("q_out", q_out), ("k_out", k_out), ("table", table))
+    with torch.cuda.device(dev):
+        _ok(_rope_qk(_ptr(q), _ptr(k), _ptr(q_out), _ptr(k_out), B, L, H, Hkv, d, _rope_c(rope),
+                     _ptr(table), frame_offset, _stream(stream, dev)))
 
 
 # -------------------------------------------------------------- attention
@@ -177,21 +254,53 @@ def vattn_attention(q, k, v, o, lse=None, scale=None, mode="full", tokens_per_fr
     torch when not given); fuse_k_rope=True passes no workspace, so the kernel
     rotates every K tile in shared memory instead.
     """
+    _rank(q, "q", 4)
+    _rank(k, "k", 4)
     B, Lq, H, d = q.shape
     Lk, Hkv = k.shape[1], k.shape[2]
+    _expect(q, "q", None, torch.bfloat16)
+    _expect(k, "k", (B, Lk, Hkv, d), torch.bfloat16)
+    _expect(v, "v", (B, Lk, Hkv, d), torch.bfloat16)
+    _expect(o, "o", (B, Lq, H, d), torch.bfloat16)
+    if lse is not None:
+        _expect(lse, "lse", (B, H, Lq), torch.float32)
+    if (rope is None) != (table is None):
+        raise ValueError("rope and table go together")
+    if table is not None:
+        _expect(table, "table", None, torch.float32)
+        _min_bytes(table, "table", vattn_rope_table_bytes(rope, d))
     if scale is None:
         scale = d ** -0.5
     m = MODES[mode] if isinstance(mode, str) else int(mode)
+    dev = _device(("q", q), ("k", k), ("v", v), ("o", o), ("lse", lse), ("table", table),
+                  ("workspace", workspace))
     ws_ptr, ws_bytes = None, 0
     if rope is not None and not fuse_k_rope:
         need = vattn_attention_workspace_bytes(B, Lk, Hkv, d, rope)
         if workspace is None:
-            workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+            workspace = torch.empty(need, dtype=torch.uint8, device=dev)
+        _min_bytes(workspace, "workspace", need)
         ws_ptr, ws_bytes = _ptr(workspace), workspace.numel() * workspace.element_size()
-    _ok(_attention(_bf16(q, "q"), _bf16(k, "k"), _bf16(v, "v"), _bf16(o, "o"), _ptr(lse), B, Lq, Lk,
-                   H, Hkv, d, float(scale), m, tokens_per_frame, chunk_frames, window_back,
-                   window_fwd, q_frame_offset, k_frame_offset, _rope_c(rope), _ptr(table), ws_ptr,
-                   ws_bytes, _stream(stream)))
+    with torch.cuda.device(dev):
+        _ok(_attention(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, Lq, Lk, H, Hkv, d, float(scale), m,
+                       tokens_per_frame, chunk_frames, window_back, window_fwd, q_frame_offset,
+                       k_frame_offset, _rope_c(rope), _ptr(table), ws_ptr, ws_bytes, _stream(stream, dev)))
+
+
+def vattn_attention_merge(o_parts, lse_parts, o, lse=None, stream=None):
+    """Exact combination of R partial attentions over disjoint key sets:
+    o_parts bf16 [R, B, L, H, d], lse_parts fp32 [R, B, H, L] -> o [B, L, H, d]
+    (and lse [B, H, L])."""
+    _rank(o_parts, "o_parts", 5)
+    R, B, L, H, d = o_parts.shape
+    _expect(o_parts, "o_parts", None, torch.bfloat16)
+    _expect(lse_parts, "lse_parts", (R, B, H, L), torch.float32)
+    _expect(o, "o", (B, L, H, d), torch.bfloat16)
+    if lse is not None:
+        _expect(lse, "lse", (B, H, L), torch.float32)
+    dev = _device(("o_parts", o_parts), ("lse_parts", lse_parts), ("o", o), ("lse", lse))
+    with torch.cuda.device(dev):
+        _ok(_merge(_ptr(o_parts), _ptr(lse_parts), R, _ptr(o), _ptr(lse), B, L, H, d, _stream(stream, dev)))
 
 
 # ---------------------------------------------------------------- KV ring
@@ -202,14 +311,19 @@ class KVCache:
     """
 
     def __init__(self, k_ring, v_ring, frame_ids, stream=None):
+        self._h = None
+        _rank(k_ring, "k_ring", 5)
         cap, B, F, Hkv, d = k_ring.shape
-        if frame_ids.dtype != torch.int32:
-            raise TypeError("frame_ids must be int32")
+        _expect(k_ring, "k_ring", None, torch.bfloat16)
+        _expect(v_ring, "v_ring", (cap, B, F, Hkv, d), torch.bfloat16)
+        _expect(frame_ids, "frame_ids", (cap,), torch.int32)
+        self.device = _device(("k_ring", k_ring), ("v_ring", v_ring), ("frame_ids", frame_ids))
         self.k_ring, self.v_ring, self.frame_ids = k_ring, v_ring, frame_ids
         self.capacity, self.B, self.F, self.Hkv, self.d = cap, B, F, Hkv, d
         h = ctypes.c_void_p()
-        _ok(_kv_init(ctypes.byref(h), _bf16(k_ring, "k_ring"), _bf16(v_ring, "v_ring"), _ptr(frame_ids),
-                     cap, B, F, Hkv, d, _stream(stream)))
+        with torch.cuda.device(self.device):
+            _ok(_kv_init(ctypes.byref(h), _ptr(k_ring), _ptr(v_ring), _ptr(frame_ids), cap, B, F, Hkv, d,
+                         _stream(stream, self.device)))
         self._h = h
 
     def append(self, k, v, frame_idx, stream=None):
@@ -226,14 +340,23 @@ class KVCache:
         return list(arr)
 
     def restore(self, host_ids, stream=None):
+        if len(host_ids) != self.capacity:
+            raise ValueError("host_ids must have %d entries" % self.capacity)
         arr = (ctypes.c_int32 * self.capacity)(*host_ids)
-        _ok(_kv_restore(self._h, arr, _stream(stream)))
+        with torch.cuda.device(self.device):
+            _ok(_kv_restore(self._h, arr, _stream(stream, self.device)))
 
     def enable_rope(self, k_ring_rot, rope: Rope, table, stream=None):
         """Rotated-key ring (bf16 [capacity + 1, B, F, Hkv, d]): keys rotated once per frame."""
+        _expect(k_ring_rot, "k_ring_rot", (self.capacity + 1, self.B, self.F, self.Hkv, self.d), torch.bfloat16)
+        _expect(table, "table", None, torch.float32)
+        _min_bytes(table, "table", vattn_rope_table_bytes(rope, self.d))
+        if _device(("k_ring_rot", k_ring_rot), ("table", table)) != self.device:
+            raise ValueError("k_ring_rot and table must be on the cache's device %s" % self.device)
         self.k_ring_rot = k_ring_rot
-        _ok(_kv_rope(self._h, _bf16(k_ring_rot, "k_ring_rot"), ctypes.byref(rope.c()), _ptr(table),
-                     _stream(stream)))
+        with torch.cuda.device(self.device):
+            _ok(_kv_rope(self._h, _ptr(k_ring_rot), ctypes.byref(rope.c()), _ptr(table),
+                         _stream(stream, self.device)))
 
     def close(self):
         if getattr(self, "_h", None):
@@ -247,18 +370,47 @@ class KVCache:
             pass
 
 
+def _frame_shape(cache, heads):
+    return (cache.B, cache.F, heads, cache.d)
+
+
+def _same_device(cache, *named):
+    dev = _device(*named)
+    if dev is not None and dev != cache.device:
+        raise ValueError("tensors are on %s, the cache on %s" % (dev, cache.device))
+    return cache.device
+
+
 def vattn_kvcache_append(cache: KVCache, k, v, frame_idx, stream=None):
-    _ok(_kv_append(cache._h, _bf16(k, "k"), _bf16(v, "v"), frame_idx, _stream(stream)))
+    _expect(k, "k", _frame_shape(cache, cache.Hkv), torch.bfloat16)
+    _expect(v, "v", _frame_shape(cache, cache.Hkv), torch.bfloat16)
+    dev = _same_device(cache, ("k", k), ("v", v))
+    with torch.cuda.device(dev):
+        _ok(_kv_append(cache._h, _ptr(k), _ptr(v), frame_idx, _stream(stream, dev)))
 
 
 def vattn_attention_stream(cache: KVCache, q, k_cur, v_cur, o, lse, frame_idx, window_back,
                            scale=None, rope=None, table=None, stream=None):
+    _rank(q, "q", 4)
     H = q.shape[2]
+    _expect(q, "q", _frame_shape(cache, H), torch.bfloat16)
+    _expect(k_cur, "k_cur", _frame_shape(cache, cache.Hkv), torch.bfloat16)
+    _expect(v_cur, "v_cur", _frame_shape(cache, cache.Hkv), torch.bfloat16)
+    _expect(o, "o", _frame_shape(cache, H), torch.bfloat16)
+    if lse is not None:
+        _expect(lse, "lse", (cache.B, H, cache.F), torch.float32)
+    if (rope is None) != (table is None):
+        raise ValueError("rope and table go together")
+    if table is not None:
+        _expect(table, "table", None, torch.float32)
+        _min_bytes(table, "table", vattn_rope_table_bytes(rope, cache.d))
     if scale is None:
         scale = cache.d ** -0.5
-    _ok(_attention_stream(cache._h, _bf16(q, "q"), _bf16(k_cur, "k_cur"), _bf16(v_cur, "v_cur"),
-                          _bf16(o, "o"), _ptr(lse), H, frame_idx, window_back, float(scale),
-                          _rope_c(rope), _ptr(table), _stream(stream)))
+    dev = _same_device(cache, ("q", q), ("k_cur", k_cur), ("v_cur", v_cur), ("o", o), ("lse", lse),
+                       ("table", table))
+    with torch.cuda.device(dev):
+        _ok(_attention_stream(cache._h, _ptr(q), _ptr(k_cur), _ptr(v_cur), _ptr(o), _ptr(lse), H, frame_idx,
+                              window_back, float(scale), _rope_c(rope), _ptr(table), _stream(stream, dev)))
 
 
 # ----------------------------------------------------------------- hybrid
@@ -266,28 +418,69 @@ def vattn_hybrid_workspace_bytes(B, L, H, d, chunk_tokens) -> int:
     return _hyb_ws(B, L, H, d, chunk_tokens)
 
 
+def _check_hybrid(q, k, v, o, S, z):
+    _rank(q, "q", 4)
+    B, L, H, d = q.shape
+    for name, t in (("q", q), ("k", k), ("v", v), ("o", o)):
+        _expect(t, name, (B, L, H, d), torch.bfloat16)
+    _expect(S, "S", (B, H, d, d), torch.float32)
+    _expect(z, "z", (B, H, d), torch.float32)
+    return B, L, H, d
+
+
 def vattn_hybrid_chunk(q, k, v, o, S, z, chunk_tokens, scale=None, workspace=None, stream=None):
     """Hybrid chunk attention; S [B,H,d,d] and z [B,H,d] fp32 are updated in place."""
-    B, L, H, d = q.shape
+    B, L, H, d = _check_hybrid(q, k, v, o, S, z)
     if scale is None:
         scale = d ** -0.5
+    dev = _device(("q", q), ("k", k), ("v", v), ("o", o), ("S", S), ("z", z), ("workspace", workspace))
     need = vattn_hybrid_workspace_bytes(B, L, H, d, chunk_tokens)
     if workspace is None:
-        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
-    _ok(_hybrid(_bf16(q, "q"), _bf16(k, "k"), _bf16(v, "v"), _bf16(o, "o"), _ptr(S), _ptr(z), B, L,
-                H, d, chunk_tokens, float(scale), _ptr(workspace), workspace.numel() * workspace.element_size(),
-                _stream(stream)))
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
+    _min_bytes(workspace, "workspace", need)
+    with torch.cuda.device(dev):
+        _ok(_hybrid(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(S), _ptr(z), B, L, H, d, chunk_tokens,
+                    float(scale), _ptr(workspace), workspace.numel() * workspace.element_size(),
+                    _stream(stream, dev)))
+
+
+def vattn_hybrid_delta(k, v, chunk_tokens, workspace, stream=None):
+    """Per-chunk state deltas of k/v [B, L, H, d] into the workspace."""
+    _rank(k, "k", 4)
+    B, L, H, d = k.shape
+    _expect(k, "k", None, torch.bfloat16)
+    _expect(v, "v", (B, L, H, d), torch.bfloat16)
+    _min_bytes(workspace, "workspace", vattn_hybrid_workspace_bytes(B, L, H, d, chunk_tokens))
+    dev = _device(("k", k), ("v", v), ("workspace", workspace))
+    with torch.cuda.device(dev):
+        _ok(_hybrid_delta(_ptr(k), _ptr(v), B, L, H, d, chunk_tokens, _ptr(workspace),
+                          workspace.numel() * workspace.element_size(), _stream(stream, dev)))
+
+
+def vattn_hybrid_scan(S, z, L, chunk_tokens, workspace, stream=None):
+    """Exclusive scan of the workspace's deltas over chunks; S [B,H,d,d], z [B,H,d] in/out."""
+    _rank(S, "S", 4)
+    B, H, d, _ = S.shape
+    _expect(S, "S", (B, H, d, d), torch.float32)
+    _expect(z, "z", (B, H, d), torch.float32)
+    _min_bytes(workspace, "workspace", vattn_hybrid_workspace_bytes(B, L, H, d, chunk_tokens))
+    dev = _device(("S", S), ("z", z), ("workspace", workspace))
+    with torch.cuda.device(dev):
+        _ok(_hybrid_scan(_ptr(S), _ptr(z), B, L, H, d, chunk_tokens, _ptr(workspace),
+                         workspace.numel() * workspace.element_size(), _stream(stream, dev)))
 
 
 def vattn_hybrid_chunk_noalloc(q, k, v, o, S, z, chunk_tokens, scale=None, stream=None):
     """vattn_hybrid_chunk for callers that cannot allocate device memory: the
     scratch is a static array inside libvattn (HYBRID_NOALLOC_MAX_BYTES);
     nothing is allocated here or in the library."""
-    B, L, H, d = q.shape
+    B, L, H, d = _check_hybrid(q, k, v, o, S, z)
     if scale is None:
         scale = d ** -0.5
-    _ok(_hybrid_noalloc(_bf16(q, "q"), _bf16(k, "k"), _bf16(v, "v"), _bf16(o, "o"), _ptr(S), _ptr(z), B, L,
-                        H, d, chunk_tokens, float(scale), _stream(stream)))
+    dev = _device(("q", q), ("k", k), ("v", v), ("o", o), ("S", S), ("z", z))
+    with torch.cuda.device(dev):
+        _ok(_hybrid_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(S), _ptr(z), B, L, H, d, chunk_tokens,
+                            float(scale), _stream(stream, dev)))
 
 
 # ------------------------------------------------------------------ misc
@@ -301,3 +494,26 @@ def vattn_selftest_umma(variant, a, b, out, stream=None):
 
 def vattn_selftest_wait_timeout(limit_us, stream=None):
     _ok(_selftest_timeout(limit_us, _stream(stream)))
+
+
+def vattn_selftest_attention_timeout(q, k, v, o, limit_us, stream=None):
+    """The two-tile attention kernel with one withheld softmax arrival and a
+    short wait bound (include/vattn_selftest.h); q/k/v/o bf16 [1, L, H, d]."""
+    _rank(q, "q", 4)
+    B, L, H, d = q.shape
+    if B != 1:
+        raise ValueError("batch 1 only")
+    for name, t in (("q", q), ("k", k), ("v", v), ("o", o)):
+        _expect(t, name, (1, L, H, d), torch.bfloat16)
+    dev = _device(("q", q), ("k", k), ("v", v), ("o", o))
+    with torch.cuda.device(dev):
+        _ok(_selftest_attn_timeout(_ptr(q), _ptr(k), _ptr(v), _ptr(o), L, H, d, limit_us, _stream(stream, dev)))
+
+
+def vattn_selftest_ex2(variant, x, y, stream=None):
+    """y = 2^x by the kernels' exponentials (0 polynomial, 1 packed polynomial, 2 MUFU)."""
+    _expect(x, "x", None, torch.float32)
+    _expect(y, "y", tuple(x.shape), torch.float32)
+    dev = _device(("x", x), ("y", y))
+    with torch.cuda.device(dev):
+        _ok(_selftest_ex2(variant, _ptr(x), _ptr(y), x.numel(), _stream(stream, dev)))

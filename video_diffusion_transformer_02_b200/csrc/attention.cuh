@@ -1,13 +1,16 @@
-// Attention forward for sm_100a: one CTA per 128-query tile of one head.
+// Attention forward for sm_100a with the key rotation fused in: one CTA per
+// 128-query tile of one head, every K tile rotated in shared memory.
 //
 // What it computes (per query row i, visible key set A(i) given by the
 // mode): o_i = sum_{j in A(i)} softmax_j(scale * q_i . k_j) v_j, with q and
-// k optionally rotated by 3D-RoPE at their (t, h, w) positions — the
-// spatiotemporal self-attention of Wan-style DiTs and of FlashDecoder
-// ("Transformer Backbone Design" Sec. 3.2; "Streaming with Rolling KV
-// Cache" Sec. 3.3).  The HYBRID variant adds MobileWan's causal linear
-// attention across chunks: the online-softmax state of each query tile
-// starts from phi(Q) S_c and phi(Q) z_c (one joint normalisation).
+// k rotated by 3D-RoPE at their (t, h, w) positions — the spatiotemporal
+// self-attention of Wan-style DiTs and of FlashDecoder ("Transformer
+// Backbone Design" Sec. 3.2; "Streaming with Rolling KV Cache" Sec. 3.3).
+// This kernel serves calls that give RoPE but no key workspace (and
+// streaming over a raw, un-rotated ring); every other attention call runs
+// the two-tile kernel of attention_pair.cuh.  This header also holds the
+// parameter block, the mask geometry and the key-segment walk both kernels
+// share.
 //
 // Warp roles (one elected lane issues for the single-thread roles):
 //   warp 0        TMA producer: Q tile once, then K tiles (multi-stage ring)
@@ -18,14 +21,11 @@
 //                 columns 0-63 of every key tile, warpgroup 1 columns 64-127
 //                 (row max exchanged in shared memory each tile, row sums
 //                 combined at the end); P (bf16) into TMEM, O rescale,
-//                 epilogue.  Warpgroup 0 also rotates the Q tile (RoPE Q
-//                 mode) or computes phi(Q) (HYBRID); warpgroup 1 splits the
-//                 chunk state S_c into bf16 hi/lo operand tiles (HYBRID).
-//   warps 12..15  (fully fused RoPE only) RoPE of the Q tile and of every K
-//                 tile in shared memory
+//                 epilogue.
+//   warps 12..15  RoPE of the Q tile and of every K tile in shared memory
 //
 // TMEM columns (512 allocated): S double buffer [0,128) and [128,256) fp32,
-// O [256, 256+D) fp32, P [384, 448) bf16 pairs (also phi(Q) for HYBRID).
+// O [256, 256+D) fp32, P [384, 448) bf16 pairs.
 // S = Q K^T is an SS MMA (both operands K-major, 128B swizzle);
 // O += P V is a TS MMA (P from TMEM, V MN-major in shared memory).
 #pragma once
@@ -54,18 +54,6 @@ template <int D>
 struct PolyMask {
   static constexpr uint32_t value = D == 64 ? 0x88u : 0x00u;
 };
-// Packed fp32x2 arithmetic for the scale-and-subtract and the row sums.
-#define VATTN_PACKED_FP32 1
-// Poll back-off (ns) of the waits of the TMA producers and of the MMA thread.
-#ifndef VATTN_SLEEP_PROD
-#define VATTN_SLEEP_PROD 0
-#endif
-#ifndef VATTN_SLEEP_MMA
-#define VATTN_SLEEP_MMA 0
-#endif
-#ifndef VATTN_SLEEP_SOFT
-#define VATTN_SLEEP_SOFT 0
-#endif
 
 enum Mode : int { kFull = 0, kChunkCausal = 1, kSliding = 2 };
 
@@ -79,6 +67,24 @@ struct KeySegment {
   int frame;    // absolute frame index (RoPE t of every key in it)
   int tile0;    // number of key tiles in earlier segments
 };
+
+// The frame a streaming step appends, copied by the step's first CTAs
+// (raw K and V into the ring slot, K rotated at its frame into the rotated
+// ring) while the attention CTAs of the same launch run.
+struct AppendWork {
+  const uint4* k;           // frame K, V: bf16 [B][F][Hkv][D]
+  const uint4* v;
+  uint4* kr;                // raw ring slot
+  uint4* vr;
+  uint4* krot;              // rotated ring slot (nullable: no rotation)
+  int32_t* ids;             // frame id table: ids[slot] = frame
+  int slot, frame;
+  long long rows;           // B * F
+  int F;                    // tokens per stream frame
+  int t0;                   // RoPE t of the frame's first token
+};
+
+constexpr int kMaxSplit = 16;   // key splits per query-tile pair
 
 struct Params {
   __nv_bfloat16* o;
@@ -96,22 +102,43 @@ struct Params {
   // RoPE
   const float2* rope_tab;   // [max_pos][D/2] (cos, sin)
   int rope_Hg, rope_Wg, rope_pt, rope_ph, rope_maxpos;
-  // HYBRID: per-chunk exclusive state prefix
+  // hybrid chunk attention: per-chunk exclusive state prefix
   const float* hyb_S;       // [C][B][H][D][D]
   const float* hyb_z;       // [C][B][H][D]
+  // self-test knobs (zero in every attention call): a bound on each wait
+  // other than the default, and withholding one softmax arrival so that a
+  // wait of the MMA issuer runs out
+  uint64_t wait_limit_ns;
+  int test_withhold;
+  // two-tile kernel only: a 1-D grid over (append CTAs, pairs, heads,
+  // batch, split) instead of (pairs, heads, batch)
+  int linear_grid;
+  int n_pairs;              // query-tile pairs per (batch, head)
+  // key split (segment mode): split s walks key tiles
+  // [s * split_tiles, (s + 1) * split_tiles); with n_split > 1 every CTA
+  // writes its partial result and the last CTA of a pair merges them
+  int n_split;
+  int split_tiles;
+  float* part_o;            // [n_split][B][H][Lq][D] fp32: the split's o (normalised by its own l)
+  float* part_lse;          // [n_split][B][H][Lq] fp32: m + log2 l of the split (log2 domain)
+  uint32_t* pair_count;     // [B][H][n_pairs] arrivals; the merging CTA puts it back to 0
+  // streaming step: CTAs [0, n_append) of the linear grid copy the frame
+  int n_append;
+  AppendWork app;
+  uint32_t* step_sync;      // [0] append shares done, [1] CTAs exited; back to 0 at the last exit
+  int wait_tile;            // key tiles >= this read keys the append CTAs write (-1: none)
+  int total_ctas;
 };
 
-template <int D, bool HYBRID>
+template <int D>
 struct Cfg {
   static constexpr int kTileBytes = kTileM * D * 2;  // one 128 x D bf16 tile
   static constexpr int kBlocks = D / 64;             // 64-column swizzle blocks per tile
-  static constexpr int kStages = (D == 128) ? (HYBRID ? 2 : 3) : 4;
+  static constexpr int kStages = (D == 128) ? 3 : 4;
   static constexpr int kOffQ = 0;
   static constexpr int kOffK = kOffQ + kTileBytes;
   static constexpr int kOffV = kOffK + kStages * kTileBytes;
-  static constexpr int kOffShi = kOffV + kStages * kTileBytes;
-  static constexpr int kOffSlo = kOffShi + (HYBRID ? D * D * 2 : 0);
-  static constexpr int kOffBar = kOffSlo + (HYBRID ? D * D * 2 : 0);
+  static constexpr int kOffBar = kOffV + kStages * kTileBytes;
   static constexpr int kNumBars = 2 + 5 * kStages + 4 + 2 + 2 + 1;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
   static constexpr int kOffXchg = kOffMisc + 64;   // row max exchange [2 parities][2 wg][128] fp32
@@ -251,21 +278,18 @@ __device__ __forceinline__ void rope_row_inplace(uint8_t* tile, uint32_t r, Rope
   }
 }
 
-// RoPE modes: 0 none; 1 Q rotated here (softmax warpgroup, once per CTA),
-// K already rotated by the caller path; 2 Q and every K tile rotated here
-// (aux warpgroup).
+// RoPE modes: 0 none; 1 Q rotated in the kernel (once per CTA), K already
+// rotated by the caller path; 2 Q and every K tile rotated in the kernel.
 constexpr int kRopeNone = 0, kRopeQ = 1, kRopeQK = 2;
 
-__host__ __device__ constexpr int attn_threads(int rope, bool hybrid) {
-  return rope == kRopeQK ? 512 : 384;
-}
+constexpr int kFusedThreads = 512;
 
-template <int D, int ROPE, bool HYBRID>
-__global__ void __launch_bounds__(attn_threads(ROPE, HYBRID), 1)
+template <int D>
+__global__ void __launch_bounds__(kFusedThreads, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmK2,
                     const __grid_constant__ CUtensorMap tmV2, const Params p) {
-  using C = Cfg<D, HYBRID>;
+  using C = Cfg<D>;
   constexpr int NS = C::kStages;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = smem_raw;
@@ -275,7 +299,6 @@ __global__ void __launch_bounds__(attn_threads(ROPE, HYBRID), 1)
     return;
   }
   const uint32_t sQ = sbase + C::kOffQ, sK = sbase + C::kOffK, sV = sbase + C::kOffV;
-  const uint32_t sShi = sbase + C::kOffShi, sSlo = sbase + C::kOffSlo;
   const uint32_t bar0 = sbase + C::kOffBar;
   // barrier map
   const uint32_t bQFull = bar0, bQReady = bar0 + 8;
@@ -288,7 +311,7 @@ __global__ void __launch_bounds__(attn_threads(ROPE, HYBRID), 1)
   auto bSFull = [&](int b) { return bx + 8 * b; };
   auto bSFree = [&](int b) { return bx + 16 + 8 * b; };
   const uint32_t bPFull = bx + 32, bPvDone = bx + 40;
-  const uint32_t bPhiReady = bx + 48, bSReady = bx + 56, bFinal = bx + 64;
+  const uint32_t bFinal = bx + 48;
   uint32_t* misc = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
   volatile uint32_t* tmem_slot = misc;
   volatile uint32_t* abort_flag = misc + 1;
@@ -318,8 +341,6 @@ __global__ void __launch_bounds__(attn_threads(ROPE, HYBRID), 1)
     }
     mbar_init(bPFull, 8);
     mbar_init(bPvDone, 1);
-    mbar_init(bPhiReady, 4);
-    mbar_init(bSReady, 4);
     mbar_init(bFinal, 1);
     *abort_flag = 0;
     fence_barrier_init();
@@ -348,7 +369,7 @@ __global__ void __launch_bounds__(attn_threads(ROPE, HYBRID), 1)
       int j = 0;
       for (; j < nk; ++j) {
         const int s = j % NS;
-        if (j >= NS && !mbar_wait(bKEmpty(s), ((j / NS) - 1) & 1, ab, kStatusTimeoutProducer, VATTN_SLEEP_PROD)) break;
+        if (j >= NS && !mbar_wait(bKEmpty(s), ((j / NS) - 1) & 1, ab, kStatusTimeoutProducer)) break;
         const KeyTile kt = key_tile(p, g, j);
         const CUtensorMap* m = kt.kmap ? &tmK2 : &tmK;
         mbar_arrive_expect_tx(bKFull(s), C::kTileBytes);
@@ -359,13 +380,9 @@ __global__ void __launch_bounds__(attn_threads(ROPE, HYBRID), 1)
       }
       // drain: wait until every load issued so far has landed
       for (int i = max(0, j - NS); i < j; ++i) {
-        const uint64_t t0 = global_timer_ns();
-        while (!mbar_try_wait(bKFull(i % NS), (i / NS) & 1) && global_timer_ns() - t0 < kWaitLimitNs) {
-        }
+        mbar_drain(bKFull(i % NS), (i / NS) & 1, ab.limit_ns);
       }
-      const uint64_t t0 = global_timer_ns();
-      while (!mbar_try_wait(bQFull, 0) && global_timer_ns() - t0 < kWaitLimitNs) {
-      }
+      mbar_drain(bQFull, 0, ab.limit_ns);
     }
   } else if (warp == 2) {
     // ----------------------------------------------------- producer: V
@@ -373,7 +390,7 @@ __global__ void __launch_bounds__(attn_threads(ROPE, HYBRID), 1)
       int j = 0;
       for (; j < nk; ++j) {
         const int s = j % NS;
-        if (j >= NS && !mbar_wait(bVEmpty(s), ((j / NS) - 1) & 1, ab, kStatusTimeoutProducer, VATTN_SLEEP_PROD)) break;
+        if (j >= NS && !mbar_wait(bVEmpty(s), ((j / NS) - 1) & 1, ab, kStatusTimeoutProducer)) break;
         const KeyTile kt = key_tile(p, g, j);
         const CUtensorMap* m = kt.vmap ? &tmV2 : &tmV;
         mbar_arrive_expect_tx(bVFull(s), C::kTileBytes);
@@ -383,9 +400,7 @@ __global__ void __launch_bounds__(attn_threads(ROPE, HYBRID), 1)
                       kt.vc3 + b);
       }
       for (int i = max(0, j - NS); i < j; ++i) {
-        const uint64_t t0 = global_timer_ns();
-        while (!mbar_try_wait(bVFull(i % NS), (i / NS) & 1) && global_timer_ns() - t0 < kWaitLimitNs) {
-        }
+        mbar_drain(bVFull(i % NS), (i / NS) & 1, ab.limit_ns);
       }
     }
   } else if (warp == 1) {
@@ -394,33 +409,18 @@ __global__ void __launch_bounds__(attn_threads(ROPE, HYBRID), 1)
       constexpr uint32_t idQK = idesc_bf16_f32(kTileM, kTileN, false, false);
       constexpr uint32_t idPV = idesc_bf16_f32(kTileM, D, false, true);
       const uint32_t tO = tmem + kColO, tP = tmem + kColP;
-      bool ok = true;
-      if constexpr (HYBRID) {
-        ok = mbar_wait(bPhiReady, 0, ab, kStatusTimeoutMma) && mbar_wait(bSReady, 0, ab, kStatusTimeoutMma);
-        if (ok) {
-          tc_fence_after();
-          // O = phi(Q) S_hi + phi(Q) S_lo   (B operands MN-major, K = key features)
-#pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk)
-            umma_ts(tO, tP + kk * 8, sdesc_sw128(sShi + kk * 2048, D * 128, 1024), idPV, kk > 0);
-#pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk)
-            umma_ts(tO, tP + kk * 8, sdesc_sw128(sSlo + kk * 2048, D * 128, 1024), idPV, 1);
-          umma_commit(bPvDone);
-        }
-      }
-      if (ok) ok = mbar_wait(ROPE != kRopeNone ? bQReady : bQFull, 0, ab, kStatusTimeoutMma);
+      bool ok = mbar_wait(bQReady, 0, ab, kStatusTimeoutMma);
       tc_fence_after();
       auto issue_pv = [&](int i) -> bool {
-        if (!mbar_wait(bPFull, i & 1, ab, kStatusTimeoutMma, VATTN_SLEEP_MMA)) return false;
+        if (!mbar_wait(bPFull, i & 1, ab, kStatusTimeoutMma)) return false;
         const int s = i % NS;
-        if (!mbar_wait(bVFull(s), (i / NS) & 1, ab, kStatusTimeoutMma, VATTN_SLEEP_MMA)) return false;
+        if (!mbar_wait(bVFull(s), (i / NS) & 1, ab, kStatusTimeoutMma)) return false;
         tc_fence_after();
         const uint64_t dVs = sdesc_sw128(sV + s * C::kTileBytes, kTileM * 128, 1024);
 #pragma unroll
         for (int kk = 0; kk < kTileN / 16; ++kk)
           umma_ts(tO, tP + kk * 8, dVs + static_cast<uint64_t>(kk * (2048 >> 4)), idPV,
-                  (HYBRID || i > 0 || kk > 0) ? 1u : 0u);
+                  (i > 0 || kk > 0) ? 1u : 0u);
         umma_commit(bPvDone);
         umma_commit(bVEmpty(s));
         return true;
@@ -435,10 +435,8 @@ __global__ void __launch_bounds__(attn_threads(ROPE, HYBRID), 1)
       // signalled right after that tile's row max, long before its P.
       auto issue_qk = [&](int t) -> bool {
         const int s = t % NS, buf = t & 1;
-        if (!mbar_wait(ROPE == kRopeQK ? bKReady(s) : bKFull(s), (t / NS) & 1, ab, kStatusTimeoutMma,
-                       VATTN_SLEEP_MMA))
-          return false;
-        if (t >= 2 && !mbar_wait(bSFree(buf), ((t - 2) >> 1) & 1, ab, kStatusTimeoutMma, VATTN_SLEEP_MMA))
+        if (!mbar_wait(bKReady(s), (t / NS) & 1, ab, kStatusTimeoutMma)) return false;
+        if (t >= 2 && !mbar_wait(bSFree(buf), ((t - 2) >> 1) & 1, ab, kStatusTimeoutMma))
           return false;
         tc_fence_after();
         const uint64_t dKs = dK + static_cast<uint64_t>((s * C::kTileBytes) >> 4);
@@ -466,9 +464,7 @@ __global__ void __launch_bounds__(attn_threads(ROPE, HYBRID), 1)
       }
       // all issued MMAs complete before teardown
       umma_commit(bFinal);
-      const uint64_t t0 = global_timer_ns();
-      while (!mbar_try_wait(bFinal, 0) && global_timer_ns() - t0 < kWaitLimitNs) {
-      }
+      mbar_drain(bFinal, 0, ab.limit_ns);
     }
   } else if (warp >= 4 && warp < 12) {
     // ---------------------------------------------------------- softmax
@@ -489,82 +485,6 @@ __global__ void __launch_bounds__(attn_threads(ROPE, HYBRID), 1)
     const float sl2 = p.scale_log2;
     bool ok = true;
     int pv_phase = 0;   // completions of bPvDone observed so far
-    if constexpr (ROPE == kRopeQ) {
-      if (wg == 0) {
-        // rotate this thread's query row of the Q tile in place, once
-        ok = mbar_wait(bQFull, 0, ab, kStatusTimeoutSoftmax);
-        const int Fr = p.rope_Hg * p.rope_Wg;
-        RopePos pos{0, 0, 0};
-        if (row_valid) {
-          const int in = qn % Fr;
-          pos = RopePos{p.qoff + qn / Fr, in / p.rope_Wg, in % p.rope_Wg};
-        }
-        rope_row_inplace<D>(smem + C::kOffQ, r, pos, p);
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(bQReady);
-      }
-    }
-    if constexpr (HYBRID) {
-      if (wg == 0) {
-        // phi(q_r) -> TMEM P columns (bf16); D_lin = phi(q_r) . z_c in fp32
-        ok = mbar_wait(bQFull, 0, ab, kStatusTimeoutSoftmax);
-        const int c = g.q0 / p.q_seg_len;
-        const float* zc = p.hyb_z + ((static_cast<size_t>(c) * p.B + b) * p.H + h) * D;
-        float dl = 0.f;
-#pragma unroll
-        for (int half = 0; half < D / 64; ++half) {
-          uint32_t pk[32];
-#pragma unroll
-          for (int c8 = 0; c8 < 8; ++c8) {
-            const uint4 v = lds128(sQ + half * (kTileM * 128) + sw128_offset(r, c8));
-            const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const int ch = half * 64 + c8 * 8 + 2 * e;
-              float x0 = bf16lo_to_f32(w4[e]), x1 = bf16hi_to_f32(w4[e]);
-              x0 = x0 > 0.f ? x0 + 1.f : __expf(x0);
-              x1 = x1 > 0.f ? x1 + 1.f : __expf(x1);
-              dl = fmaf(x0, __ldg(zc + ch), dl);
-              dl = fmaf(x1, __ldg(zc + ch + 1), dl);
-              pk[c8 * 4 + e] = pack_bf16x2(x0, x1);
-            }
-          }
-          tmem_st32(trow + kColP + half * 32, pk);
-        }
-        tmem_st_wait();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(bPhiReady);
-        l_run = dl;
-      } else {
-        // S_c (fp32 [D][D], row a = key feature) -> bf16 hi + lo, MN-major
-        // 128B-swizzled B operand tiles (64-column blocks of D rows).
-        const int c = g.q0 / p.q_seg_len;
-        const float* src = p.hyb_S + (((static_cast<size_t>(c) * p.B + b) * p.H + h) * D + r) * D;
-        if (r < D) {
-#pragma unroll 2
-          for (int c8 = 0; c8 < D / 8; ++c8) {
-            const float4 a0 = __ldg(reinterpret_cast<const float4*>(src + c8 * 8));
-            const float4 a1 = __ldg(reinterpret_cast<const float4*>(src + c8 * 8 + 4));
-            const float x[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
-            uint32_t hi4[4], lo4[4];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              hi4[e] = pack_bf16x2(x[2 * e], x[2 * e + 1]);
-              lo4[e] = pack_bf16x2(x[2 * e] - bf16lo_to_f32(hi4[e]), x[2 * e + 1] - bf16hi_to_f32(hi4[e]));
-            }
-            const uint32_t off = (c8 >> 3) * (D * 128) + sw128_offset(r, c8 & 7);
-            sts128(sShi + off, make_uint4(hi4[0], hi4[1], hi4[2], hi4[3]));
-            sts128(sSlo + off, make_uint4(lo4[0], lo4[1], lo4[2], lo4[3]));
-          }
-        }
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(bSReady);
-      }
-      m_run = 0.f;            // the linear part enters with reference max 0
-    }
     const int cbase = wg * 64;    // first score column of this warpgroup
     // No early exit: after a failed wait (which only happens once the CTA has
     // aborted, when every later wait fails at once) the remaining tiles run
@@ -572,7 +492,7 @@ __global__ void __launch_bounds__(attn_threads(ROPE, HYBRID), 1)
     // meet the epilogue barrier exactly once.
     for (int j = 0; j < nk; ++j) {
       const int buf = j & 1;
-      if (!mbar_wait(bSFull(buf), (j >> 1) & 1, ab, kStatusTimeoutSoftmax, VATTN_SLEEP_SOFT)) ok = false;
+      if (!mbar_wait(bSFull(buf), (j >> 1) & 1, ab, kStatusTimeoutSoftmax)) ok = false;
       tc_fence_after();
       const uint32_t tS = trow + (buf ? kColS1 : kColS0) + cbase;
       int col_lo = 0, col_hi = kTileN;
@@ -639,24 +559,14 @@ __global__ void __launch_bounds__(attn_threads(ROPE, HYBRID), 1)
           for (int c = 0; c < 32; c += 2) {
             const uint32_t u0 = hq ? bb[c] : a[c], u1 = hq ? bb[c + 1] : a[c + 1];
             float x0, x1, p0, p1;
-#if VATTN_PACKED_FP32
             ffma2(x0, x1, __uint_as_float(u0), __uint_as_float(u1), sl2, sl2, nm, nm);
-#else
-            x0 = fmaf(__uint_as_float(u0), sl2, nm);
-            x1 = fmaf(__uint_as_float(u1), sl2, nm);
-#endif
             if ((PolyMask<D>::value >> ((c >> 1) & 7)) & 1u) {
               ex2_poly2(p0, p1, x0, x1);
             } else {
               p0 = ex2_approx(x0);
               p1 = ex2_approx(x1);
             }
-#if VATTN_PACKED_FP32
             fadd2(rs2[(c >> 1) & 3][0], rs2[(c >> 1) & 3][1], p0, p1);
-#else
-            rs2[(c >> 1) & 3][0] += p0;
-            rs2[(c >> 1) & 3][1] += p1;
-#endif
             pk[hq * 16 + c / 2] = pack_bf16x2(p0, p1);
           }
         }
@@ -679,15 +589,14 @@ __global__ void __launch_bounds__(attn_threads(ROPE, HYBRID), 1)
       }
       const float rs = ((rs2[0][0] + rs2[0][1]) + (rs2[1][0] + rs2[1][1])) +
                        ((rs2[2][0] + rs2[2][1]) + (rs2[3][0] + rs2[3][1]));
-      // the previous P V (or the hybrid linear init) reads the P columns and
-      // accumulates into O: it must be complete before either is touched
-      const int need = j + (HYBRID ? 1 : 0);   // bPvDone completions required
-      if (pv_phase < need) {
-        if (!mbar_wait(bPvDone, (need - 1) & 1, ab, kStatusTimeoutSoftmax, VATTN_SLEEP_SOFT)) ok = false;
-        pv_phase = need;
+      // the previous P V reads the P columns and accumulates into O: it must
+      // be complete before either is touched
+      if (pv_phase < j) {
+        if (!mbar_wait(bPvDone, (j - 1) & 1, ab, kStatusTimeoutSoftmax)) ok = false;
+        pv_phase = j;
         tc_fence_after();
       }
-      const bool o_valid = HYBRID || j > 0;
+      const bool o_valid = j > 0;
       if (__any_sync(0xffffffffu, resc && o_valid)) {
         const float f = (resc && o_valid) ? factor : 1.f;
 #pragma unroll 1
@@ -709,7 +618,7 @@ __global__ void __launch_bounds__(attn_threads(ROPE, HYBRID), 1)
     }
     // epilogue: O / l -> bf16 (each warpgroup writes its half of the
     // columns), lse from warpgroup 0
-    const int need = nk + (HYBRID ? 1 : 0);
+    const int need = nk;
     if (ok && need > 0 && pv_phase < need) {
       ok = mbar_wait(bPvDone, (need - 1) & 1, ab, kStatusTimeoutSoftmax);
       tc_fence_after();
@@ -753,7 +662,7 @@ __global__ void __launch_bounds__(attn_threads(ROPE, HYBRID), 1)
     // ------------------------------------------------------ aux warpgroup
     // RoPE of the Q tile and of every K tile, in shared memory, in place.
     const int r = threadIdx.x - 384;
-    if constexpr (ROPE == kRopeQK) {
+    {
       const int Fr = p.rope_Hg * p.rope_Wg;
       bool ok = mbar_wait(bQFull, 0, ab, kStatusTimeoutAux);
       if (ok) {

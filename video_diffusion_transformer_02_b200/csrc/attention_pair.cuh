@@ -55,9 +55,10 @@ struct PairGeom {
   int q0[2], q_end[2];
   bool hasB;
   TileGeom tg;   // q0 / q_end span both tiles; kbeg, kend, n_tiles: the union
+  int t0;        // segment mode: the CTA's first key tile (key split); 0 otherwise
 };
 
-__device__ __forceinline__ PairGeom pair_geom(const Params& p, int pr) {
+__device__ __forceinline__ PairGeom pair_geom(const Params& p, int pr, int split) {
   PairGeom g;
   const int pps = (p.q_tiles_per_seg + 1) / 2;
   const int seg = pr / pps;
@@ -71,6 +72,7 @@ __device__ __forceinline__ PairGeom pair_geom(const Params& p, int pr) {
   g.hasB = g.q0[1] < g.q_end[1];
   g.tg.q0 = g.q0[0];
   g.tg.q_end = g.hasB ? g.q_end[1] : g.q_end[0];
+  g.t0 = 0;
   if (p.n_kseg == 0) {
     int lo0, hi0, lo1, hi1;
     key_range(p, g.tg.q0, lo0, hi0);
@@ -81,9 +83,86 @@ __device__ __forceinline__ PairGeom pair_geom(const Params& p, int pr) {
   } else {
     g.tg.kbeg = g.tg.kend = 0;
     const KeySegment& last = p.kseg[p.n_kseg - 1];
-    g.tg.n_tiles = last.tile0 + (last.n_tok + kTileN - 1) / kTileN;
+    const int total = last.tile0 + (last.n_tok + kTileN - 1) / kTileN;
+    const int per = p.n_split > 1 ? p.split_tiles : total;
+    g.t0 = min(total, split * per);
+    g.tg.n_tiles = min(total, g.t0 + per) - g.t0;
   }
   return g;
+}
+
+// A streaming step's append share: CTA `part` of the n_append leading CTAs
+// copies its range of the frame's 16-byte chunks (raw K and V into the ring
+// slot, K rotated at its (t, h, w) into the rotated ring), then counts
+// itself done with a release; attention CTAs of the same launch wait for
+// all shares before loading the rotated current frame.
+template <int D>
+__device__ __forceinline__ void append_share(const Params& p, int part) {
+  const AppendWork& a = p.app;
+  constexpr int D8 = D / 8;   // 16-byte chunks per head vector
+  const long long cpr = static_cast<long long>(p.Hkv) * D8;
+  const long long total = a.rows * cpr;
+  const long long per = (total + p.n_append - 1) / p.n_append;
+  const long long c0 = static_cast<long long>(part) * per;
+  const long long c1 = min(total, c0 + per);
+  const int Fr = p.rope_Hg * p.rope_Wg;
+  const int pt = p.rope_pt, pth = p.rope_pt + p.rope_ph;
+  constexpr int U = 4;   // chunks per thread and step: all loads before the stores
+  for (long long base = c0 + threadIdx.x; base < c1; base += static_cast<long long>(blockDim.x) * U) {
+    uint4 kv[U], vv[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const long long i = base + static_cast<long long>(u) * blockDim.x;
+      if (i < c1) {
+        kv[u] = __ldg(a.k + i);
+        vv[u] = __ldg(a.v + i);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const long long i = base + static_cast<long long>(u) * blockDim.x;
+      if (i >= c1) continue;
+      a.kr[i] = kv[u];
+      a.vr[i] = vv[u];
+      if (a.krot) {
+        const int n = static_cast<int>((i / cpr) % a.F);   // token of the frame
+        const int c16 = static_cast<int>(i % D8);          // chunk of the head vector
+        const int in = n % Fr;
+        const int pos[3] = {a.t0 + n / Fr, in / p.rope_Wg, in % p.rope_Wg};
+        uint32_t w4[4] = {kv[u].x, kv[u].y, kv[u].z, kv[u].w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int j = c16 * 4 + e;
+          const int ax = j < pt ? 0 : (j < pth ? 1 : 2);
+          const float2 cs = __ldg(p.rope_tab + pos[ax] * (D / 2) + j);
+          const float x0 = bf16lo_to_f32(w4[e]), x1 = bf16hi_to_f32(w4[e]);
+          w4[e] = pack_bf16x2(x0 * cs.x - x1 * cs.y, x0 * cs.y + x1 * cs.x);
+        }
+        a.krot[i] = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+      }
+    }
+  }
+  if (part == 0 && threadIdx.x == 0) a.ids[a.slot] = a.frame;
+  // every thread's stores visible to the async proxy (TMA) and at gpu scope
+  // before the CTA counts itself done
+  fence_proxy_async_global();
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) atomicAdd(p.step_sync, 1u);
+}
+
+// Last act of every CTA of a streaming step: count the exit; the last CTA
+// puts both counters back to zero for the next launch.
+__device__ __forceinline__ void step_exit(const Params& p) {
+  if (threadIdx.x == 0) {
+    __threadfence();
+    const uint32_t old = atomicAdd(p.step_sync + 1, 1u);
+    if (old == static_cast<uint32_t>(p.total_ctas) - 1u) {
+      p.step_sync[0] = 0u;
+      p.step_sync[1] = 0u;
+      __threadfence();
+    }
+  }
 }
 
 // Keep the 32 registers of r after every earlier volatile statement (the
@@ -106,9 +185,33 @@ __global__ void __launch_bounds__(kPairThreads, 1)
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = smem_raw;
   const uint32_t sbase = smem_addr(smem);
+  const bool stepping = p.linear_grid && p.step_sync;
   if (sbase & 1023u) {   // 128B-swizzled operand tiles need 1024-byte alignment
     if (threadIdx.x == 0 && p.status) atomicCAS(p.status, 0u, kStatusSmemAlign);
+    if (stepping) step_exit(p);
     return;
+  }
+  // which work this CTA does: (pair, head, batch) of a 3-D grid, or an
+  // append share / (pair, head, batch, split) of a streaming step's 1-D grid
+  int pr, h, b, split = 0;
+  if (p.linear_grid) {
+    int idx = static_cast<int>(blockIdx.x);
+    if (idx < p.n_append) {
+      append_share<D>(p, idx);
+      step_exit(p);
+      return;
+    }
+    idx -= p.n_append;
+    pr = idx % p.n_pairs;
+    idx /= p.n_pairs;
+    h = idx % p.H;
+    idx /= p.H;
+    b = idx % p.B;
+    split = idx / p.B;
+  } else {
+    h = blockIdx.y;
+    b = blockIdx.z;
+    pr = p.reverse_q ? static_cast<int>(gridDim.x - 1 - blockIdx.x) : static_cast<int>(blockIdx.x);
   }
   const uint32_t sQ = sbase + C::kOffQ, sK = sbase + C::kOffK, sV = sbase + C::kOffV;
   const uint32_t bar0 = sbase + C::kOffBar;
@@ -131,14 +234,15 @@ __global__ void __launch_bounds__(kPairThreads, 1)
   uint32_t* misc = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
   volatile uint32_t* tmem_slot = misc;
   volatile uint32_t* abort_flag = misc + 1;
-  Abort ab{abort_flag, p.status};
+  Abort ab{abort_flag, p.status, p.wait_limit_ns ? p.wait_limit_ns : kWaitLimitNs};
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int h = blockIdx.y, b = blockIdx.z;
   const int kvh = h / (p.H / p.Hkv);
-  const int pr = p.reverse_q ? static_cast<int>(gridDim.x - 1 - blockIdx.x) : static_cast<int>(blockIdx.x);
-  const PairGeom g = pair_geom(p, pr);
-  if (g.q0[0] >= g.q_end[0]) return;   // pair past the end of a short last segment
+  const PairGeom g = pair_geom(p, pr, split);
+  if (g.q0[0] >= g.q_end[0]) {   // pair past the end of a short last segment
+    if (stepping) step_exit(p);
+    return;
+  }
   const int nk = g.tg.n_tiles;          // 128-key stages
   const int ns = 2 * nk;                // 64-key score sub-tiles
   const bool hasB = g.hasB;
@@ -196,10 +300,17 @@ __global__ void __launch_bounds__(kPairThreads, 1)
                       x ? g.q0[1] : g.q0[0], b);
       }
       int j = 0;
+      bool waited = p.wait_tile < 0 || !stepping;
       for (; j < nk; ++j) {
         const int s = j % NS;
         if (j >= NS && !mbar_wait(bKEmpty(s), ((j / NS) - 1) & 1, ab, kStatusTimeoutProducer)) break;
-        const KeyTile kt = key_tile(p, g.tg, j);
+        if (!waited && g.t0 + j >= p.wait_tile) {
+          // this tile's keys are written by the step's append CTAs
+          if (!wait_counter(p.step_sync, static_cast<uint32_t>(p.n_append), ab, kStatusTimeoutStep)) break;
+          fence_proxy_async_global();
+          waited = true;
+        }
+        const KeyTile kt = key_tile(p, g.tg, g.t0 + j);
         const CUtensorMap* m = kt.kmap ? &tmK2 : &tmK;
         mbar_arrive_expect_tx(bKFull(s), C::kTileBytes);
 #pragma unroll
@@ -209,14 +320,10 @@ __global__ void __launch_bounds__(kPairThreads, 1)
       }
       // drain: every load issued so far has landed before the CTA exits
       for (int i = max(0, j - NS); i < j; ++i) {
-        const uint64_t t0 = global_timer_ns();
-        while (!mbar_try_wait(bKFull(i % NS), (i / NS) & 1) && global_timer_ns() - t0 < kWaitLimitNs) {
-        }
+        mbar_drain(bKFull(i % NS), (i / NS) & 1, ab.limit_ns);
       }
       for (int x = 0; x < (hasB ? 2 : 1); ++x) {
-        const uint64_t t0 = global_timer_ns();
-        while (!mbar_try_wait(bQFull(x), 0) && global_timer_ns() - t0 < kWaitLimitNs) {
-        }
+        mbar_drain(bQFull(x), 0, ab.limit_ns);
       }
     }
   } else if (warp == 2) {
@@ -226,7 +333,7 @@ __global__ void __launch_bounds__(kPairThreads, 1)
       for (; j < nk; ++j) {
         const int s = j % NS;
         if (j >= NS && !mbar_wait(bVEmpty(s), ((j / NS) - 1) & 1, ab, kStatusTimeoutProducer)) break;
-        const KeyTile kt = key_tile(p, g.tg, j);
+        const KeyTile kt = key_tile(p, g.tg, g.t0 + j);
         const CUtensorMap* m = kt.vmap ? &tmV2 : &tmV;
         mbar_arrive_expect_tx(bVFull(s), C::kTileBytes);
 #pragma unroll
@@ -235,9 +342,7 @@ __global__ void __launch_bounds__(kPairThreads, 1)
                       kt.vc3 + b);
       }
       for (int i = max(0, j - NS); i < j; ++i) {
-        const uint64_t t0 = global_timer_ns();
-        while (!mbar_try_wait(bVFull(i % NS), (i / NS) & 1) && global_timer_ns() - t0 < kWaitLimitNs) {
-        }
+        mbar_drain(bVFull(i % NS), (i / NS) & 1, ab.limit_ns);
       }
     }
   } else if (warp == 1 || warp == 3) {
@@ -339,9 +444,7 @@ __global__ void __launch_bounds__(kPairThreads, 1)
       }
       // all issued MMAs complete before teardown
       umma_commit(bFinal(x));
-      const uint64_t t0 = global_timer_ns();
-      while (!mbar_try_wait(bFinal(x), 0) && global_timer_ns() - t0 < kWaitLimitNs) {
-      }
+      mbar_drain(bFinal(x), 0, ab.limit_ns);
     }
   } else if (warp >= 4 && warp < 12) {
     // ---------------------------------------------------------- softmax
@@ -387,7 +490,7 @@ __global__ void __launch_bounds__(kPairThreads, 1)
           col_lo = lo - k0;
           col_hi = hi - k0;
         } else {
-          col_hi = key_tile(p, g.tg, u >> 1).valid - bb * kSub;
+          col_hi = key_tile(p, g.tg, g.t0 + (u >> 1)).valid - bb * kSub;
         }
         const bool masked = col_lo > 0 || col_hi < kSub;
         uint32_t s0[32], s1[32];
@@ -481,7 +584,10 @@ __global__ void __launch_bounds__(kPairThreads, 1)
         tmem_st_wait();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(bPFull(x, bb));
+        // (self-test only: the first warp of tile A withholds its arrival for
+        // sub-tile 1, so tile A's issuer waits until its bound runs out)
+        const bool withhold = p.test_withhold && x == 0 && warp == 4 && u == 1;
+        if (lane == 0 && !withhold) mbar_arrive(bPFull(x, bb));
         l_run = l_run * factor + rs;
       }
       float dl = 0.f;   // hybrid: phi(q_r) . z_c
@@ -510,9 +616,10 @@ __global__ void __launch_bounds__(kPairThreads, 1)
               float x0 = bf16lo_to_f32(w4[e]), x1 = bf16hi_to_f32(w4[e]);
               x0 = x0 > 0.f ? x0 + 1.f : __expf(x0);
               x1 = x1 > 0.f ? x1 + 1.f : __expf(x1);
-              dl = fmaf(x0, zz[2 * e], dl);
-              dl = fmaf(x1, zz[2 * e + 1], dl);
               w4[e] = pack_bf16x2(x0, x1);
+              // the denominator takes the same bf16 values the read-out MMA multiplies
+              dl = fmaf(bf16lo_to_f32(w4[e]), zz[2 * e], dl);
+              dl = fmaf(bf16hi_to_f32(w4[e]), zz[2 * e + 1], dl);
             }
             sts128(addr, make_uint4(w4[0], w4[1], w4[2], w4[3]));
           }

@@ -109,9 +109,7 @@ __global__ void __launch_bounds__(kDeltaThreads, 1)
         }
       }
       for (int i = max(0, t - NS); i < t; ++i) {
-        const uint64_t t0 = global_timer_ns();
-        while (!mbar_try_wait(bFull(i % NS), (i / NS) & 1) && global_timer_ns() - t0 < kWaitLimitNs) {
-        }
+        mbar_drain(bFull(i % NS), (i / NS) & 1, ab.limit_ns);
       }
     }
   } else if (warp == 1) {
@@ -131,9 +129,7 @@ __global__ void __launch_bounds__(kDeltaThreads, 1)
         umma_commit(bEmpty(s));
       }
       umma_commit(bDone);
-      const uint64_t t0 = global_timer_ns();
-      while (!mbar_try_wait(bDone, 0) && global_timer_ns() - t0 < kWaitLimitNs) {
-      }
+      mbar_drain(bDone, 0, ab.limit_ns);
     }
   } else if (warp >= 4) {
     const int tid = threadIdx.x - 128;

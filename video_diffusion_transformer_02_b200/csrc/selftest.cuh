@@ -124,5 +124,22 @@ __global__ void __launch_bounds__(32, 1) wait_timeout_kernel(uint64_t limit_ns, 
   mbar_wait_limit(b, 0, ab, kStatusTimeoutAux, limit_ns);
 }
 
+// The exponentials of the softmax, element by element:
+//   variant 0: y = ex2_poly(x)       (FMA-pipe polynomial)
+//   variant 1: (y[2i], y[2i+1]) = ex2_poly2(x[2i], x[2i+1])   (packed form; n even)
+//   variant 2: y = ex2_approx(x)     (MUFU ex2.approx.ftz)
+__global__ void ex2_kernel(const float* __restrict__ x, float* __restrict__ y, int n, int variant) {
+  const int stride = gridDim.x * blockDim.x;
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < n; i += stride) {
+    if (variant == 0) {
+      y[i] = ex2_poly(x[i]);
+    } else if (variant == 1) {
+      if (2 * i + 1 < n) ex2_poly2(y[2 * i], y[2 * i + 1], x[2 * i], x[2 * i + 1]);
+    } else {
+      y[i] = ex2_approx(x[i]);
+    }
+  }
+}
+
 }  // namespace selftest
 }  // namespace vattn

@@ -21,6 +21,7 @@ enum : uint32_t {
   kStatusTimeoutSoftmax = 3,
   kStatusTimeoutAux = 4,
   kStatusSmemAlign = 5,   // dynamic shared memory not 1024-byte aligned
+  kStatusTimeoutStep = 6, // a streaming step's attention CTA waited too long for the frame's keys
 };
 // Wall-clock bound of a single wait (nanoseconds of %globaltimer).
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
@@ -68,6 +69,7 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 struct Abort {
   volatile uint32_t* flag;   // shared memory
   uint32_t* status;          // global memory (may be null)
+  uint64_t limit_ns = kWaitLimitNs;   // bound of each wait
 };
 
 __device__ __forceinline__ void raise_abort(const Abort& ab, uint32_t code) {
@@ -93,20 +95,57 @@ __device__ __forceinline__ bool mbar_wait_limit(uint32_t bar, uint32_t parity, c
 }
 
 // Wait until phase `parity` of `bar` has completed.  Returns false if the
-// CTA aborted or the wait exceeded kWaitLimitNs (then the abort is raised
-// with `code`).  sleep_ns > 0 backs off between polls (for threads whose
-// reaction time matters less than the issue slots their polling would take
-// from warps sharing the sub-partition).
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, const Abort& ab,
-                                          uint32_t code, uint32_t sleep_ns = 0) {
+// CTA aborted or the wait exceeded ab.limit_ns (then the abort is raised
+// with `code`).
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, const Abort& ab, uint32_t code) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_timer_ns();
   for (uint32_t it = 1;; ++it) {
-    if (sleep_ns) __nanosleep(sleep_ns);
     if (mbar_try_wait(bar, parity)) return true;
     if ((it & 63u) == 0u) {
       if (*ab.flag) return false;
-      if (global_timer_ns() - t0 > kWaitLimitNs) {
+      if (global_timer_ns() - t0 > ab.limit_ns) {
+        raise_abort(ab, code);
+        return false;
+      }
+    }
+  }
+}
+
+// Poll `bar` until phase `parity` completes or limit_ns passes, without
+// raising anything: the teardown drains of a CTA (loads and MMAs already in
+// flight) that must end whether or not the CTA aborted.
+__device__ __forceinline__ void mbar_drain(uint32_t bar, uint32_t parity, uint64_t limit_ns) {
+  const uint64_t t0 = global_timer_ns();
+  while (!mbar_try_wait(bar, parity) && global_timer_ns() - t0 < limit_ns) {
+  }
+}
+
+// ------------------------------------------------- cross-CTA signalling
+// Generic-proxy global writes made visible to later async-proxy (TMA) reads,
+// by this thread or (after a release/acquire pair) by another CTA.
+__device__ __forceinline__ void fence_proxy_async_global() {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+__device__ __forceinline__ uint32_t ld_acquire_gpu(const uint32_t* p) {
+  uint32_t v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+// Wait until *counter >= target (another CTA of the same launch counts up
+// with a release), bounded like mbar_wait.  Returns false on abort or when
+// ab.limit_ns passes (the abort is then raised with `code`).
+__device__ __forceinline__ bool wait_counter(const uint32_t* counter, uint32_t target, const Abort& ab,
+                                             uint32_t code) {
+  if (ld_acquire_gpu(counter) >= target) return true;
+  const uint64_t t0 = global_timer_ns();
+  for (uint32_t it = 1;; ++it) {
+    __nanosleep(64);
+    if (ld_acquire_gpu(counter) >= target) return true;
+    if ((it & 15u) == 0u) {
+      if (*ab.flag) return false;
+      if (global_timer_ns() - t0 > ab.limit_ns) {
         raise_abort(ab, code);
         return false;
       }
@@ -315,10 +354,11 @@ __device__ __forceinline__ float bf16hi_to_f32(uint32_t v) { return __uint_as_fl
 
 // 2^x on the FMA pipe (offloads the MUFU unit): Cody-Waite reduction
 // x = j + f with j = round(x) (via the 1.5*2^23 shifter), f in [-0.5, 0.5],
-// degree-3 minimax polynomial for 2^f (max relative error 7.5e-5; the
-// coefficients come from fit_exp2_poly.py), then j added to the exponent
-// field.  Arguments below -126 return a value below 2^-126 (consumers
-// treat it as zero after bf16 rounding of the probability).
+// degree-3 minimax polynomial for 2^f (max relative error 7.5e-5 for
+// x >= -125, below 7.6e-5 with fp32 evaluation; the coefficients come from
+// fit_exp2_poly.py), then j added to the exponent field.  Arguments below
+// -125 return a value in [0, 2^-124] (the softmax's probabilities there are
+// zero to every digit that counts).
 __device__ __forceinline__ float ex2_poly(float x) {
   x = fmaxf(x, -126.0f);
   const float t = x + 12582912.0f;
@@ -326,12 +366,14 @@ __device__ __forceinline__ float ex2_poly(float x) {
   float p = fmaf(5.517166853e-02f, f, 2.426111251e-01f);
   p = fmaf(p, f, 6.932609677e-01f);
   p = fmaf(p, f, 9.999280572e-01f);
-  return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
+  // t's low mantissa bits hold j (two's complement); shifted by 23 they land
+  // in the exponent field (unsigned arithmetic: the wrap is defined)
+  return __uint_as_float(__float_as_uint(p) + (__float_as_uint(t) << 23));
 }
 
 // Two lanes of ex2_poly with packed fp32x2 arithmetic: the same reduction,
-// polynomial and exponent insertion (exponent added with an integer
-// multiply-add of j * 2^23 onto the polynomial's bits).
+// polynomial and exponent insertion (j * 2^23 added onto the polynomial's
+// bits in unsigned 32-bit arithmetic).
 __device__ __forceinline__ void ex2_poly2(float& y0, float& y1, float x0, float x1) {
   x0 = fmaxf(x0, -126.0f);
   x1 = fmaxf(x1, -126.0f);
@@ -342,8 +384,8 @@ __device__ __forceinline__ void ex2_poly2(float& y0, float& y1, float x0, float 
   ffma2(p0, p1, f0, f1, 5.517166853e-02f, 5.517166853e-02f, 2.426111251e-01f, 2.426111251e-01f);
   ffma2(p0, p1, p0, p1, f0, f1, 6.932609677e-01f, 6.932609677e-01f);
   ffma2(p0, p1, p0, p1, f0, f1, 9.999280572e-01f, 9.999280572e-01f);
-  y0 = __int_as_float(__float_as_int(t0) * (1 << 23) + __float_as_int(p0));
-  y1 = __int_as_float(__float_as_int(t1) * (1 << 23) + __float_as_int(p1));
+  y0 = __uint_as_float((__float_as_uint(t0) << 23) + __float_as_uint(p0));
+  y1 = __uint_as_float((__float_as_uint(t1) << 23) + __float_as_uint(p1));
 }
 
 __device__ __forceinline__ float ex2_approx(float x) {

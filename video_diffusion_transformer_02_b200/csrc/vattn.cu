@@ -13,14 +13,9 @@
 #include "../../include/vattn.h"
 #include "attention.cuh"
 #include "attention_pair.cuh"
-
-// 1: attention with keys already rotated (or without RoPE) runs two query
-// tiles per CTA; 0: one query tile per CTA.
-#ifndef VATTN_PAIR_TILES
-#define VATTN_PAIR_TILES 1
-#endif
 #include "hybrid.cuh"
 #include "kvcache.cuh"
+#include "merge.cuh"
 #include "rope.cuh"
 #include "selftest.cuh"
 
@@ -147,25 +142,23 @@ vattn_status check_rope(const vattn_rope* r, int d) {
 
 bool supported_d(int d) { return d == 64 || d == 128; }
 
-uint64_t g_attn_smem_done[16][1];
+uint64_t g_fused_smem_done[2][1];
 
-template <int D, int ROPE, bool HYB>
-vattn_status launch_attention(const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v,
-                              const CUtensorMap& k2, const CUtensorMap& v2, const vattn::attn::Params& p,
-                              cudaStream_t s) {
-  using Cfg = vattn::attn::Cfg<D, HYB>;
-  constexpr int slot = (D == 64 ? 0 : 4) + ROPE + (HYB ? 8 : 0);
-  constexpr int threads = vattn::attn::attn_threads(ROPE, HYB);
-  auto kern = vattn::attn::attn_fwd_kernel<D, ROPE, HYB>;
-  vattn_status st = ensure_smem(kern, Cfg::kSmemBytes, g_attn_smem_done[slot]);
+// One query tile per CTA, Q and every K tile rotated in the kernel
+// (attention.cuh): grid = query tiles x heads x batch.
+template <int D>
+vattn_status launch_fused(const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v, const CUtensorMap& k2,
+                          const CUtensorMap& v2, const vattn::attn::Params& p, cudaStream_t s) {
+  using Cfg = vattn::attn::Cfg<D>;
+  auto kern = vattn::attn::attn_fwd_kernel<D>;
+  vattn_status st = ensure_smem(kern, Cfg::kSmemBytes, g_fused_smem_done[D == 64 ? 0 : 1]);
   if (st) return st;
   const dim3 grid(p.n_q_tiles, p.H, p.B);
-  kern<<<grid, threads, Cfg::kSmemBytes, s>>>(q, k, v, k2, v2, p);
+  kern<<<grid, vattn::attn::kFusedThreads, Cfg::kSmemBytes, s>>>(q, k, v, k2, v2, p);
   VATTN_CUDA(cudaGetLastError());
   return VATTN_OK;
 }
 
-#if VATTN_PAIR_TILES
 uint64_t g_pair_smem_done[5][1];
 
 // Two query tiles per CTA (attention_pair.cuh): grid = tile pairs x heads x
@@ -187,30 +180,19 @@ vattn_status launch_pair(const CUtensorMap& q, const CUtensorMap& k, const CUten
   return VATTN_OK;
 }
 
-#endif
-
 vattn_status dispatch_attention(int d, int rope_mode, const CUtensorMap& q, const CUtensorMap& k,
                                 const CUtensorMap& v, const CUtensorMap& k2, const CUtensorMap& v2,
                                 const vattn::attn::Params& p, cudaStream_t s) {
   using namespace vattn::attn;
-#if VATTN_PAIR_TILES
+  // keys rotated inside the kernel: the one-tile kernel with the RoPE warpgroup
+  if (rope_mode == kRopeQK)
+    return d == 64 ? launch_fused<64>(q, k, v, k2, v2, p, s) : launch_fused<128>(q, k, v, k2, v2, p, s);
   // keys already rotated (or no RoPE): the two-tile kernel
-  if (rope_mode != kRopeQK) {
-    if (d == 64)
-      return rope_mode == kRopeQ ? launch_pair<64, kRopeQ>(q, k, v, k2, v2, p, s)
-                                 : launch_pair<64, kRopeNone>(q, k, v, k2, v2, p, s);
-    return rope_mode == kRopeQ ? launch_pair<128, kRopeQ>(q, k, v, k2, v2, p, s)
-                               : launch_pair<128, kRopeNone>(q, k, v, k2, v2, p, s);
-  }
-#endif
-  if (d == 64) {
-    if (rope_mode == kRopeQK) return launch_attention<64, kRopeQK, false>(q, k, v, k2, v2, p, s);
-    if (rope_mode == kRopeQ) return launch_attention<64, kRopeQ, false>(q, k, v, k2, v2, p, s);
-    return launch_attention<64, kRopeNone, false>(q, k, v, k2, v2, p, s);
-  }
-  if (rope_mode == kRopeQK) return launch_attention<128, kRopeQK, false>(q, k, v, k2, v2, p, s);
-  if (rope_mode == kRopeQ) return launch_attention<128, kRopeQ, false>(q, k, v, k2, v2, p, s);
-  return launch_attention<128, kRopeNone, false>(q, k, v, k2, v2, p, s);
+  if (d == 64)
+    return rope_mode == kRopeQ ? launch_pair<64, kRopeQ>(q, k, v, k2, v2, p, s)
+                               : launch_pair<64, kRopeNone>(q, k, v, k2, v2, p, s);
+  return rope_mode == kRopeQ ? launch_pair<128, kRopeQ>(q, k, v, k2, v2, p, s)
+                             : launch_pair<128, kRopeNone>(q, k, v, k2, v2, p, s);
 }
 
 // Rotate K once into k_out (the standalone RoPE kernel on keys only).
@@ -394,11 +376,14 @@ size_t vattn_attention_workspace_bytes(int B, int Lk, int Hkv, int d, const vatt
   return static_cast<size_t>(B) * Lk * Hkv * d * 2;
 }
 
-vattn_status vattn_attention(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Lq,
-                             int Lk, int H, int Hkv, int d, float scale, vattn_mode mode, int tokens_per_frame,
-                             int chunk_frames, int window_back, int window_fwd, int q_frame_offset,
-                             int k_frame_offset, const vattn_rope* rope, const float* table,
-                             void* workspace, size_t workspace_bytes, vattn_stream stream) {
+// vattn_attention with the two self-test knobs of the parameter block (a
+// wait bound other than the default, one withheld softmax arrival).
+static vattn_status attention_impl(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                                   int Lq, int Lk, int H, int Hkv, int d, float scale, vattn_mode mode,
+                                   int tokens_per_frame, int chunk_frames, int window_back, int window_fwd,
+                                   int q_frame_offset, int k_frame_offset, const vattn_rope* rope,
+                                   const float* table, void* workspace, size_t workspace_bytes,
+                                   vattn_stream stream, uint64_t wait_limit_ns, int withhold) {
   if (!q || !k || !v || !o) return fail(VATTN_ERR_INVALID_ARG, "q, k, v, o must be non-NULL");
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o))
     return fail(VATTN_ERR_INVALID_ARG, "q, k, v, o must be 16-byte aligned");
@@ -456,6 +441,8 @@ vattn_status vattn_attention(const void* q, const void* k, const void* v, void* 
   p.n_q_tiles = p.q_tiles_per_seg;
   p.reverse_q = mode == VATTN_CHUNK_CAUSAL ? 1 : 0;
   p.n_kseg = 0;
+  p.wait_limit_ns = wait_limit_ns;
+  p.test_withhold = withhold;
   fill_rope_params(p, rope, table);
 
   CUtensorMap mq, mk, mv;
@@ -472,6 +459,16 @@ vattn_status vattn_attention(const void* q, const void* k, const void* v, void* 
   }
   return dispatch_attention(d, rope ? vattn::attn::kRopeQK : vattn::attn::kRopeNone, mq, mk, mv, mk, mv, p,
                             stream);
+}
+
+vattn_status vattn_attention(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Lq,
+                             int Lk, int H, int Hkv, int d, float scale, vattn_mode mode, int tokens_per_frame,
+                             int chunk_frames, int window_back, int window_fwd, int q_frame_offset,
+                             int k_frame_offset, const vattn_rope* rope, const float* table,
+                             void* workspace, size_t workspace_bytes, vattn_stream stream) {
+  return attention_impl(q, k, v, o, lse, B, Lq, Lk, H, Hkv, d, scale, mode, tokens_per_frame, chunk_frames,
+                        window_back, window_fwd, q_frame_offset, k_frame_offset, rope, table, workspace,
+                        workspace_bytes, stream, 0, 0);
 }
 
 // ------------------------------------------------------------- KV cache
@@ -692,22 +689,92 @@ size_t vattn_hybrid_workspace_bytes(int B, int L, int H, int d, int chunk_tokens
   return C * B * H * (static_cast<size_t>(d) * d + d) * sizeof(float);
 }
 
-vattn_status vattn_hybrid_chunk(const void* q, const void* k, const void* v, void* o, float* S, float* z, int B,
-                                int L, int H, int d, int chunk_tokens, float scale, void* workspace,
-                                size_t workspace_bytes, vattn_stream stream) {
-  if (!q || !k || !v || !o || !S || !z || !workspace) return fail(VATTN_ERR_INVALID_ARG, "NULL pointer");
-  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(S) || !aligned16(z) ||
-      !aligned16(workspace))
-    return fail(VATTN_ERR_INVALID_ARG, "pointers must be 16-byte aligned");
+}  // extern "C"
+
+namespace {
+// Shared argument checks of the hybrid calls; C = number of chunks.
+vattn_status check_hybrid(int B, int L, int H, int d, int chunk_tokens, const void* workspace,
+                          size_t workspace_bytes, int* C) {
+  if (!workspace) return fail(VATTN_ERR_INVALID_ARG, "NULL workspace");
+  if (!aligned16(workspace)) return fail(VATTN_ERR_INVALID_ARG, "workspace must be 16-byte aligned");
   if (B < 1 || L < 1 || H < 1 || chunk_tokens < 1) return fail(VATTN_ERR_INVALID_ARG, "sizes must be >= 1");
   if (B > 65535 || H > 65535) return fail(VATTN_ERR_UNSUPPORTED, "B or H above 65535");
   if (d != 128) return fail(VATTN_ERR_UNSUPPORTED, "hybrid supports head dim 128 (got %d)", d);
-  if (!std::isfinite(scale)) return fail(VATTN_ERR_INVALID_ARG, "scale not finite");
   const size_t need = vattn_hybrid_workspace_bytes(B, L, H, d, chunk_tokens);
   if (workspace_bytes < need)
     return fail(VATTN_ERR_INVALID_ARG, "workspace %zu bytes < %zu required", workspace_bytes, need);
-  const int C = (L + chunk_tokens - 1) / chunk_tokens;
-  if (C > 65535) return fail(VATTN_ERR_UNSUPPORTED, "more than 65535 chunks");
+  *C = (L + chunk_tokens - 1) / chunk_tokens;
+  if (*C > 65535) return fail(VATTN_ERR_UNSUPPORTED, "more than 65535 chunks");
+  return VATTN_OK;
+}
+
+// Launch 1 of the hybrid call: per-chunk state deltas into the workspace.
+vattn_status launch_delta(const CUtensorMap& mk, const CUtensorMap& mv, float* wsS, float* wsz, uint32_t* status,
+                          int B, int L, int H, int C, int chunk_tokens, cudaStream_t stream) {
+  static uint64_t done[1];
+  auto kern = vattn::hyb::delta_kernel<128>;
+  const int smem = vattn::hyb::DeltaCfg<128>::kSmemBytes;
+  if (vattn_status st = ensure_smem(kern, smem, done)) return st;
+  vattn::hyb::DeltaParams dp{wsS, wsz, status, B, L, H, chunk_tokens};
+  kern<<<dim3(H, C, B), vattn::hyb::kDeltaThreads, smem, stream>>>(mk, mv, dp);
+  VATTN_CUDA(cudaGetLastError());
+  return VATTN_OK;
+}
+
+// Launch 2: exclusive scan over chunks, in place, plus the state out.
+vattn_status launch_scan(float* wsS, float* wsz, float* S, float* z, int B, int H, int d, int C,
+                         cudaStream_t stream) {
+  const long long nS4 = static_cast<long long>(B) * H * d * d / 4, nz4 = static_cast<long long>(B) * H * d / 4;
+  int sms = 148, dev;
+  if (current_device(&dev) == VATTN_OK) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const long long want = (nS4 + nz4 + 255) / 256;
+  const int blocks = static_cast<int>(want < sms * 4LL ? want : sms * 4LL);
+  vattn::hyb::scan_kernel<<<blocks, 256, 0, stream>>>(reinterpret_cast<float4*>(wsS), reinterpret_cast<float4*>(S),
+                                                      nS4, reinterpret_cast<float4*>(wsz),
+                                                      reinterpret_cast<float4*>(z), nz4, C);
+  VATTN_CUDA(cudaGetLastError());
+  return VATTN_OK;
+}
+}  // namespace
+
+extern "C" {
+
+vattn_status vattn_hybrid_delta(const void* k, const void* v, int B, int L, int H, int d, int chunk_tokens,
+                                void* workspace, size_t workspace_bytes, vattn_stream stream) {
+  if (!k || !v) return fail(VATTN_ERR_INVALID_ARG, "NULL pointer");
+  if (!aligned16(k) || !aligned16(v)) return fail(VATTN_ERR_INVALID_ARG, "k, v must be 16-byte aligned");
+  int C;
+  if (vattn_status st = check_hybrid(B, L, H, d, chunk_tokens, workspace, workspace_bytes, &C)) return st;
+  float* wsS = static_cast<float*>(workspace);
+  float* wsz = wsS + static_cast<size_t>(C) * B * H * d * d;
+  uint32_t* status;
+  if (vattn_status st = status_ptr(&status)) return st;
+  CUtensorMap mk, mv;
+  if (vattn_status st = make_map(&mk, k, d, H, L, B, 128)) return st;
+  if (vattn_status st = make_map(&mv, v, d, H, L, B, 128)) return st;
+  return launch_delta(mk, mv, wsS, wsz, status, B, L, H, C, chunk_tokens, stream);
+}
+
+vattn_status vattn_hybrid_scan(float* S, float* z, int B, int L, int H, int d, int chunk_tokens, void* workspace,
+                               size_t workspace_bytes, vattn_stream stream) {
+  if (!S || !z) return fail(VATTN_ERR_INVALID_ARG, "NULL pointer");
+  if (!aligned16(S) || !aligned16(z)) return fail(VATTN_ERR_INVALID_ARG, "S, z must be 16-byte aligned");
+  int C;
+  if (vattn_status st = check_hybrid(B, L, H, d, chunk_tokens, workspace, workspace_bytes, &C)) return st;
+  float* wsS = static_cast<float*>(workspace);
+  float* wsz = wsS + static_cast<size_t>(C) * B * H * d * d;
+  return launch_scan(wsS, wsz, S, z, B, H, d, C, stream);
+}
+
+vattn_status vattn_hybrid_chunk(const void* q, const void* k, const void* v, void* o, float* S, float* z, int B,
+                                int L, int H, int d, int chunk_tokens, float scale, void* workspace,
+                                size_t workspace_bytes, vattn_stream stream) {
+  if (!q || !k || !v || !o || !S || !z) return fail(VATTN_ERR_INVALID_ARG, "NULL pointer");
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(S) || !aligned16(z))
+    return fail(VATTN_ERR_INVALID_ARG, "pointers must be 16-byte aligned");
+  if (!std::isfinite(scale)) return fail(VATTN_ERR_INVALID_ARG, "scale not finite");
+  int C;
+  if (vattn_status st = check_hybrid(B, L, H, d, chunk_tokens, workspace, workspace_bytes, &C)) return st;
   float* wsS = static_cast<float*>(workspace);
   float* wsz = wsS + static_cast<size_t>(C) * B * H * d * d;
   uint32_t* status;
@@ -718,28 +785,9 @@ vattn_status vattn_hybrid_chunk(const void* q, const void* k, const void* v, voi
   if (vattn_status st = make_map(&mk, k, d, H, L, B, 128)) return st;
   if (vattn_status st = make_map(&mv, v, d, H, L, B, 128)) return st;
 
-  // (1) per-chunk state deltas
-  {
-    static uint64_t done[1];
-    auto kern = vattn::hyb::delta_kernel<128>;
-    const int smem = vattn::hyb::DeltaCfg<128>::kSmemBytes;
-    if (vattn_status st = ensure_smem(kern, smem, done)) return st;
-    vattn::hyb::DeltaParams dp{wsS, wsz, status, B, L, H, chunk_tokens};
-    kern<<<dim3(H, C, B), vattn::hyb::kDeltaThreads, smem, stream>>>(mk, mv, dp);
-    VATTN_CUDA(cudaGetLastError());
-  }
-  // (2) exclusive scan over chunks (+ state out)
-  {
-    const long long nS4 = static_cast<long long>(B) * H * d * d / 4, nz4 = static_cast<long long>(B) * H * d / 4;
-    int sms = 148, dev;
-    if (current_device(&dev) == VATTN_OK) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    const long long want = (nS4 + nz4 + 255) / 256;
-    const int blocks = static_cast<int>(want < sms * 4LL ? want : sms * 4LL);
-    vattn::hyb::scan_kernel<<<blocks, 256, 0, stream>>>(reinterpret_cast<float4*>(wsS), reinterpret_cast<float4*>(S),
-                                                        nS4, reinterpret_cast<float4*>(wsz),
-                                                        reinterpret_cast<float4*>(z), nz4, C);
-    VATTN_CUDA(cudaGetLastError());
-  }
+  // (1) per-chunk state deltas, (2) exclusive scan over chunks (+ state out)
+  if (vattn_status st = launch_delta(mk, mv, wsS, wsz, status, B, L, H, C, chunk_tokens, stream)) return st;
+  if (vattn_status st = launch_scan(wsS, wsz, S, z, B, H, d, C, stream)) return st;
   // (3) attention with linear-state initialisation
   vattn::attn::Params p{};
   p.o = static_cast<__nv_bfloat16*>(o);
@@ -761,11 +809,7 @@ vattn_status vattn_hybrid_chunk(const void* q, const void* k, const void* v, voi
   p.n_q_tiles = C * p.q_tiles_per_seg;
   p.hyb_S = wsS;
   p.hyb_z = wsz;
-#if VATTN_PAIR_TILES
   return launch_pair<128, vattn::attn::kRopeNone, true>(mq, mk, mv, mk, mv, p, stream);
-#else
-  return launch_attention<128, vattn::attn::kRopeNone, true>(mq, mk, mv, mk, mv, p, stream);
-#endif
 }
 
 // ------------------------------------------------- hybrid without workspace
@@ -813,6 +857,29 @@ vattn_status vattn_hybrid_chunk_noalloc(const void* q, const void* k, const void
                             VATTN_HYBRID_NOALLOC_MAX_BYTES, stream);
 }
 
+// ----------------------------------------------------------------- merge
+vattn_status vattn_attention_merge(const void* o_parts, const float* lse_parts, int R, void* o, float* lse, int B,
+                                   int L, int H, int d, vattn_stream stream) {
+  if (!o_parts || !lse_parts || !o) return fail(VATTN_ERR_INVALID_ARG, "NULL pointer");
+  if (!aligned16(o_parts) || !aligned16(o) || (reinterpret_cast<uintptr_t>(lse_parts) & 3u) ||
+      (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)))
+    return fail(VATTN_ERR_INVALID_ARG, "o_parts and o must be 16-byte aligned, lse 4-byte aligned");
+  if (R < 1 || R > vattn::merge::kMaxParts) return fail(VATTN_ERR_INVALID_ARG, "R=%d (1..%d)", R,
+                                                         vattn::merge::kMaxParts);
+  if (B < 1 || L < 1 || H < 1) return fail(VATTN_ERR_INVALID_ARG, "sizes must be >= 1");
+  if (d < 8 || d % 8) return fail(VATTN_ERR_UNSUPPORTED, "head dim %d (multiple of 8 required)", d);
+  vattn::merge::MergeParams mp{static_cast<const uint4*>(o_parts), lse_parts, static_cast<uint4*>(o), lse,
+                               R, B, L, H, d};
+  const long long n = static_cast<long long>(B) * L * H * (d / 8);
+  int sms = 148, dev;
+  if (current_device(&dev) == VATTN_OK) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const long long want = (n + 255) / 256;
+  const int blocks = static_cast<int>(want < sms * 8LL ? want : sms * 8LL);
+  vattn::merge::merge_kernel<<<blocks, 256, 0, stream>>>(mp);
+  VATTN_CUDA(cudaGetLastError());
+  return VATTN_OK;
+}
+
 // ------------------------------------------------------------- self-test
 // Not part of the attention interface: checks the tensor-core operand
 // layouts (see include/vattn_selftest.h).
@@ -840,6 +907,32 @@ vattn_status vattn_selftest_wait_timeout(uint32_t limit_us, vattn_stream stream)
   uint32_t* status;
   if (vattn_status st = status_ptr(&status)) return st;
   vattn::selftest::wait_timeout_kernel<<<1, 32, 0, stream>>>(static_cast<uint64_t>(limit_us) * 1000ull, status);
+  VATTN_CUDA(cudaGetLastError());
+  return VATTN_OK;
+}
+
+// Not part of the attention interface: the two-tile attention kernel with
+// one softmax arrival withheld and a short wait bound (see
+// include/vattn_selftest.h).
+vattn_status vattn_selftest_attention_timeout(const void* q, const void* k, const void* v, void* o, int L, int H,
+                                              int d, uint32_t limit_us, vattn_stream stream) {
+  if (limit_us == 0 || limit_us > 2000000) return fail(VATTN_ERR_INVALID_ARG, "limit_us must be 1..2000000");
+  if (L < 2 * vattn::attn::kTileN)
+    return fail(VATTN_ERR_INVALID_ARG, "L=%d: at least two key tiles are needed to withhold sub-tile 1", L);
+  return attention_impl(q, k, v, o, nullptr, 1, L, L, H, H, d, d == 64 ? 0.125f : 0.08838834764831845f,
+                        VATTN_FULL, 0, 1, 0, 0, 0, 0, nullptr, nullptr, nullptr, 0, stream,
+                        static_cast<uint64_t>(limit_us) * 1000ull, 1);
+}
+
+// Not part of the attention interface: the softmax's exponentials element
+// by element (see include/vattn_selftest.h).
+vattn_status vattn_selftest_ex2(int variant, const float* x, float* y, int n, vattn_stream stream) {
+  if (variant < 0 || variant > 2) return fail(VATTN_ERR_INVALID_ARG, "variant %d", variant);
+  if (!x || !y || n < 1 || (variant == 1 && (n & 1)))
+    return fail(VATTN_ERR_INVALID_ARG, "x, y non-NULL, n >= 1 (even for variant 1)");
+  int blocks = (n + 255) / 256;
+  if (blocks > 4096) blocks = 4096;
+  vattn::selftest::ex2_kernel<<<blocks, 256, 0, stream>>>(x, y, n, variant);
   VATTN_CUDA(cudaGetLastError());
   return VATTN_OK;
 }
