@@ -453,7 +453,24 @@ def secondary_measurements(va, torch, device, flush):
                         "clocks": batch["clocks"]}
     out["stream"] = stream
     cache.close()
-    del qd, kd, vd, kr, vr
+    del kr, vr
+    # the same stream through the one-launch step (attend + append fused),
+    # ring of W + 1 = 5 frames
+    out["stream_step"] = stream_step_figure(va, torch, device, frames, c, pk, window_relative=False)
+    del qd, kd, vd, frames
+    # FlashDecoder-XL-shaped streams: 24 heads on 3 KV heads, window 2,
+    # positions relative to the window, one launch per step
+    for name in ("xl480", "xl720", "xl480_refine"):
+        cx = si.CONFIGS[name]
+        Fx = cx["sub"] * cx["Hg"] * cx["Wg"]
+        qx, kx, vx = si.qkv(name)
+        Tx = cx["T"]
+        qd = dev(qx).view(Tx, Fx, cx["H"], cx["d"])
+        kd = dev(kx).view(Tx, Fx, cx["Hkv"], cx["d"])
+        vd = dev(vx).view(Tx, Fx, cx["Hkv"], cx["d"])
+        fr = [(qd[f].unsqueeze(0), kd[f].unsqueeze(0), vd[f].unsqueeze(0)) for f in range(Tx)]
+        out[name] = stream_step_figure(va, torch, device, fr, cx, pk, window_relative=True)
+        del qd, kd, vd, fr
     # hybrid chunk attention
     c = si.CONFIGS["hybrid"]
     L, H, d = c["T"] * c["Hg"] * c["Wg"], c["H"], c["d"]
@@ -496,8 +513,63 @@ def secondary_measurements(va, torch, device, flush):
     del g, wss
     hyb["scan"] = {"single_launch": _hbm(pk, scan_bytes, one), "graph16": _hbm(pk, scan_bytes, batch)}
     out["hybrid"] = hyb
+    # the MobileWan page variant on the same inputs: chunks of 4 frames
+    # overlapping 2 frames, polynomial feature maps
+    cp = si.CONFIGS["hybrid_page"]
+    ctp = cp["chunk_frames"] * cp["Hg"] * cp["Wg"]
+    ovp = cp["overlap_frames"] * cp["Hg"] * cp["Wg"]
+    coef = torch.from_numpy(si.poly_coef(cp["coef_seed"], H).astype(np.float32)).to(device)
+    wsp = torch.empty(va.vattn_hybrid_workspace_bytes_ex(1, L, H, d, ctp, ovp), dtype=torch.uint8, device=device)
+    fn = lambda: va.vattn_hybrid_chunk_ex(qd, kd, vd, o, S, z, ctp, ovp, coef=coef, workspace=wsp)
+    m = _measure(torch, fn)
+    pairs = 0
+    for ci in range((L + ctp - 1) // ctp):
+        q0, q1 = ci * ctp, min(L, (ci + 1) * ctp)
+        pairs += (q1 - q0) * (q1 - max(0, q0 - ovp))
+    flops = 4.0 * d * pairs * H + (2.0 * d * d + 2.0 * d) * L * H * 2
+    tf = flops / m["median_ms"] * 1e-9
+    out["hybrid_page"] = dict(m, tflops=tf, frac_of_peak=tf / pk["bf16_tflops"], mask_adjusted_flops=flops)
     va.vattn_check()
     return out
+
+
+def stream_step_figure(va, torch, device, frames, c, pk, window_relative):
+    """Frames/s of a whole stream decoded with vattn_kvcache_step (attend and
+    append in one launch per frame), ring of W + 1 frames, with its fraction
+    of the tensor-peak ceiling (the stream's mask-adjusted FLOPs at the
+    measured bf16 peak)."""
+    T = len(frames)
+    _, F, H, d = frames[0][0].shape
+    Hkv = frames[0][1].shape[2]
+    wb = c["window_back"]
+    cap = wb + 1
+    kr = torch.zeros((cap, 1, F, Hkv, d), dtype=torch.bfloat16, device=device)
+    cache = va.KVCache(kr, torch.zeros_like(kr), torch.zeros(cap, dtype=torch.int32, device=device))
+    sub = c.get("sub", 1)
+    rope = va.Rope(Hg=c["Hg"], Wg=c["Wg"], pairs=c["pairs"], max_pos=max(64, c["Hg"], c["Wg"]))
+    tab = va.rope_table(rope, d, device=device)
+    cache.enable_rope(torch.zeros((cap + 1, 1, F, Hkv, d), dtype=torch.bfloat16, device=device), rope, tab)
+    of = torch.empty((1, F, H, d), dtype=torch.bfloat16, device=device)
+    ws = cache.step_workspace(H, wb)
+
+    def run():
+        for f in range(T):
+            qf, kf, vf = frames[f]
+            cache.step(qf, kf, vf, of, f, wb, rope=rope, table=tab, window_relative=window_relative, workspace=ws)
+
+    m = _measure(torch, run)
+    va.vattn_check()
+    cache.close()
+    pairs = sum(min(f, wb) + 1 for f in range(T))
+    flops = 4.0 * d * F * F * H * pairs
+    tf = flops / m["median_ms"] * 1e-9
+    fps = T / (m["median_ms"] / 1e3)
+    ceiling = T / (flops / (pk["bf16_tflops"] * 1e12))
+    return dict(m, frames_per_s=fps, latent_frames_per_s=fps * sub, ms_per_frame=m["median_ms"] / T, tflops=tf,
+                frac_of_ceiling=fps / ceiling, ceiling_frames_per_s=ceiling, launches_per_frame=1,
+                workload="%d steps of %d tokens (%d latent frames of %dx%d), H=%d on %d KV heads, d=%d, "
+                         "window %d, %s positions" % (T, F, sub, c["Hg"], c["Wg"], H, Hkv, d, wb + 1,
+                                                     "window-relative" if window_relative else "absolute"))
 
 
 def cpu_baseline(w, rows=20480):
@@ -559,6 +631,69 @@ def run_reference(args, rank, world):
                 e2e={"value": val, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0})
 
 
+def run_case(args, device):
+    """One workload's calls, `steps` times after `warmup`, for profilers (ncu
+    captures one kernel of one case): prints one line with the mean time."""
+    import torch
+    import video_diffusion_transformer_02_b200 as va
+    torch.cuda.set_device(device)
+    dev = lambda x: torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).to(device)
+    name = args.case
+    if name in ("stream_frame", "xl480_frame", "xl720_frame"):
+        cname = {"stream_frame": "stream", "xl480_frame": "xl480", "xl720_frame": "xl720"}[name]
+        c = si.CONFIGS[cname]
+        F, H, d, wb = c["Hg"] * c["Wg"], c["H"], c["d"], c["window_back"]
+        Hkv = c.get("Hkv", H)
+        nf = wb + 1
+        q, k, v = si.qkv(cname, L=nf * F)
+        qd, kd, vd = dev(q).view(nf, F, H, d), dev(k).view(nf, F, Hkv, d), dev(v).view(nf, F, Hkv, d)
+        cap = wb + 1
+        kr = torch.zeros((cap, 1, F, Hkv, d), dtype=torch.bfloat16, device=device)
+        cache = va.KVCache(kr, torch.zeros_like(kr), torch.zeros(cap, dtype=torch.int32, device=device))
+        rope = va.Rope(Hg=c["Hg"], Wg=c["Wg"], pairs=c["pairs"], max_pos=4096)   # frame index grows per call
+        tab = va.rope_table(rope, d, device=device)
+        cache.enable_rope(torch.zeros((cap + 1, 1, F, Hkv, d), dtype=torch.bfloat16, device=device), rope, tab)
+        of = torch.empty((1, F, H, d), dtype=torch.bfloat16, device=device)
+        rel = cname != "stream"
+        for f in range(wb):   # fill the window
+            cache.step(qd[f:f + 1], kd[f:f + 1], vd[f:f + 1], of, f, wb, rope=rope, table=tab, window_relative=rel)
+        i = [wb]
+
+        def fn():   # one steady frame (the window full), the frame index advancing
+            f = i[0]
+            cache.step(qd[wb:wb + 1], kd[wb:wb + 1], vd[wb:wb + 1], of, f, wb, rope=rope, table=tab,
+                       window_relative=rel)
+            i[0] += 1
+    elif name in ("hybrid", "hybrid_page"):
+        c = si.CONFIGS[name]
+        L, H, d = c["T"] * c["Hg"] * c["Wg"], c["H"], c["d"]
+        ct = c["chunk_frames"] * c["Hg"] * c["Wg"]
+        ov = c.get("overlap_frames", 0) * c["Hg"] * c["Wg"]
+        q, k, v = si.qkv(name)
+        qd, kd, vd = dev(q), dev(k), dev(v)
+        o = torch.empty_like(qd)
+        S = torch.zeros((1, H, d, d), dtype=torch.float32, device=device)
+        z = torch.zeros((1, H, d), dtype=torch.float32, device=device)
+        coef = (torch.from_numpy(si.poly_coef(c["coef_seed"], H).astype(np.float32)).to(device)
+                if "coef_seed" in c else None)
+        fn = lambda: va.vattn_hybrid_chunk_ex(qd, kd, vd, o, S, z, ct, ov, coef=coef)
+    elif name == "wan13b":
+        w = wan13b_workload(va, torch, device)
+        fn = lambda: va.vattn_attention(w["q"], w["k"], w["v"], w["o"], scale=w["scale"], rope=w["rope"],
+                                        table=w["tab"], workspace=w["ws"])
+    else:
+        raise SystemExit("unknown case %s" % name)
+    for _ in range(args.warmup):
+        fn()
+    torch.cuda.synchronize()
+    ms = _event_list(torch, fn, args.steps)
+    va.vattn_check()
+    print(json.dumps({"case": name, "steps": args.steps, "mean_ms": statistics.mean(ms), "ms": ms}), flush=True)
+
+
+CASES = ("wan13b", "stream_frame", "xl480_frame", "xl720_frame", "hybrid", "hybrid_page")
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -569,7 +704,13 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-rows", type=int, default=20480)
     ap.add_argument("--ref-rows", type=int, default=512)
+    ap.add_argument("--case", choices=CASES, default=None,
+                    help="run only this workload's calls (for profilers); prints its mean time")
     args = ap.parse_args()
+    if args.case:
+        import torch
+        run_case(args, torch.device("cuda", int(os.environ.get("LOCAL_RANK", "0"))))
+        return
     args.warmup = max(args.warmup, 3) if args.impl == "ours" else args.warmup
 
     world = int(os.environ.get("WORLD_SIZE", "1"))

@@ -195,7 +195,9 @@ vattn_status vattn_kvcache_restore(vattn_kvcache* cache, const int32_t* host_ids
  * Keep a second, rotated copy of the keys so that each frame's keys are
  * rotated once, at their absolute frame index, instead of once per query
  * tile that reads them (FlashDecoder applies RoPE with precomputed tables,
- * "Inference Optimization", Sec. 4.6).  k_ring_rot: caller-owned bf16
+ * "Inference Optimization", Sec. 4.6).  The frame tokens F must be a
+ * multiple of rope->Hg * rope->Wg (F / (Hg*Wg) latent frames per cache
+ * frame, see vattn_kvcache_step).  k_ring_rot: caller-owned bf16
  * [capacity + 1][B][F][Hkv][d]; frame f's rotated keys live in slot
  * f % (capacity + 1).  From then on vattn_attention_stream (which must then
  * be given the same rope and table) rotates the current frame's keys into
@@ -210,6 +212,50 @@ vattn_status vattn_kvcache_restore(vattn_kvcache* cache, const int32_t* host_ids
 vattn_status vattn_kvcache_enable_rope(vattn_kvcache* cache, void* k_ring_rot, const vattn_rope* rope,
                                        const float* table, vattn_stream stream);
 vattn_status vattn_kvcache_destroy(vattn_kvcache* cache);
+
+/*
+ * One whole streaming step in a single launch (FlashDecoder "Streaming with
+ * Rolling KV Cache", Sec. 3.3, Frame-by-Frame Processing; the fixed,
+ * data-independent per-frame work that "Inference Optimization", Sec. 4.6,
+ * captures in a CUDA graph): the F query tokens of frame `frame_idx` attend
+ * to the current frame (k_cur, v_cur) and to the cached frames
+ * frame_idx-window_back .. frame_idx-1 present in the ring, and the current
+ * frame is appended: raw K and V into slot frame_idx % capacity, frame_ids
+ * updated, and (with rope) its keys rotated into the rotated ring.  The
+ * result equals vattn_attention_stream followed by vattn_kvcache_append.
+ *  - capacity must exceed window_back: the slot written is then never one
+ *    the window reads (capacity W + 1 for a window of W frames).
+ *  - rope/table (both or neither): the cache must have a rotated-key ring
+ *    with the same rope and table (vattn_kvcache_enable_rope).  A cache frame
+ *    of F tokens holds r = F / (Hg*Wg) latent frames (r > 1: the temporal
+ *    refinement layers' r_t * L_frm tokens per step, FlashDecoder
+ *    "Complexity Analysis", Sec. 3.3); token n of cache frame f sits at
+ *    t = r * (f - base) + n / (Hg*Wg).
+ *  - window_relative = 0: base = 0 (absolute frame index).  1: base =
+ *    max(0, frame_idx - window_back), positions relative to the current
+ *    window ("Long Video Decoding", Sec. 4.3), so the table needs only
+ *    r * (window_back + 1) frame rows however long the video; the window's
+ *    earlier frames are rotated again at their new positions (one HBM pass
+ *    each) before the launch.
+ *  - workspace: device memory of vattn_kvcache_step_workspace_bytes(cache,
+ *    H, window_back) bytes (the value depends on the current device's SM
+ *    count), zero-filled before its first use; every step leaves its
+ *    counters at zero.  Steps sharing a workspace must not overlap on the
+ *    GPU.
+ * The first CTAs of the launch copy and rotate the frame; attention CTAs
+ * wait for them (a bounded wait on a counter in the workspace) only before
+ * loading the current frame's rotated keys, which they reach last.  For a
+ * small number of query tiles the key tiles are split across CTAs and each
+ * query-tile pair's last CTA merges the partial results exactly.  When the
+ * window holds no earlier frame the append runs as a separate launch first.
+ * A wait that gives up records VATTN_ERR_TIMEOUT; zero the workspace again
+ * before the next step after that.
+ */
+size_t vattn_kvcache_step_workspace_bytes(const vattn_kvcache* cache, int H, int window_back);
+vattn_status vattn_kvcache_step(vattn_kvcache* cache, const void* q, const void* k_cur, const void* v_cur, void* o,
+                                float* lse, int H, int frame_idx, int window_back, float scale,
+                                const vattn_rope* rope, const float* table, int window_relative, void* workspace,
+                                size_t workspace_bytes, vattn_stream stream);
 
 /*
  * Hybrid chunk attention (MobileWan recurrence distillation: softmax
@@ -235,6 +281,30 @@ vattn_status vattn_hybrid_chunk(const void* q, const void* k, const void* v, voi
                                 float* z, int B, int L, int H, int d, int chunk_tokens,
                                 float scale, void* workspace, size_t workspace_bytes,
                                 vattn_stream stream);
+
+/*
+ * Hybrid chunk attention, general form: the MobileWan page variant (review
+ * of "MobileWan", axiom ledger / App. A.3.1: learnable polynomial feature
+ * maps of degree 3 for phi_q and phi_k, softmax chunks overlapping the
+ * previous chunk by T_o frames).
+ *   fmap VATTN_FMAP_ELU1: phi(x) = elu(x) + 1 (coef unused, may be NULL);
+ *   fmap VATTN_FMAP_POLY3: phi_q(x) = a0 + a1 x + a2 x^2 + a3 x^3 with
+ *     (a0..a3) = coef[(0 * H + h) * 4 ..], phi_k likewise from
+ *     coef[(1 * H + h) * 4 ..]; coef: device fp32 [2][H][4], 16-byte aligned.
+ *   overlap_tokens ov >= 0: the softmax part of chunk c covers the keys
+ *     [max(0, c * ct - ov), min(L, (c + 1) * ct)) -- its chunk and the last
+ *     ov tokens before it -- and the linear part the keys before that window
+ *     (plus the incoming state).  The overlap reaches back inside this call
+ *     only: chunk 0 has none.  S, z leave as the state after all L tokens.
+ *   workspace: vattn_hybrid_workspace_bytes_ex(...) bytes.
+ * With fmap ELU1 and ov = 0 this is vattn_hybrid_chunk.
+ */
+typedef enum { VATTN_FMAP_ELU1 = 0, VATTN_FMAP_POLY3 = 1 } vattn_feature_map;
+size_t vattn_hybrid_workspace_bytes_ex(int B, int L, int H, int d, int chunk_tokens, int overlap_tokens);
+vattn_status vattn_hybrid_chunk_ex(const void* q, const void* k, const void* v, void* o, float* S, float* z, int B,
+                                   int L, int H, int d, int chunk_tokens, int overlap_tokens, float scale,
+                                   vattn_feature_map fmap, const float* coef, void* workspace,
+                                   size_t workspace_bytes, vattn_stream stream);
 
 /*
  * The state part of vattn_hybrid_chunk as two separate calls, for callers

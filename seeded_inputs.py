@@ -103,11 +103,44 @@ CONFIGS = {
     # index 3: MobileWan-style hybrid chunk attention (31 frames of 15x26)
     "hybrid": dict(index=3, B=1, H=24, d=128, T=31, Hg=15, Wg=26,
                    pairs=None, theta=None, mode="hybrid", chunk_frames=3),
+    # the MobileWan page variant on the same inputs as "hybrid": chunks of
+    # T_c = 4 latent frames whose softmax reaches T_o = 2 frames into the
+    # previous chunk, degree-3 polynomial feature maps (synthetic
+    # coefficients, poly_coef(seed 0x9017, H))
+    "hybrid_page": dict(index=3, B=1, H=24, d=128, T=31, Hg=15, Wg=26,
+                        pairs=None, theta=None, mode="hybrid", chunk_frames=4,
+                        overlap_frames=2, coef_seed=0x9017),
     # index 4: Wan2.1-14B-like 720p, full and chunk-causal (chunk = 3 frames)
     "wan14b": dict(index=4, B=1, H=40, d=128, T=21, Hg=45, Wg=80,
                    pairs=(22, 21, 21), theta=10000.0, mode="full+chunk",
                    chunk_frames=3),
+    # indices 5-7: FlashDecoder-XL-shaped streaming (24 query heads sharing 3
+    # KV heads, head dim 64, window W_frm = 2: itself + 1 previous frame),
+    # Wan2.2 latent grids of 480p (30x52) and 720p (45x80), positions
+    # relative to the window; xl480_refine: a temporal-refinement layer
+    # (r_t = 4 latent frames of 30x52 per step, window r_t * W_frm frames)
+    "xl480": dict(index=5, B=1, H=24, Hkv=3, d=64, T=16, Hg=30, Wg=52, sub=1,
+                  pairs=(12, 10, 10), theta=10000.0, mode="stream",
+                  window_back=1, capacity=2),
+    "xl720": dict(index=6, B=1, H=24, Hkv=3, d=64, T=16, Hg=45, Wg=80, sub=1,
+                  pairs=(12, 10, 10), theta=10000.0, mode="stream",
+                  window_back=1, capacity=2),
+    "xl480_refine": dict(index=7, B=1, H=24, Hkv=3, d=64, T=8, Hg=30, Wg=52, sub=4,
+                         pairs=(12, 10, 10), theta=10000.0, mode="stream",
+                         window_back=1, capacity=2),
 }
+
+
+def poly_coef(seed: int, H: int) -> np.ndarray:
+    """Synthetic coefficients (a0, a1, a2, a3) of degree-3 polynomial feature
+    maps, one per head for q (index 0) and for k (index 1): [2, H, 4]
+    float64 values that are exactly representable in fp32.  Ranges keep the
+    maps positive on average over N(0, 1) inputs: a0 in [0.5, 1), a1 in
+    [0.2, 0.5), a2 in [0.1, 0.3), a3 in [0, 0.05)."""
+    u = uniform01(seed, 2 * H * 4).reshape(2, H, 4)
+    lo = np.array([0.5, 0.2, 0.1, 0.0])
+    hi = np.array([1.0, 0.5, 0.3, 0.05])
+    return (lo + u * (hi - lo)).astype(np.float32).astype(np.float64)
 
 
 def qkv(config: str, L: int | None = None, H: int | None = None):
@@ -117,10 +150,12 @@ def qkv(config: str, L: int | None = None, H: int | None = None):
     the same stream order is NOT implied: a smaller shape is a new draw).
     """
     c = CONFIGS[config]
-    L = c["T"] * c["Hg"] * c["Wg"] if L is None else L
+    L = c["T"] * c.get("sub", 1) * c["Hg"] * c["Wg"] if L is None else L
     H = c["H"] if H is None else H
-    shape = (c["B"], L, H, c["d"])
-    return tuple(normal_bf16(seed_for(c["index"], w), shape) for w in ("q", "k", "v"))
+    Hkv = c.get("Hkv", H) if H == c["H"] else H
+    return (normal_bf16(seed_for(c["index"], "q"), (c["B"], L, H, c["d"])),
+            normal_bf16(seed_for(c["index"], "k"), (c["B"], L, Hkv, c["d"])),
+            normal_bf16(seed_for(c["index"], "v"), (c["B"], L, Hkv, c["d"])))
 
 
 def sample_rows(seed: int, n: int, B: int, H: int, L: int, forced=()) -> np.ndarray:

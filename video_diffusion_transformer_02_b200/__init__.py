@@ -84,9 +84,14 @@ _kv_ids = _sig("vattn_kvcache_frame_ids", _I, _P, _P)
 _kv_restore = _sig("vattn_kvcache_restore", _I, _P, _P, _P)
 _kv_rope = _sig("vattn_kvcache_enable_rope", _I, _P, _P, _RP, _P, _P)
 _kv_destroy = _sig("vattn_kvcache_destroy", _I, _P)
+_kv_step_ws = _sig("vattn_kvcache_step_workspace_bytes", _S, _P, _I, _I)
+_kv_step = _sig("vattn_kvcache_step", _I, _P, _P, _P, _P, _P, _P, _I, _I, _I, _F, _RP, _P, _I, _P, _S, _P)
 _hyb_ws = _sig("vattn_hybrid_workspace_bytes", _S, _I, _I, _I, _I, _I)
 _hybrid = _sig("vattn_hybrid_chunk", _I, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _P, _S, _P)
 _hybrid_delta = _sig("vattn_hybrid_delta", _I, _P, _P, _I, _I, _I, _I, _I, _P, _S, _P)
+_hyb_ws_ex = _sig("vattn_hybrid_workspace_bytes_ex", _S, _I, _I, _I, _I, _I, _I)
+_hybrid_ex = _sig("vattn_hybrid_chunk_ex", _I, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _I, _P, _P, _S, _P)
+FMAP_ELU1, FMAP_POLY3 = 0, 1
 _hybrid_scan = _sig("vattn_hybrid_scan", _I, _P, _P, _I, _I, _I, _I, _I, _P, _S, _P)
 _hybrid_noalloc = _sig("vattn_hybrid_chunk_noalloc", _I, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _P)
 _selftest = _sig("vattn_selftest_umma", _I, _I, _P, _P, _P, _P)
@@ -334,6 +339,25 @@ class KVCache:
         vattn_attention_stream(self, q, k_cur, v_cur, o, lse, frame_idx, window_back, scale, rope,
                                table, stream)
 
+    def step(self, q, k_cur, v_cur, o, frame_idx, window_back, scale=None, lse=None, rope=None, table=None,
+             window_relative=False, workspace=None, stream=None):
+        """Attend and append frame frame_idx in one launch (vattn_kvcache_step)."""
+        vattn_kvcache_step(self, q, k_cur, v_cur, o, lse, frame_idx, window_back, scale, rope, table,
+                           window_relative, workspace, stream)
+
+    def step_workspace(self, H, window_back):
+        """A zero-filled workspace for step() (kept by the cache per (H, window_back))."""
+        key = (H, window_back)
+        ws = getattr(self, "_step_ws", {})
+        if key not in ws:
+            with torch.cuda.device(self.device):
+                n = vattn_kvcache_step_workspace_bytes(self, H, window_back)
+            if n == 0:
+                raise VattnError(ERR_INVALID_ARG, "no step workspace for H=%d window_back=%d" % key)
+            ws[key] = torch.zeros(n, dtype=torch.uint8, device=self.device)
+            self._step_ws = ws
+        return ws[key]
+
     def host_frame_ids(self):
         arr = (ctypes.c_int32 * self.capacity)()
         _ok(_kv_ids(self._h, arr))
@@ -413,6 +437,39 @@ def vattn_attention_stream(cache: KVCache, q, k_cur, v_cur, o, lse, frame_idx, w
                               window_back, float(scale), _rope_c(rope), _ptr(table), _stream(stream, dev)))
 
 
+def vattn_kvcache_step_workspace_bytes(cache: KVCache, H, window_back) -> int:
+    return _kv_step_ws(cache._h, H, window_back)
+
+
+def vattn_kvcache_step(cache: KVCache, q, k_cur, v_cur, o, lse, frame_idx, window_back, scale=None, rope=None,
+                       table=None, window_relative=False, workspace=None, stream=None):
+    _rank(q, "q", 4)
+    H = q.shape[2]
+    _expect(q, "q", _frame_shape(cache, H), torch.bfloat16)
+    _expect(k_cur, "k_cur", _frame_shape(cache, cache.Hkv), torch.bfloat16)
+    _expect(v_cur, "v_cur", _frame_shape(cache, cache.Hkv), torch.bfloat16)
+    _expect(o, "o", _frame_shape(cache, H), torch.bfloat16)
+    if lse is not None:
+        _expect(lse, "lse", (cache.B, H, cache.F), torch.float32)
+    if (rope is None) != (table is None):
+        raise ValueError("rope and table go together")
+    if table is not None:
+        _expect(table, "table", None, torch.float32)
+        _min_bytes(table, "table", vattn_rope_table_bytes(rope, cache.d))
+    if scale is None:
+        scale = cache.d ** -0.5
+    dev = _same_device(cache, ("q", q), ("k_cur", k_cur), ("v_cur", v_cur), ("o", o), ("lse", lse),
+                       ("table", table), ("workspace", workspace))
+    if workspace is None:
+        workspace = cache.step_workspace(H, window_back)
+    with torch.cuda.device(dev):
+        need = vattn_kvcache_step_workspace_bytes(cache, H, window_back)
+        _min_bytes(workspace, "workspace", need)
+        _ok(_kv_step(cache._h, _ptr(q), _ptr(k_cur), _ptr(v_cur), _ptr(o), _ptr(lse), H, frame_idx, window_back,
+                     float(scale), _rope_c(rope), _ptr(table), int(bool(window_relative)), _ptr(workspace),
+                     workspace.numel() * workspace.element_size(), _stream(stream, dev)))
+
+
 # ----------------------------------------------------------------- hybrid
 def vattn_hybrid_workspace_bytes(B, L, H, d, chunk_tokens) -> int:
     return _hyb_ws(B, L, H, d, chunk_tokens)
@@ -442,6 +499,32 @@ def vattn_hybrid_chunk(q, k, v, o, S, z, chunk_tokens, scale=None, workspace=Non
         _ok(_hybrid(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(S), _ptr(z), B, L, H, d, chunk_tokens,
                     float(scale), _ptr(workspace), workspace.numel() * workspace.element_size(),
                     _stream(stream, dev)))
+
+
+def vattn_hybrid_workspace_bytes_ex(B, L, H, d, chunk_tokens, overlap_tokens) -> int:
+    return _hyb_ws_ex(B, L, H, d, chunk_tokens, overlap_tokens)
+
+
+def vattn_hybrid_chunk_ex(q, k, v, o, S, z, chunk_tokens, overlap_tokens=0, scale=None, coef=None,
+                          workspace=None, stream=None):
+    """Hybrid chunk attention with chunk overlap and, when coef (fp32 [2, H, 4],
+    on the device) is given, the per-head degree-3 polynomial feature maps
+    (elu + 1 otherwise)."""
+    B, L, H, d = _check_hybrid(q, k, v, o, S, z)
+    if scale is None:
+        scale = d ** -0.5
+    if coef is not None:
+        _expect(coef, "coef", (2, H, 4), torch.float32)
+    dev = _device(("q", q), ("k", k), ("v", v), ("o", o), ("S", S), ("z", z), ("coef", coef),
+                  ("workspace", workspace))
+    need = vattn_hybrid_workspace_bytes_ex(B, L, H, d, chunk_tokens, overlap_tokens)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=dev)
+    _min_bytes(workspace, "workspace", need)
+    with torch.cuda.device(dev):
+        _ok(_hybrid_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(S), _ptr(z), B, L, H, d, chunk_tokens,
+                       overlap_tokens, float(scale), FMAP_POLY3 if coef is not None else FMAP_ELU1, _ptr(coef),
+                       _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream, dev)))
 
 
 def vattn_hybrid_delta(k, v, chunk_tokens, workspace, stream=None):

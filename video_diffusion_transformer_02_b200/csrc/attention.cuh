@@ -105,6 +105,9 @@ struct Params {
   // hybrid chunk attention: per-chunk exclusive state prefix
   const float* hyb_S;       // [C][B][H][D][D]
   const float* hyb_z;       // [C][B][H][D]
+  int hyb_fmap;             // feature map of the read-out (fmap::kFmapElu1 / kFmapPoly3)
+  const float* hyb_coef;    // [2][H][4] polynomial coefficients (map 0 = q is used here)
+  int lead;                 // SLIDING only: the key window also reaches this many tokens back
   // self-test knobs (zero in every attention call): a bound on each wait
   // other than the default, and withholding one softmax arrival so that a
   // wait of the MMA issuer runs out
@@ -167,6 +170,7 @@ __device__ __forceinline__ void key_range(const Params& p, int n, int& lo, int& 
   }
   a *= p.F;
   b *= p.F;
+  if (p.mode == kSliding) a -= p.lead;
   lo = static_cast<int>(a < 0 ? 0 : (a > p.Lk ? p.Lk : a));
   hi = static_cast<int>(b < 0 ? 0 : (b > p.Lk ? p.Lk : b));
 }

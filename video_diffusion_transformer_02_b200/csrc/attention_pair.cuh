@@ -29,6 +29,7 @@
 // sub-tile j+2 only after the P V of sub-tile j has completed.
 #pragma once
 #include "attention.cuh"
+#include "feature_map.cuh"
 
 namespace vattn {
 namespace attn {
@@ -149,6 +150,76 @@ __device__ __forceinline__ void append_share(const Params& p, int part) {
   __threadfence();
   __syncthreads();
   if (threadIdx.x == 0) atomicAdd(p.step_sync, 1u);
+}
+
+// The merge of a query-tile pair's key splits, by the pair's last CTA
+// (ReGenVC Sec. 3.5's exact combination, here of splits of one CTA's keys):
+// with lse_s = m_s + log2 l_s per split s, o = sum_s 2^(lse_s - M) o_s /
+// sum_s 2^(lse_s - M), M = max_s lse_s.  Warp w of the softmax warpgroups
+// merges 32 rows of its tile: each lane first forms its own row's weights,
+// then the warp walks the rows, lane l reading and writing columns
+// [l D/32, (l+1) D/32) (coalesced rows of the partials, from L2).
+template <int D>
+__device__ __forceinline__ void merge_splits(const Params& p, const PairGeom& g, int b, int h, int warp, int lane) {
+  const int x = (warp - 4) >> 2;
+  if (x == 1 && !g.hasB) return;
+  const int r0 = (x ? g.q0[1] : g.q0[0]) + (warp & 3) * 32;
+  const int q_end = x ? g.q_end[1] : g.q_end[0];
+  if (r0 >= q_end) return;
+  const int S = p.n_split;
+  const size_t split_rows = static_cast<size_t>(p.B) * p.H * p.Lq;   // rows of one split's partials
+  const size_t bh = (static_cast<size_t>(b) * p.H + h) * p.Lq;
+  const int myrow = r0 + lane;
+  float wts[kMaxSplit];
+  float M = -INFINITY;
+#pragma unroll
+  for (int s = 0; s < kMaxSplit; ++s) {
+    wts[s] = (s < S && myrow < q_end) ? __ldcg(p.part_lse + s * split_rows + bh + myrow) : -INFINITY;
+    M = fmaxf(M, wts[s]);
+  }
+  float W = 0.f;
+#pragma unroll
+  for (int s = 0; s < kMaxSplit; ++s) {
+    wts[s] = M == -INFINITY ? 0.f : ex2_approx(wts[s] - M);   // 0 for an empty split
+    W += wts[s];
+  }
+  const float invW = W > 0.f ? 1.f / W : 0.f;
+  if (p.lse && myrow < q_end)
+    p.lse[bh + myrow] = W > 0.f ? (M + __log2f(W)) * 0.69314718055994531f : -INFINITY;
+  constexpr int CPL = D / 32;   // columns per lane
+  const int nrows = min(32, q_end - r0);
+#pragma unroll 1
+  for (int rr = 0; rr < nrows; ++rr) {
+    float acc[CPL];
+#pragma unroll
+    for (int e = 0; e < CPL; ++e) acc[e] = 0.f;
+#pragma unroll
+    for (int s = 0; s < kMaxSplit; ++s) {
+      if (s < S) {
+        const float w = __shfl_sync(0xffffffffu, wts[s], rr);
+        const float* src = p.part_o + (s * split_rows + bh + r0 + rr) * D + lane * CPL;
+        if constexpr (CPL == 2) {
+          const float2 v = __ldcg(reinterpret_cast<const float2*>(src));
+          acc[0] = fmaf(w, v.x, acc[0]);
+          acc[1] = fmaf(w, v.y, acc[1]);
+        } else {
+          const float4 v = __ldcg(reinterpret_cast<const float4*>(src));
+          acc[0] = fmaf(w, v.x, acc[0]);
+          acc[1] = fmaf(w, v.y, acc[1]);
+          acc[2] = fmaf(w, v.z, acc[2]);
+          acc[3] = fmaf(w, v.w, acc[3]);
+        }
+      }
+    }
+    const float iw = __shfl_sync(0xffffffffu, invW, rr);
+    __nv_bfloat16* dst = p.o + ((static_cast<size_t>(b) * p.Lq + r0 + rr) * p.H + h) * D + lane * CPL;
+    if constexpr (CPL == 2) {
+      *reinterpret_cast<uint32_t*>(dst) = pack_bf16x2(acc[0] * iw, acc[1] * iw);
+    } else {
+      *reinterpret_cast<uint2*>(dst) = make_uint2(pack_bf16x2(acc[0] * iw, acc[1] * iw),
+                                                  pack_bf16x2(acc[2] * iw, acc[3] * iw));
+    }
+  }
 }
 
 // Last act of every CTA of a streaming step: count the exit; the last CTA
@@ -598,8 +669,9 @@ __global__ void __launch_bounds__(kPairThreads, 1)
                    (!hasB || mbar_wait(bODone(1), 0, ab, kStatusTimeoutSoftmax));
         tc_fence_after();
         const int c = g.q0[0] / p.q_seg_len;   // the pair's chunk
-        // phi(q_r) = elu(q_r) + 1 in place of row r of Q_x (bf16), and phi(q_r) . z_c in fp32
+        // phi(q_r) in place of row r of Q_x (bf16), and phi(q_r) . z_c in fp32
         const float* zc = p.hyb_z + ((static_cast<size_t>(c) * p.B + b) * p.H + h) * D;
+        const fmap::Poly aq = fmap::load_poly(p.hyb_coef, 0, p.H, h);
         const uint32_t qrow = sQ + static_cast<uint32_t>(x * C::kTileBytes);
 #pragma unroll 1
         for (int blk = 0; blk < D / 64; ++blk) {
@@ -614,8 +686,8 @@ __global__ void __launch_bounds__(kPairThreads, 1)
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
               float x0 = bf16lo_to_f32(w4[e]), x1 = bf16hi_to_f32(w4[e]);
-              x0 = x0 > 0.f ? x0 + 1.f : __expf(x0);
-              x1 = x1 > 0.f ? x1 + 1.f : __expf(x1);
+              x0 = fmap::feature(p.hyb_fmap, aq, x0);
+              x1 = fmap::feature(p.hyb_fmap, aq, x1);
               w4[e] = pack_bf16x2(x0, x1);
               // the denominator takes the same bf16 values the read-out MMA multiplies
               dl = fmaf(bf16lo_to_f32(w4[e]), zz[2 * e], dl);
@@ -669,7 +741,27 @@ __global__ void __launch_bounds__(kPairThreads, 1)
         tc_fence_after();
       }
       ok = __all_sync(0xffffffffu, ok);   // the TMEM loads below are warp-collective
-      if (ok) {
+      if (ok && !HYB && p.n_split > 1) {
+        // key split: this CTA's partial result, o / l in fp32 and m + log2 l,
+        // for the pair's merging CTA
+        const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
+        const size_t prow = ((static_cast<size_t>(split) * p.B + b) * p.H + h) * p.Lq + qn;
+        float* dst = p.part_o + prow * D;
+#pragma unroll 1
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t orr[32];
+          tmem_ld32(tO + c * 32, orr);
+          tmem_ld_wait_dep(orr);
+          if (row_valid) {
+#pragma unroll
+            for (int e = 0; e < 8; ++e)
+              __stcg(reinterpret_cast<float4*>(dst + c * 32) + e,
+                     make_float4(__uint_as_float(orr[4 * e]) * inv, __uint_as_float(orr[4 * e + 1]) * inv,
+                                 __uint_as_float(orr[4 * e + 2]) * inv, __uint_as_float(orr[4 * e + 3]) * inv));
+          }
+        }
+        if (row_valid) __stcg(p.part_lse + prow, l_run > 0.f ? m_run + __log2f(l_run) : -INFINITY);
+      } else if (ok) {
         // hybrid: o = (2^m O + lin) / (2^m l + phi(q).z) with O, l relative
         // to the softmax's reference max m; scaled by 2^-m when m > 0, so
         // neither factor overflows
@@ -714,12 +806,31 @@ __global__ void __launch_bounds__(kPairThreads, 1)
     }
   }
 
+  if (!HYB && p.n_split > 1 && warp >= 4 && warp < 12) {
+    // key split: count this CTA's partial in; the pair's last CTA merges
+    __threadfence();
+    asm volatile("bar.sync 2, 256;" ::: "memory");
+    volatile uint32_t* last = misc + 2;
+    const size_t pc = (static_cast<size_t>(b) * p.H + h) * p.n_pairs + pr;
+    if (threadIdx.x == 128) {
+      const uint32_t old = atomicAdd(p.pair_count + pc, 1u);
+      *last = old == static_cast<uint32_t>(p.n_split) - 1u ? 1u : 0u;
+      __threadfence();
+    }
+    asm volatile("bar.sync 2, 256;" ::: "memory");
+    if (*last) {
+      merge_splits<D>(p, g, b, h, warp, lane);
+      if (threadIdx.x == 128) p.pair_count[pc] = 0u;
+    }
+  }
+
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);
   }
+  if (stepping) step_exit(p);
 }
 
 }  // namespace attn

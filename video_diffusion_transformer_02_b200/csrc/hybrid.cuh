@@ -1,15 +1,23 @@
 // Hybrid chunk attention, state part (MobileWan recurrence distillation:
 // causal linear attention across chunks carried in a running state (s, z),
-// feature map phi(x) = elu(x) + 1 after Katharopoulos et al.).
+// feature map phi = elu + 1 or a per-head degree-3 polynomial, see
+// feature_map.cuh).
 //
-//   dS_c = sum_{j in chunk c} phi(k_j) v_j^T   (D x D, fp32)   -- tcgen05 MMA
-//   dz_c = sum_{j in chunk c} phi(k_j)          (D, fp32)       -- CUDA cores
-//   S_c  = S_in + sum_{c' < c} dS_c'  (exclusive scan over chunks), same for z
+//   dS_c = sum_{j in range c} phi(k_j) v_j^T   (D x D, fp32)   -- tcgen05 MMA
+//   dz_c = sum_{j in range c} phi(k_j)          (D, fp32)       -- CUDA cores
+//   S_c  = S_in + sum_{c' < c} dS_c'  (exclusive scan over ranges), same for z
+//
+// Range c holds the tokens [c ct - ov, (c + 1) ct - ov) clipped to [0, L):
+// with softmax chunks that reach ov tokens back into the previous chunk, the
+// state read by chunk c covers exactly the keys before its softmax window,
+// and the last range ends at L, so the total is the state after all L
+// tokens.  ov = 0: ranges are the chunks.
 //
 // The attention part (softmax inside the chunk plus the linear read-out of
 // S_c, z_c) is the HYBRID variant of the attention kernel.
 #pragma once
 #include "common.cuh"
+#include "feature_map.cuh"
 
 namespace vattn {
 namespace hyb {
@@ -21,6 +29,9 @@ struct DeltaParams {
   float* wsz;        // [C][B][H][D]
   uint32_t* status;
   int B, L, H, chunk;
+  int overlap;       // ov: ranges are shifted back by it
+  int fmap;          // fmap::kFmapElu1 or kFmapPoly3
+  const float* coef; // [2][H][4] polynomial coefficients (map 1 = k is used here)
 };
 
 constexpr int kRows = 128;   // tokens per tile
@@ -71,8 +82,8 @@ __global__ void __launch_bounds__(kDeltaThreads, 1)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int h = blockIdx.x, c = blockIdx.y, b = blockIdx.z;   // heads fastest: CTAs running together read whole token rows
-  const int c0 = c * p.chunk;
-  const int c1 = min(p.L, c0 + p.chunk);
+  const int c0 = max(0, c * p.chunk - p.overlap);
+  const int c1 = max(c0, min(p.L, (c + 1) * p.chunk - p.overlap));
   const int nt = (c1 - c0 + kRows - 1) / kRows;
 
   if (threadIdx.x == 0) {
@@ -140,6 +151,7 @@ __global__ void __launch_bounds__(kDeltaThreads, 1)
     float zacc[8];
 #pragma unroll
     for (int e = 0; e < 8; ++e) zacc[e] = 0.f;
+    const fmap::Poly ak = fmap::load_poly(p.coef, 1, p.H, h);
     bool ok = true;
     // No early exit (a failed wait only follows an abort): every thread
     // reaches the reduction barrier below.
@@ -158,8 +170,8 @@ __global__ void __launch_bounds__(kDeltaThreads, 1)
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           float x0 = bf16lo_to_f32(w4[e]), x1 = bf16hi_to_f32(w4[e]);
-          x0 = valid ? (x0 > 0.f ? x0 + 1.f : __expf(x0)) : 0.f;
-          x1 = valid ? (x1 > 0.f ? x1 + 1.f : __expf(x1)) : 0.f;
+          x0 = valid ? fmap::feature(p.fmap, ak, x0) : 0.f;
+          x1 = valid ? fmap::feature(p.fmap, ak, x1) : 0.f;
           w4[e] = pack_bf16x2(x0, x1);
           // z sums the same bf16 values the MMA multiplies
           zacc[2 * e] += bf16lo_to_f32(w4[e]);

@@ -16,6 +16,7 @@
 #include "hybrid.cuh"
 #include "kvcache.cuh"
 #include "merge.cuh"
+#include "feature_map.cuh"
 #include "rope.cuh"
 #include "selftest.cuh"
 
@@ -250,14 +251,20 @@ struct vattn_kvcache {
   // into the rotated ring (host-side record; cleared by restore/enable_rope)
   const void* rotated_k = nullptr;
   int rotated_frame = -1;
+  int sub = 1;              // latent frames (Hg x Wg tokens) per cache frame
+  // positions of the rotated ring: -1 absolute frame index; otherwise the
+  // window start frame of the last window-relative step
+  int rot_base = -1;
 };
 
 namespace {
 size_t frame_bytes(const vattn_kvcache* c) { return static_cast<size_t>(c->B) * c->F * c->Hkv * c->d * 2; }
 
-// Launch the append / rotate pass for one frame.  kr/vr null: rotate only.
+// Launch the append / rotate pass for one frame: rotated K into slot
+// frame % (capacity + 1) of the rotated ring, the frame's first token at
+// RoPE t = t0.  kr/vr null: rotate only.
 vattn_status launch_append_rope(const vattn_kvcache* c, const void* k, const void* v, void* kr, void* vr,
-                                int32_t* ids, int slot, int frame, cudaStream_t stream) {
+                                int32_t* ids, int slot, int frame, int t0, cudaStream_t stream) {
   vattn::rope::RotParams p{};
   p.src = static_cast<const uint4*>(k);
   p.dst = reinterpret_cast<uint4*>(static_cast<uint8_t*>(c->k_rot) +
@@ -269,7 +276,7 @@ vattn_status launch_append_rope(const vattn_kvcache* c, const void* k, const voi
   p.L = c->F;
   p.heads = c->Hkv;
   p.d = c->d;
-  p.frame_offset = frame;
+  p.frame_offset = t0;
   p.Hg = c->rope.Hg;
   p.Wg = c->rope.Wg;
   p.pt = c->rope.pairs_t;
@@ -280,6 +287,31 @@ vattn_status launch_append_rope(const vattn_kvcache* c, const void* k, const voi
   p.frame = frame;
   VATTN_CUDA(kr ? launch_rotate_rows<true>(p, stream) : launch_rotate_rows<false>(p, stream));
   return VATTN_OK;
+}
+
+// Rotate every frame present in the raw ring into the rotated-key ring at
+// its absolute frame index.
+vattn_status rerotate_present(vattn_kvcache* c, cudaStream_t stream) {
+  const size_t bytes = frame_bytes(c);
+  for (int i = 0; i < c->capacity; ++i) {
+    const int fr = c->host_ids[i];
+    if (fr < 0) continue;
+    if (static_cast<long long>(c->sub) * (fr + 1) > c->rope.max_pos)
+      return fail(VATTN_ERR_INVALID_ARG, "frame %d beyond rope max_pos", fr);
+    const uint8_t* kraw = static_cast<const uint8_t*>(c->k_ring) + static_cast<size_t>(i) * bytes;
+    const uint8_t* vraw = static_cast<const uint8_t*>(c->v_ring) + static_cast<size_t>(i) * bytes;
+    if (vattn_status st = launch_append_rope(c, kraw, vraw, nullptr, nullptr, nullptr, 0, fr, c->sub * fr, stream))
+      return st;
+  }
+  c->rot_base = -1;
+  return VATTN_OK;
+}
+
+// Put the rotated ring back at absolute positions after window-relative
+// steps (which leave it rotated relative to their last window).
+vattn_status to_absolute(vattn_kvcache* c, cudaStream_t stream) {
+  if (!c->k_rot || c->rot_base < 0) return VATTN_OK;
+  return rerotate_present(c, stream);
 }
 
 bool same_rope(const vattn_rope& a, const vattn_rope& b) {
@@ -521,8 +553,12 @@ vattn_status vattn_kvcache_append(vattn_kvcache* c, const void* k, const void* v
   c->rotated_k = nullptr;
   c->rotated_frame = -1;
   if (c->k_rot && !rotated) {
-    if (frame_idx >= c->rope.max_pos) return fail(VATTN_ERR_INVALID_ARG, "frame index beyond rope max_pos");
-    if (vattn_status st = launch_append_rope(c, k, v, kr, vr, c->frame_ids, slot, frame_idx, stream)) return st;
+    if (static_cast<long long>(c->sub) * (frame_idx + 1) > c->rope.max_pos)
+      return fail(VATTN_ERR_INVALID_ARG, "frame index beyond rope max_pos");
+    if (vattn_status st = to_absolute(c, stream)) return st;
+    if (vattn_status st = launch_append_rope(c, k, v, kr, vr, c->frame_ids, slot, frame_idx, c->sub * frame_idx,
+                                             stream))
+      return st;
     c->host_ids[slot] = frame_idx;
     return VATTN_OK;
   }
@@ -556,11 +592,16 @@ vattn_status vattn_attention_stream(vattn_kvcache* c, const void* q, const void*
     return fail(VATTN_ERR_INVALID_ARG, "window_back %d outside 0..capacity(%d)", window_back, c->capacity);
   if (!std::isfinite(scale)) return fail(VATTN_ERR_INVALID_ARG, "scale not finite");
   if ((rope == nullptr) != (table == nullptr)) return fail(VATTN_ERR_INVALID_ARG, "rope and table go together");
+  const bool rot_ring = rope && c->k_rot;
   if (rope) {
     if (vattn_status st = check_rope(rope, c->d)) return st;
-    if (static_cast<long long>(rope->Hg) * rope->Wg != c->F)
-      return fail(VATTN_ERR_INVALID_ARG, "rope grid Hg*Wg != frame tokens %d", c->F);
-    if (frame_idx >= rope->max_pos) return fail(VATTN_ERR_INVALID_ARG, "frame index beyond rope max_pos");
+    const long long Fr = static_cast<long long>(rope->Hg) * rope->Wg;
+    // keys rotated in the kernel (no rotated ring) need one latent frame
+    // per cache frame; the rotated ring allows several
+    if (rot_ring ? (c->F % Fr) : (Fr != c->F))
+      return fail(VATTN_ERR_INVALID_ARG, "rope grid Hg*Wg does not fit frame tokens %d", c->F);
+    if ((c->F / Fr) * (static_cast<long long>(frame_idx) + 1) > rope->max_pos)
+      return fail(VATTN_ERR_INVALID_ARG, "frame index beyond rope max_pos");
   }
   vattn::attn::Params p{};
   p.o = static_cast<__nv_bfloat16*>(o);
@@ -575,7 +616,7 @@ vattn_status vattn_attention_stream(vattn_kvcache* c, const void* q, const void*
   p.mode = 0;
   p.F = c->F;
   p.chunk = 1;
-  p.qoff = frame_idx;
+  p.qoff = rot_ring ? c->sub * frame_idx : frame_idx;
   p.q_seg_len = c->F;
   p.q_tiles_per_seg = (c->F + 127) / 128;
   p.n_q_tiles = p.q_tiles_per_seg;
@@ -583,13 +624,14 @@ vattn_status vattn_attention_stream(vattn_kvcache* c, const void* q, const void*
   // Keys come from the rotated-key ring (rotated once per frame) when the
   // cache has one and the call rotates; otherwise from the raw ring, rotated
   // tile by tile in the kernel when rope is given.
-  const bool rot_ring = rope && c->k_rot;
   if (rot_ring) {
     if (!same_rope(*rope, c->rope) || table != c->table)
       return fail(VATTN_ERR_INVALID_ARG, "rope/table differ from those given to vattn_kvcache_enable_rope");
+    if (vattn_status st = to_absolute(c, stream)) return st;
     // the current frame's rotated keys: slot frame_idx % (capacity + 1),
     // which holds a frame outside the window
-    if (vattn_status st = launch_append_rope(c, k_cur, v_cur, nullptr, nullptr, nullptr, 0, frame_idx, stream))
+    if (vattn_status st = launch_append_rope(c, k_cur, v_cur, nullptr, nullptr, nullptr, 0, frame_idx,
+                                             c->sub * frame_idx, stream))
       return st;
     c->rotated_k = k_cur;
     c->rotated_frame = frame_idx;
@@ -629,21 +671,7 @@ vattn_status vattn_kvcache_frame_ids(const vattn_kvcache* c, int32_t* host_ids) 
   return VATTN_OK;
 }
 
-namespace {
-// Rotate every frame present in the raw ring into the rotated-key ring.
-vattn_status rerotate_present(vattn_kvcache* c, cudaStream_t stream) {
-  const size_t bytes = frame_bytes(c);
-  for (int i = 0; i < c->capacity; ++i) {
-    const int fr = c->host_ids[i];
-    if (fr < 0) continue;
-    if (fr >= c->rope.max_pos) return fail(VATTN_ERR_INVALID_ARG, "frame %d beyond rope max_pos", fr);
-    const uint8_t* kraw = static_cast<const uint8_t*>(c->k_ring) + static_cast<size_t>(i) * bytes;
-    const uint8_t* vraw = static_cast<const uint8_t*>(c->v_ring) + static_cast<size_t>(i) * bytes;
-    if (vattn_status st = launch_append_rope(c, kraw, vraw, nullptr, nullptr, nullptr, 0, fr, stream)) return st;
-  }
-  return VATTN_OK;
-}
-}  // namespace
+
 
 vattn_status vattn_kvcache_restore(vattn_kvcache* c, const int32_t* host_ids, vattn_stream stream) {
   if (!c || !host_ids) return fail(VATTN_ERR_INVALID_ARG, "NULL pointer");
@@ -662,13 +690,14 @@ vattn_status vattn_kvcache_enable_rope(vattn_kvcache* c, void* k_ring_rot, const
   if (!c || !k_ring_rot || !table) return fail(VATTN_ERR_INVALID_ARG, "NULL pointer");
   if (!aligned16(k_ring_rot)) return fail(VATTN_ERR_INVALID_ARG, "k_ring_rot must be 16-byte aligned");
   if (vattn_status st = check_rope(rope, c->d)) return st;
-  if (static_cast<long long>(rope->Hg) * rope->Wg != c->F)
-    return fail(VATTN_ERR_INVALID_ARG, "rope grid Hg*Wg != frame tokens %d", c->F);
+  const long long Fr = static_cast<long long>(rope->Hg) * rope->Wg;
+  if (c->F % Fr) return fail(VATTN_ERR_INVALID_ARG, "frame tokens %d not a multiple of Hg*Wg=%lld", c->F, Fr);
   if (static_cast<long long>(c->capacity + 1) * c->B > 65535)
     return fail(VATTN_ERR_UNSUPPORTED, "(capacity+1)*B too large");
   CUtensorMap m;
   if (vattn_status st = make_map(&m, k_ring_rot, c->d, c->Hkv, c->F, (c->capacity + 1) * c->B, 128)) return st;
   c->k_rot = k_ring_rot;
+  c->sub = static_cast<int>(c->F / Fr);
   c->rope = *rope;
   c->table = table;
   c->map_krot = m;
@@ -679,6 +708,233 @@ vattn_status vattn_kvcache_enable_rope(vattn_kvcache* c, void* k_ring_rot, const
 
 vattn_status vattn_kvcache_destroy(vattn_kvcache* c) {
   delete c;
+  return VATTN_OK;
+}
+
+}  // extern "C"
+
+// ------------------------------------------------- fused streaming step
+namespace {
+int sm_count() {
+  int sms = 148, dev;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  return sms;
+}
+
+// Key splits for `items` (pair, head, batch) work units of n_tiles key tiles
+// each on `sms` SMs (one CTA per SM): the count minimising
+//   waves * (tiles per split + 1.5 + merge) + merge,
+// where 1.5 tiles stand for a CTA's prologue and epilogue and a split's
+// partial write and merge read cost about 0.1 tile each.  Counts that would
+// leave a split empty are skipped.
+int choose_splits(long long items, int n_tiles, int sms) {
+  double best = 1e300;
+  int best_s = 1;
+  for (int s = 1; s <= vattn::attn::kMaxSplit && s <= n_tiles; ++s) {
+    const int per = (n_tiles + s - 1) / s;
+    if ((n_tiles + per - 1) / per != s) continue;
+    const double waves = std::ceil(static_cast<double>(items) * s / sms);
+    const double cost = waves * (per + 1.5 + (s > 1 ? 0.1 : 0.0)) + (s > 1 ? 0.1 * s : 0.0);
+    if (cost < best - 1e-9) {
+      best = cost;
+      best_s = s;
+    }
+  }
+  return best_s;
+}
+
+struct StepLayout {
+  int pairs, per_tiles, n_split_max;
+  size_t off_count, off_lse, off_o, bytes;
+};
+
+// Workspace of vattn_kvcache_step: [0, 256) the step counters; then the
+// pairs' arrival counters; then split partials (lse, o) for the largest
+// split count any frame of this window can use.
+StepLayout step_layout(const vattn_kvcache* c, int H, int window_back) {
+  StepLayout L{};
+  const int qt = (c->F + 127) / 128;
+  L.pairs = (qt + 1) / 2;
+  L.per_tiles = (c->F + 127) / 128;
+  const int sms = sm_count();
+  const long long items = static_cast<long long>(L.pairs) * H * c->B;
+  L.n_split_max = 1;
+  for (int nseg = 1; nseg <= window_back + 1; ++nseg) {
+    const int s = choose_splits(items, nseg * L.per_tiles, sms);
+    if (s > L.n_split_max) L.n_split_max = s;
+  }
+  auto up = [](size_t x) { return (x + 255) & ~static_cast<size_t>(255); };
+  L.off_count = 256;
+  L.off_lse = L.off_count + up(static_cast<size_t>(c->B) * H * L.pairs * 4);
+  const size_t rows = static_cast<size_t>(c->B) * H * c->F;
+  L.off_o = L.off_lse + (L.n_split_max > 1 ? up(L.n_split_max * rows * 4) : 0);
+  L.bytes = L.off_o + (L.n_split_max > 1 ? L.n_split_max * rows * c->d * 4 : 0);
+  return L;
+}
+
+uint64_t g_step_smem_done[4][1];
+
+template <int D, int ROPE>
+vattn_status launch_step(const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v, const CUtensorMap& k2,
+                         const CUtensorMap& v2, const vattn::attn::Params& p, cudaStream_t s) {
+  using Cfg = vattn::attn::PairCfg<D>;
+  auto kern = vattn::attn::attn_pair_kernel<D, ROPE, false>;
+  vattn_status st = ensure_smem(kern, Cfg::kSmemBytes,
+                                g_step_smem_done[(D == 64 ? 0 : 2) + (ROPE == vattn::attn::kRopeQ ? 1 : 0)]);
+  if (st) return st;
+  kern<<<p.total_ctas, vattn::attn::kPairThreads, Cfg::kSmemBytes, s>>>(q, k, v, k2, v2, p);
+  VATTN_CUDA(cudaGetLastError());
+  return VATTN_OK;
+}
+}  // namespace
+
+extern "C" {
+
+size_t vattn_kvcache_step_workspace_bytes(const vattn_kvcache* c, int H, int window_back) {
+  if (!c || H < 1 || window_back < 0 || window_back >= c->capacity) return 0;
+  return step_layout(c, H, window_back).bytes;
+}
+
+vattn_status vattn_kvcache_step(vattn_kvcache* c, const void* q, const void* k_cur, const void* v_cur, void* o,
+                                float* lse, int H, int frame_idx, int window_back, float scale,
+                                const vattn_rope* rope, const float* table, int window_relative, void* workspace,
+                                size_t workspace_bytes, vattn_stream stream) {
+  if (!c || !q || !k_cur || !v_cur || !o || !workspace) return fail(VATTN_ERR_INVALID_ARG, "NULL pointer");
+  if (!aligned16(q) || !aligned16(k_cur) || !aligned16(v_cur) || !aligned16(o) || !aligned16(workspace))
+    return fail(VATTN_ERR_INVALID_ARG, "tensors and workspace must be 16-byte aligned");
+  if (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)) return fail(VATTN_ERR_INVALID_ARG, "lse misaligned");
+  if (H < 1 || H % c->Hkv) return fail(VATTN_ERR_INVALID_ARG, "H=%d vs Hkv=%d", H, c->Hkv);
+  if (frame_idx < 0) return fail(VATTN_ERR_INVALID_ARG, "frame_idx < 0");
+  if (window_back < 0 || window_back >= c->capacity)
+    return fail(VATTN_ERR_INVALID_ARG,
+                "window_back %d: the step appends into slot frame %% capacity, so capacity (%d) must exceed it",
+                window_back, c->capacity);
+  if (!std::isfinite(scale)) return fail(VATTN_ERR_INVALID_ARG, "scale not finite");
+  if ((rope == nullptr) != (table == nullptr)) return fail(VATTN_ERR_INVALID_ARG, "rope and table go together");
+  if (rope && !c->k_rot)
+    return fail(VATTN_ERR_INVALID_ARG, "a step with RoPE needs the rotated-key ring (vattn_kvcache_enable_rope)");
+  if (rope && (!same_rope(*rope, c->rope) || table != c->table))
+    return fail(VATTN_ERR_INVALID_ARG, "rope/table differ from those given to vattn_kvcache_enable_rope");
+  if (window_relative && !rope) return fail(VATTN_ERR_INVALID_ARG, "window_relative needs rope");
+  const StepLayout Ly = step_layout(c, H, window_back);
+  if (workspace_bytes < Ly.bytes)
+    return fail(VATTN_ERR_INVALID_ARG, "workspace %zu bytes < %zu required", workspace_bytes, Ly.bytes);
+  const int cap = c->capacity, rcap = cap + 1, sub = c->sub;
+  const int base = window_relative ? std::max(0, frame_idx - window_back) : 0;
+  if (rope && static_cast<long long>(sub) * (frame_idx - base + 1) > rope->max_pos)
+    return fail(VATTN_ERR_INVALID_ARG, "frame position beyond rope max_pos");
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+
+  // the window's earlier frames present in the ring
+  std::vector<int> past;
+  for (int fr = frame_idx - window_back; fr < frame_idx; ++fr)
+    if (fr >= 0 && c->host_ids[fr % cap] == fr) past.push_back(fr);
+
+  // positions of the rotated ring for this step
+  if (rope) {
+    if (window_relative) {
+      // every earlier frame of the window again, relative to its start
+      const size_t bytes = frame_bytes(c);
+      for (int fr : past) {
+        const uint8_t* kraw = static_cast<const uint8_t*>(c->k_ring) + static_cast<size_t>(fr % cap) * bytes;
+        if (vattn_status st = launch_append_rope(c, kraw, nullptr, nullptr, nullptr, nullptr, 0, fr,
+                                                 sub * (fr - base), stream))
+          return st;
+      }
+      c->rot_base = base;
+    } else if (vattn_status st = to_absolute(c, stream)) {
+      return st;
+    }
+  }
+
+  vattn::attn::Params p{};
+  p.o = static_cast<__nv_bfloat16*>(o);
+  p.lse = lse;
+  if (vattn_status st = status_ptr(&p.status)) return st;
+  p.B = c->B;
+  p.Lq = c->F;
+  p.Lk = c->F;
+  p.H = H;
+  p.Hkv = c->Hkv;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.mode = 0;
+  p.F = c->F;
+  p.chunk = 1;
+  p.qoff = sub * (frame_idx - base);
+  p.q_seg_len = c->F;
+  p.q_tiles_per_seg = (c->F + 127) / 128;
+  p.n_q_tiles = p.q_tiles_per_seg;
+  const int per = Ly.per_tiles;
+  int n = 0, tiles = 0;
+  for (int fr : past) {
+    const int kc3 = rope ? (fr % rcap) * c->B : (fr % cap) * c->B;
+    p.kseg[n++] = vattn::attn::KeySegment{0, kc3, 0, (fr % cap) * c->B, 0, c->F, fr, tiles};
+    tiles += per;
+  }
+  const int cur_tile = tiles;
+  if (rope)   // the current frame's keys: rotated into its spare-ring slot by this launch
+    p.kseg[n++] = vattn::attn::KeySegment{0, (frame_idx % rcap) * c->B, 1, 0, 0, c->F, frame_idx, tiles};
+  else
+    p.kseg[n++] = vattn::attn::KeySegment{1, 0, 1, 0, 0, c->F, frame_idx, tiles};
+  tiles += per;
+  p.n_kseg = n;
+  fill_rope_params(p, rope, table);
+
+  // the append: raw K and V into slot frame % capacity (outside the window),
+  // K rotated into the rotated ring, by the launch's first CTAs; attention
+  // CTAs wait for them only before the current frame's rotated keys.  When
+  // the window holds no earlier frame every CTA would wait at once: then
+  // the append runs as its own launch first.
+  const size_t fb = frame_bytes(c);
+  const int slot = frame_idx % cap;
+  uint8_t* kr = static_cast<uint8_t*>(c->k_ring) + static_cast<size_t>(slot) * fb;
+  uint8_t* vr = static_cast<uint8_t*>(c->v_ring) + static_cast<size_t>(slot) * fb;
+  uint8_t* krot = rope ? static_cast<uint8_t*>(c->k_rot) + static_cast<size_t>(frame_idx % rcap) * fb : nullptr;
+  const int t0 = sub * (frame_idx - base);
+  const bool fold = !rope || cur_tile > 0;
+  if (!fold) {
+    if (vattn_status st = launch_append_rope(c, k_cur, v_cur, kr, vr, c->frame_ids, slot, frame_idx, t0, stream))
+      return st;
+  }
+  const long long chunks = static_cast<long long>(c->B) * c->F * c->Hkv * (c->d / 8);
+  p.n_append = fold ? static_cast<int>(std::min<long long>(16, (chunks + 384 * 4 - 1) / (384 * 4))) : 0;
+  p.app = vattn::attn::AppendWork{static_cast<const uint4*>(k_cur), static_cast<const uint4*>(v_cur),
+                                  reinterpret_cast<uint4*>(kr), reinterpret_cast<uint4*>(vr),
+                                  reinterpret_cast<uint4*>(krot), c->frame_ids, slot, frame_idx,
+                                  static_cast<long long>(c->B) * c->F, c->F, t0};
+  p.wait_tile = (fold && rope) ? cur_tile : -1;
+  // key splits
+  const long long items = static_cast<long long>(Ly.pairs) * H * c->B;
+  p.n_split = choose_splits(items, tiles, sm_count());
+  if (p.n_split > Ly.n_split_max) p.n_split = Ly.n_split_max;
+  p.split_tiles = (tiles + p.n_split - 1) / p.n_split;
+  p.n_split = (tiles + p.split_tiles - 1) / p.split_tiles;
+  p.pair_count = reinterpret_cast<uint32_t*>(ws + Ly.off_count);
+  p.part_lse = reinterpret_cast<float*>(ws + Ly.off_lse);
+  p.part_o = reinterpret_cast<float*>(ws + Ly.off_o);
+  p.step_sync = reinterpret_cast<uint32_t*>(ws);
+  p.linear_grid = 1;
+  p.n_pairs = Ly.pairs;
+  const long long total = p.n_append + items * p.n_split;
+  if (total > 0x7fffffffLL) return fail(VATTN_ERR_UNSUPPORTED, "grid too large");
+  p.total_ctas = static_cast<int>(total);
+
+  CUtensorMap mq, mk2, mv2;
+  if (vattn_status st = make_map(&mq, q, c->d, H, c->F, c->B, 128)) return st;
+  if (vattn_status st = make_map(&mk2, k_cur, c->d, c->Hkv, c->F, c->B, 128)) return st;
+  if (vattn_status st = make_map(&mv2, v_cur, c->d, c->Hkv, c->F, c->B, 128)) return st;
+  const CUtensorMap& mk = rope ? c->map_krot : c->map_k;
+  vattn_status st;
+  if (c->d == 64)
+    st = rope ? launch_step<64, vattn::attn::kRopeQ>(mq, mk, c->map_v, mk2, mv2, p, stream)
+              : launch_step<64, vattn::attn::kRopeNone>(mq, mk, c->map_v, mk2, mv2, p, stream);
+  else
+    st = rope ? launch_step<128, vattn::attn::kRopeQ>(mq, mk, c->map_v, mk2, mv2, p, stream)
+              : launch_step<128, vattn::attn::kRopeNone>(mq, mk, c->map_v, mk2, mv2, p, stream);
+  if (st) return st;
+  c->host_ids[slot] = frame_idx;
+  c->rotated_k = nullptr;
+  c->rotated_frame = -1;
   return VATTN_OK;
 }
 
@@ -708,14 +964,15 @@ vattn_status check_hybrid(int B, int L, int H, int d, int chunk_tokens, const vo
   return VATTN_OK;
 }
 
-// Launch 1 of the hybrid call: per-chunk state deltas into the workspace.
+// Launch 1 of the hybrid call: per-range state deltas into the workspace.
 vattn_status launch_delta(const CUtensorMap& mk, const CUtensorMap& mv, float* wsS, float* wsz, uint32_t* status,
-                          int B, int L, int H, int C, int chunk_tokens, cudaStream_t stream) {
+                          int B, int L, int H, int C, int chunk_tokens, cudaStream_t stream, int overlap = 0,
+                          int fmap = vattn::fmap::kFmapElu1, const float* coef = nullptr) {
   static uint64_t done[1];
   auto kern = vattn::hyb::delta_kernel<128>;
   const int smem = vattn::hyb::DeltaCfg<128>::kSmemBytes;
   if (vattn_status st = ensure_smem(kern, smem, done)) return st;
-  vattn::hyb::DeltaParams dp{wsS, wsz, status, B, L, H, chunk_tokens};
+  vattn::hyb::DeltaParams dp{wsS, wsz, status, B, L, H, chunk_tokens, overlap, fmap, coef};
   kern<<<dim3(H, C, B), vattn::hyb::kDeltaThreads, smem, stream>>>(mk, mv, dp);
   VATTN_CUDA(cudaGetLastError());
   return VATTN_OK;
@@ -766,17 +1023,34 @@ vattn_status vattn_hybrid_scan(float* S, float* z, int B, int L, int H, int d, i
   return launch_scan(wsS, wsz, S, z, B, H, d, C, stream);
 }
 
-vattn_status vattn_hybrid_chunk(const void* q, const void* k, const void* v, void* o, float* S, float* z, int B,
-                                int L, int H, int d, int chunk_tokens, float scale, void* workspace,
-                                size_t workspace_bytes, vattn_stream stream) {
+size_t vattn_hybrid_workspace_bytes_ex(int B, int L, int H, int d, int chunk_tokens, int overlap_tokens) {
+  if (overlap_tokens < 0) return 0;
+  return vattn_hybrid_workspace_bytes(B, L + overlap_tokens, H, d, chunk_tokens);
+}
+
+}  // extern "C"
+
+namespace {
+// The three launches of a hybrid call.  With overlap ov the state deltas
+// cover the ranges [c ct - ov, (c + 1) ct - ov) (R = ceil((L + ov) / ct)
+// of them) and each query chunk's softmax window starts ov tokens early.
+vattn_status hybrid_impl(const void* q, const void* k, const void* v, void* o, float* S, float* z, int B, int L,
+                         int H, int d, int chunk_tokens, int overlap, float scale, int fmap, const float* coef,
+                         void* workspace, size_t workspace_bytes, cudaStream_t stream) {
   if (!q || !k || !v || !o || !S || !z) return fail(VATTN_ERR_INVALID_ARG, "NULL pointer");
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(S) || !aligned16(z))
     return fail(VATTN_ERR_INVALID_ARG, "pointers must be 16-byte aligned");
   if (!std::isfinite(scale)) return fail(VATTN_ERR_INVALID_ARG, "scale not finite");
-  int C;
+  if (overlap < 0 || overlap > (1 << 30) - L) return fail(VATTN_ERR_INVALID_ARG, "overlap %d", overlap);
+  if (fmap != vattn::fmap::kFmapElu1 && fmap != vattn::fmap::kFmapPoly3)
+    return fail(VATTN_ERR_INVALID_ARG, "feature map %d", fmap);
+  if (fmap == vattn::fmap::kFmapPoly3 && (!coef || !aligned16(coef)))
+    return fail(VATTN_ERR_INVALID_ARG, "the polynomial feature map needs 16-byte aligned coefficients");
+  int C, R;
   if (vattn_status st = check_hybrid(B, L, H, d, chunk_tokens, workspace, workspace_bytes, &C)) return st;
+  if (vattn_status st = check_hybrid(B, L + overlap, H, d, chunk_tokens, workspace, workspace_bytes, &R)) return st;
   float* wsS = static_cast<float*>(workspace);
-  float* wsz = wsS + static_cast<size_t>(C) * B * H * d * d;
+  float* wsz = wsS + static_cast<size_t>(R) * B * H * d * d;
   uint32_t* status;
   if (vattn_status st = status_ptr(&status)) return st;
 
@@ -785,9 +1059,11 @@ vattn_status vattn_hybrid_chunk(const void* q, const void* k, const void* v, voi
   if (vattn_status st = make_map(&mk, k, d, H, L, B, 128)) return st;
   if (vattn_status st = make_map(&mv, v, d, H, L, B, 128)) return st;
 
-  // (1) per-chunk state deltas, (2) exclusive scan over chunks (+ state out)
-  if (vattn_status st = launch_delta(mk, mv, wsS, wsz, status, B, L, H, C, chunk_tokens, stream)) return st;
-  if (vattn_status st = launch_scan(wsS, wsz, S, z, B, H, d, C, stream)) return st;
+  // (1) per-range state deltas, (2) exclusive scan over ranges (+ state out)
+  if (vattn_status st = launch_delta(mk, mv, wsS, wsz, status, B, L, H, R, chunk_tokens, stream, overlap, fmap,
+                                     coef))
+    return st;
+  if (vattn_status st = launch_scan(wsS, wsz, S, z, B, H, d, R, stream)) return st;
   // (3) attention with linear-state initialisation
   vattn::attn::Params p{};
   p.o = static_cast<__nv_bfloat16*>(o);
@@ -809,7 +1085,28 @@ vattn_status vattn_hybrid_chunk(const void* q, const void* k, const void* v, voi
   p.n_q_tiles = C * p.q_tiles_per_seg;
   p.hyb_S = wsS;
   p.hyb_z = wsz;
+  p.hyb_fmap = fmap;
+  p.hyb_coef = coef;
+  p.lead = overlap;
   return launch_pair<128, vattn::attn::kRopeNone, true>(mq, mk, mv, mk, mv, p, stream);
+}
+}  // namespace
+
+extern "C" {
+
+vattn_status vattn_hybrid_chunk(const void* q, const void* k, const void* v, void* o, float* S, float* z, int B,
+                                int L, int H, int d, int chunk_tokens, float scale, void* workspace,
+                                size_t workspace_bytes, vattn_stream stream) {
+  return hybrid_impl(q, k, v, o, S, z, B, L, H, d, chunk_tokens, 0, scale, vattn::fmap::kFmapElu1, nullptr,
+                     workspace, workspace_bytes, stream);
+}
+
+vattn_status vattn_hybrid_chunk_ex(const void* q, const void* k, const void* v, void* o, float* S, float* z, int B,
+                                   int L, int H, int d, int chunk_tokens, int overlap_tokens, float scale,
+                                   vattn_feature_map fmap, const float* coef, void* workspace,
+                                   size_t workspace_bytes, vattn_stream stream) {
+  return hybrid_impl(q, k, v, o, S, z, B, L, H, d, chunk_tokens, overlap_tokens, scale, static_cast<int>(fmap),
+                     coef, workspace, workspace_bytes, stream);
 }
 
 // ------------------------------------------------- hybrid without workspace
