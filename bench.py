@@ -559,12 +559,22 @@ def stream_step_figure(va, torch, device, frames, c, pk, window_relative):
 
     m = _measure(torch, run)
     va.vattn_check()
+    # the same T steps captured once in a CUDA graph and replayed (the
+    # per-frame work is fixed, FlashDecoder "Inference Optimization", Sec.
+    # 4.6): no host work between the launches
+    g = _graph(torch, [run])
+    mg = _measure(torch, g.replay)
+    del g
+    va.vattn_check()
     cache.close()
     pairs = sum(min(f, wb) + 1 for f in range(T))
     flops = 4.0 * d * F * F * H * pairs
     tf = flops / m["median_ms"] * 1e-9
     fps = T / (m["median_ms"] / 1e3)
     ceiling = T / (flops / (pk["bf16_tflops"] * 1e12))
+    fps_g = T / (mg["median_ms"] / 1e3)
+    m["graph"] = dict(mg, frames_per_s=fps_g, latent_frames_per_s=fps_g * sub, ms_per_frame=mg["median_ms"] / T,
+                      tflops=flops / mg["median_ms"] * 1e-9, frac_of_ceiling=fps_g / ceiling)
     return dict(m, frames_per_s=fps, latent_frames_per_s=fps * sub, ms_per_frame=m["median_ms"] / T, tflops=tf,
                 frac_of_ceiling=fps / ceiling, ceiling_frames_per_s=ceiling, launches_per_frame=1,
                 workload="%d steps of %d tokens (%d latent frames of %dx%d), H=%d on %d KV heads, d=%d, "

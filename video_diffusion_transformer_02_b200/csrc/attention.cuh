@@ -99,6 +99,7 @@ struct Params {
   int reverse_q;            // heaviest tiles first (chunk-causal)
   int n_kseg;               // 0: contiguous keys with the mode's masks
   KeySegment kseg[kMaxKeySegments];
+  int seg_tok;              // segment mode: every segment holds this many tokens (0: lengths differ)
   // RoPE
   const float2* rope_tab;   // [max_pos][D/2] (cos, sin)
   int rope_Hg, rope_Wg, rope_pt, rope_ph, rope_maxpos;

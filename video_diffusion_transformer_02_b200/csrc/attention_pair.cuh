@@ -43,12 +43,21 @@ struct PairCfg {
   static constexpr int kOffK = 2 * kTileBytes;
   static constexpr int kOffV = kOffK + kStages * kTileBytes;
   static constexpr int kOffBar = kOffV + kStages * kTileBytes;
-  static constexpr int kNumBars = 4 + 4 * kStages + 12 + 2 + 5;
+  static constexpr int kNumBars = 4 + 4 * kStages + 12 + 2 + 5 + 2 + 3;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
-  static constexpr int kSmemBytes = kOffMisc + 64;
+  static constexpr int kOffZ = kOffMisc + 64;        // hybrid: z_c, fp32 [D]
+  static constexpr int kSmemBytes = kOffZ + D * 4;
 };
 
 constexpr int kPairThreads = 384;
+// The two softmax warpgroups take turns on their exponential phases at head
+// dim 64, where the exponentials outweigh the tensor-core work per score
+// (measured: +4 % on the 16-head stream); at head dim 128 the turns cost
+// 3 % and are off.
+template <int D>
+struct TakeTurns {
+  static constexpr bool value = D == 64;
+};
 
 // Rows of the two query tiles of pair `pr` and the key tiles they need
 // (the union of both tiles' visible ranges; rows mask what they do not see).
@@ -129,13 +138,13 @@ __device__ __forceinline__ void append_share(const Params& p, int part) {
         const int n = static_cast<int>((i / cpr) % a.F);   // token of the frame
         const int c16 = static_cast<int>(i % D8);          // chunk of the head vector
         const int in = n % Fr;
-        const int pos[3] = {a.t0 + n / Fr, in / p.rope_Wg, in % p.rope_Wg};
+        const int pt_t = a.t0 + n / Fr, pt_h = in / p.rope_Wg, pt_w = in % p.rope_Wg;
         uint32_t w4[4] = {kv[u].x, kv[u].y, kv[u].z, kv[u].w};
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           const int j = c16 * 4 + e;
-          const int ax = j < pt ? 0 : (j < pth ? 1 : 2);
-          const float2 cs = __ldg(p.rope_tab + pos[ax] * (D / 2) + j);
+          const int pos = j < pt ? pt_t : (j < pth ? pt_h : pt_w);
+          const float2 cs = __ldg(p.rope_tab + pos * (D / 2) + j);
           const float x0 = bf16lo_to_f32(w4[e]), x1 = bf16hi_to_f32(w4[e]);
           w4[e] = pack_bf16x2(x0 * cs.x - x1 * cs.y, x0 * cs.y + x1 * cs.x);
         }
@@ -246,7 +255,8 @@ template <int D, int ROPE, bool HYB>
 __global__ void __launch_bounds__(kPairThreads, 1)
     attn_pair_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                      const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmK2,
-                     const __grid_constant__ CUtensorMap tmV2, const Params p) {
+                     const __grid_constant__ CUtensorMap tmV2, const __grid_constant__ CUtensorMap tmO,
+                     const Params p) {
   static_assert(ROPE == kRopeNone || ROPE == kRopeQ, "keys are rotated before this kernel");
   static_assert(!HYB || (D == 128 && ROPE == kRopeNone), "hybrid: head dim 128, no RoPE");
   using C = PairCfg<D>;
@@ -302,6 +312,14 @@ __global__ void __launch_bounds__(kPairThreads, 1)
   auto bPhiReady = [&](int x) { return bx + 112 + 8 * x; };
   const uint32_t bScReady = bx + 128;
   auto bLinDone = [&](int x) { return bx + 136 + 8 * x; };
+  // exponential phases of the two softmax warpgroups take turns: tile A's
+  // phase for sub-tile u waits on bTurnA (tile B done with u - 1), tile B's
+  // on bTurnB (tile A done with u)
+  const uint32_t bTurnA = bx + 152, bTurnB = bx + 160;
+  // hybrid: each tile's last Q K^T complete (Q_x and, with both, the K
+  // stages free); z_c landed in shared memory
+  auto bQKDone = [&](int x) { return bx + 168 + 8 * x; };
+  const uint32_t bZFull = bx + 184;
   uint32_t* misc = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
   volatile uint32_t* tmem_slot = misc;
   volatile uint32_t* abort_flag = misc + 1;
@@ -340,9 +358,14 @@ __global__ void __launch_bounds__(kPairThreads, 1)
     mbar_init(bFinal(1), 1);
     mbar_init(bPhiReady(0), 4);
     mbar_init(bPhiReady(1), 4);
-    mbar_init(bScReady, hasB ? 8 : 4);
+    mbar_init(bScReady, 4);
+    mbar_init(bQKDone(0), 1);
+    mbar_init(bQKDone(1), 1);
+    mbar_init(bZFull, 1);
     mbar_init(bLinDone(0), 1);
     mbar_init(bLinDone(1), 1);
+    mbar_init(bTurnA, 4);
+    mbar_init(bTurnB, 4);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -400,6 +423,12 @@ __global__ void __launch_bounds__(kPairThreads, 1)
   } else if (warp == 2) {
     // ----------------------------------------------------- producer: V
     if (lane == 0) {
+      if constexpr (HYB) {
+        // z_c (the pair's chunk state, 512 bytes) for the read-out, now
+        const int c = g.q0[0] / p.q_seg_len;
+        mbar_arrive_expect_tx(bZFull, D * 4);
+        bulk_load(sbase + C::kOffZ, p.hyb_z + ((static_cast<size_t>(c) * p.B + b) * p.H + h) * D, D * 4, bZFull);
+      }
       int j = 0;
       for (; j < nk; ++j) {
         const int s = j % NS;
@@ -415,6 +444,7 @@ __global__ void __launch_bounds__(kPairThreads, 1)
       for (int i = max(0, j - NS); i < j; ++i) {
         mbar_drain(bVFull(i % NS), (i / NS) & 1, ab.limit_ns);
       }
+      if constexpr (HYB) mbar_drain(bZFull, 0, ab.limit_ns);
     }
   } else if (warp == 1 || warp == 3) {
     // ------------------------------------------------------------- MMA
@@ -466,6 +496,7 @@ __global__ void __launch_bounds__(kPairThreads, 1)
         if (ok) {
           tc_fence_after();
           issue_qk(0);
+          if (HYB && ns == 1) umma_commit(bQKDone(x));
         }
       }
       // per sub-tile u: S_x(u + 1) into the buffer that P_x(u - 1) V released,
@@ -481,6 +512,7 @@ __global__ void __launch_bounds__(kPairThreads, 1)
           if (u > 0 && !mbar_wait(bPvDone(x), (u - 1) & 1, ab, kStatusTimeoutMma)) break;
           tc_fence_after();
           issue_qk(un);
+          if (HYB && un == ns - 1) umma_commit(bQKDone(x));
           if (un & 1) umma_commit(bKEmpty(stn));   // both sub-tiles of the stage issued
         }
         const int st = (u >> 1) & (NS - 1);
@@ -527,6 +559,7 @@ __global__ void __launch_bounds__(kPairThreads, 1)
       const int q_end = x ? g.q_end[1] : g.q_end[0];
       const int qn = (x ? g.q0[1] : g.q0[0]) + r;
       const bool row_valid = qn < q_end;
+      const bool full_tile = q_end - (x ? g.q0[1] : g.q0[0]) == kTileM;   // uniform in the warpgroup
       int lo = 0, hi = 0;
       if (p.n_kseg == 0) key_range(p, row_valid ? qn : q_end - 1, lo, hi);
       float m_run = -INFINITY, l_run = 0.f;
@@ -547,6 +580,10 @@ __global__ void __launch_bounds__(kPairThreads, 1)
         __syncwarp();
         if (lane == 0) mbar_arrive(bQReady(x));
       }
+      // segment mode with equal segments: the valid keys of each tile follow
+      // from the tile's index inside its segment, kept as a running count
+      const int seg_tiles = p.seg_tok > 0 ? (p.seg_tok + kTileN - 1) / kTileN : 1;
+      int seg_t = p.seg_tok > 0 ? g.t0 % seg_tiles : 0;
       // No early exit: a failed wait only happens after the CTA aborted,
       // when every later wait fails at once; the warp stays converged for
       // the warp-collective TMEM accesses.
@@ -560,6 +597,9 @@ __global__ void __launch_bounds__(kPairThreads, 1)
           const int k0 = g.tg.kbeg + u * kSub;
           col_lo = lo - k0;
           col_hi = hi - k0;
+        } else if (p.seg_tok > 0) {
+          col_hi = min(kTileN, p.seg_tok - seg_t * kTileN) - bb * kSub;
+          if (bb && ++seg_t == seg_tiles) seg_t = 0;
         } else {
           col_hi = key_tile(p, g.tg, g.t0 + (u >> 1)).valid - bb * kSub;
         }
@@ -596,6 +636,15 @@ __global__ void __launch_bounds__(kPairThreads, 1)
           resc = true;
         }
         const float nm = (m_run == -INFINITY) ? 0.f : -m_run;
+        // turns: the MUFU serves one warpgroup's exponentials at a time
+        // while the other loads, reduces and publishes
+        if (TakeTurns<D>::value && hasB) {
+          if (x == 0) {
+            if (u > 0 && !mbar_wait(bTurnA, (u - 1) & 1, ab, kStatusTimeoutSoftmax)) ok = false;
+          } else if (!mbar_wait(bTurnB, u & 1, ab, kStatusTimeoutSoftmax)) {
+            ok = false;
+          }
+        }
         // P = exp2(s * scale * log2e - m) into the first half of the S
         // buffer, 16 columns (32 keys) at a time; row sums as packed fp32x2
         float rs2[2][2] = {{0.f, 0.f}, {0.f, 0.f}};
@@ -632,6 +681,10 @@ __global__ void __launch_bounds__(kPairThreads, 1)
           }
           tmem_st16(tS + q * 16, pk);
         }
+        if (TakeTurns<D>::value && hasB) {
+          __syncwarp();
+          if (lane == 0 && (x == 0 || u + 1 < ns)) mbar_arrive(x == 0 ? bTurnB : bTurnA);
+        }
         const float rs = (rs2[0][0] + rs2[0][1]) + (rs2[1][0] + rs2[1][1]);
         // O_x rescale: wait until the P V of the previous sub-tile (which
         // accumulates into O_x) has completed; the next one waits for P below
@@ -663,25 +716,24 @@ __global__ void __launch_bounds__(kPairThreads, 1)
       }
       float dl = 0.f;   // hybrid: phi(q_r) . z_c
       if constexpr (HYB) {
-        // the Q tiles and the K / V stages are free once both tiles' last
-        // P V (and so every MMA reading them) has completed
-        bool okh = ok && ns > 0 && mbar_wait(bODone(0), 0, ab, kStatusTimeoutSoftmax) &&
-                   (!hasB || mbar_wait(bODone(1), 0, ab, kStatusTimeoutSoftmax));
-        tc_fence_after();
+        // Q_x is free as soon as this tile's last scores are in: every MMA
+        // reading it has completed.  z_c was copied into shared memory at
+        // the start.
+        bool okh = ok && mbar_wait(bZFull, 0, ab, kStatusTimeoutSoftmax);
         const int c = g.q0[0] / p.q_seg_len;   // the pair's chunk
         // phi(q_r) in place of row r of Q_x (bf16), and phi(q_r) . z_c in fp32
-        const float* zc = p.hyb_z + ((static_cast<size_t>(c) * p.B + b) * p.H + h) * D;
         const fmap::Poly aq = fmap::load_poly(p.hyb_coef, 0, p.H, h);
         const uint32_t qrow = sQ + static_cast<uint32_t>(x * C::kTileBytes);
+        const uint32_t sz = sbase + C::kOffZ;
 #pragma unroll 1
         for (int blk = 0; blk < D / 64; ++blk) {
-#pragma unroll 2
+#pragma unroll
           for (int c8 = 0; c8 < 8; ++c8) {
             const uint32_t addr = qrow + blk * (kTileM * 128) + sw128_offset(r, c8);
             const uint4 v = lds128(addr);
-            const float4 z0 = __ldg(reinterpret_cast<const float4*>(zc + blk * 64 + c8 * 8));
-            const float4 z1 = __ldg(reinterpret_cast<const float4*>(zc + blk * 64 + c8 * 8 + 4));
-            const float zz[8] = {z0.x, z0.y, z0.z, z0.w, z1.x, z1.y, z1.z, z1.w};
+            const uint4 z0 = lds128(sz + (blk * 64 + c8 * 8) * 4);
+            const uint4 z1 = lds128(sz + (blk * 64 + c8 * 8 + 4) * 4);
+            const uint32_t zz[8] = {z0.x, z0.y, z0.z, z0.w, z1.x, z1.y, z1.z, z1.w};
             uint32_t w4[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
@@ -690,8 +742,8 @@ __global__ void __launch_bounds__(kPairThreads, 1)
               x1 = fmap::feature(p.hyb_fmap, aq, x1);
               w4[e] = pack_bf16x2(x0, x1);
               // the denominator takes the same bf16 values the read-out MMA multiplies
-              dl = fmaf(bf16lo_to_f32(w4[e]), zz[2 * e], dl);
-              dl = fmaf(bf16hi_to_f32(w4[e]), zz[2 * e + 1], dl);
+              dl = fmaf(bf16lo_to_f32(w4[e]), __uint_as_float(zz[2 * e]), dl);
+              dl = fmaf(bf16hi_to_f32(w4[e]), __uint_as_float(zz[2 * e + 1]), dl);
             }
             sts128(addr, make_uint4(w4[0], w4[1], w4[2], w4[3]));
           }
@@ -699,36 +751,37 @@ __global__ void __launch_bounds__(kPairThreads, 1)
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) mbar_arrive(bPhiReady(x));
-        // S_c (fp32 [D][D], row a = key feature) -> bf16 hi + lo, MN-major
-        // 128B-swizzled B operand tiles (64-column blocks of D rows) in the K
-        // stages; with two tiles, warpgroup x converts rows [64 x, 64 x + 64),
-        // thread r the column half r / 64
-        {
-          const int a = hasB ? x * 64 + (r & 63) : r;
-          const int h0 = hasB ? (r >> 6) : 0, h1 = hasB ? h0 + 1 : 2;
-          const float* src = p.hyb_S + (((static_cast<size_t>(c) * p.B + b) * p.H + h) * D + a) * D;
-#pragma unroll 1
-          for (int half = h0; half < h1; ++half) {
-#pragma unroll 2
-            for (int c8 = 0; c8 < 8; ++c8) {
-              const float4 a0 = __ldg(reinterpret_cast<const float4*>(src + half * 64 + c8 * 8));
-              const float4 a1 = __ldg(reinterpret_cast<const float4*>(src + half * 64 + c8 * 8 + 4));
-              const float xs[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
-              uint32_t hi4[4], lo4[4];
+        if (x == 0) {
+          // S_c (fp32 [D][D], row a = key feature) -> bf16 hi + lo, MN-major
+          // 128B-swizzled B operand tiles (64-column blocks of D rows) in the
+          // K stages, which are free once tile B's last Q K^T has completed
+          // too.  Tile A's warpgroup converts all of it, so tile A's read-out
+          // does not wait for tile B's loop to end; consecutive threads take
+          // consecutive 32-byte pieces of S_c (coalesced loads).
+          if (hasB) okh = okh && mbar_wait(bQKDone(1), 0, ab, kStatusTimeoutSoftmax);
+          tc_fence_after();
+          const float* src = p.hyb_S + ((static_cast<size_t>(c) * p.B + b) * p.H + h) * D * D;
+#pragma unroll 4
+          for (int i = 0; i < D * D / (8 * kTileM); ++i) {
+            const int id = i * kTileM + r;        // 8-float piece: row id / 16, piece id % 16
+            const int a = id >> 4, cc = id & 15;
+            const float4 a0 = __ldg(reinterpret_cast<const float4*>(src + a * D + cc * 8));
+            const float4 a1 = __ldg(reinterpret_cast<const float4*>(src + a * D + cc * 8 + 4));
+            const float xs[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+            uint32_t hi4[4], lo4[4];
 #pragma unroll
-              for (int e = 0; e < 4; ++e) {
-                hi4[e] = pack_bf16x2(xs[2 * e], xs[2 * e + 1]);
-                lo4[e] = pack_bf16x2(xs[2 * e] - bf16lo_to_f32(hi4[e]), xs[2 * e + 1] - bf16hi_to_f32(hi4[e]));
-              }
-              const uint32_t off = half * (D * 128) + sw128_offset(a, c8);
-              sts128(sK + off, make_uint4(hi4[0], hi4[1], hi4[2], hi4[3]));
-              sts128(sK + D * D * 2 + off, make_uint4(lo4[0], lo4[1], lo4[2], lo4[3]));
+            for (int e = 0; e < 4; ++e) {
+              hi4[e] = pack_bf16x2(xs[2 * e], xs[2 * e + 1]);
+              lo4[e] = pack_bf16x2(xs[2 * e] - bf16lo_to_f32(hi4[e]), xs[2 * e + 1] - bf16hi_to_f32(hi4[e]));
             }
+            const uint32_t off = (cc >> 3) * (D * 128) + sw128_offset(a, cc & 7);
+            sts128(sK + off, make_uint4(hi4[0], hi4[1], hi4[2], hi4[3]));
+            sts128(sK + D * D * 2 + off, make_uint4(lo4[0], lo4[1], lo4[2], lo4[3]));
           }
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(bScReady);
         }
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(bScReady);
         okh = okh && mbar_wait(bLinDone(x), 0, ab, kStatusTimeoutSoftmax);
         tc_fence_after();
         ok = okh;
@@ -770,6 +823,11 @@ __global__ void __launch_bounds__(kPairThreads, 1)
         const float den = as * l_run + fl * dl;
         const float inv = den > 0.f ? 1.f / den : 0.f;
         __nv_bfloat16* orow = p.o + ((static_cast<size_t>(b) * p.Lq + qn) * p.H + h) * D;
+        // a full tile's rows go through its Q buffer (free: every MMA reading
+        // it has completed) and leave with one TMA store per 64-column block;
+        // a partial tile's rows past its end may belong to the next segment,
+        // so its threads store their own rows
+        const uint32_t stage = sQ + static_cast<uint32_t>(x * C::kTileBytes);
 #pragma unroll 1
         for (int c = 0; c < D / 32; ++c) {
           uint32_t orr[32];
@@ -792,7 +850,12 @@ __global__ void __launch_bounds__(kPairThreads, 1)
 #pragma unroll
           for (int e = 0; e < 16; ++e)
             w[e] = pack_bf16x2(__uint_as_float(orr[2 * e]) * inv, __uint_as_float(orr[2 * e + 1]) * inv);
-          if (row_valid) {
+          if (full_tile) {
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+              sts128(stage + (c >> 1) * (kTileM * 128) + sw128_offset(r, (c & 1) * 4 + e),
+                     make_uint4(w[4 * e], w[4 * e + 1], w[4 * e + 2], w[4 * e + 3]));
+          } else if (row_valid) {
             uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
 #pragma unroll
             for (int e = 0; e < 4; ++e) dst[e] = make_uint4(w[4 * e], w[4 * e + 1], w[4 * e + 2], w[4 * e + 3]);
@@ -801,6 +864,20 @@ __global__ void __launch_bounds__(kPairThreads, 1)
         if (p.lse && row_valid) {
           const float lse = l_run > 0.f ? (m_run + __log2f(l_run)) * 0.69314718055994531f : -INFINITY;
           p.lse[(static_cast<size_t>(b) * p.H + h) * p.Lq + qn] = lse;
+        }
+      }
+      if (full_tile && (HYB || p.n_split <= 1)) {
+        // every thread of the warpgroup takes part (no early exit above), so
+        // the barrier completes; the store runs only if all rows were staged
+        fence_proxy_async_smem();
+        const bool all_ok = x ? bar_and<4, 128>(ok) : bar_and<3, 128>(ok);
+        if (all_ok && threadIdx.x == 128 + 128 * x) {
+#pragma unroll
+          for (int blk = 0; blk < D / 64; ++blk)
+            tma_store_4d(&tmO, sQ + x * C::kTileBytes + blk * (kTileM * 128), blk * 64, h, x ? g.q0[1] : g.q0[0],
+                         b);
+          bulk_commit();
+          bulk_wait_read_all();
         }
       }
     }

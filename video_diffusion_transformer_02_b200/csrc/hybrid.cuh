@@ -34,7 +34,11 @@ struct DeltaParams {
   const float* coef; // [2][H][4] polynomial coefficients (map 1 = k is used here)
 };
 
-constexpr int kRows = 128;   // tokens per tile
+// Tokens per stage: 64-row K and V tiles keep a CTA at 97 KB of shared
+// memory and 128 TMEM columns, so two CTAs share an SM and the whole grid
+// (chunks x heads, 264 CTAs for the MobileWan-style workload) is resident at
+// once: no second wave, HBM streamed by every CTA together.
+constexpr int kRows = 64;
 
 template <int D>
 struct DeltaCfg {
@@ -58,7 +62,7 @@ constexpr int kDeltaThreads = 384;
 constexpr int kPhiThreads = 256;
 
 template <int D>
-__global__ void __launch_bounds__(kDeltaThreads, 1)
+__global__ void __launch_bounds__(kDeltaThreads, 2)
     delta_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                  const DeltaParams p) {
   static_assert(D == 128, "state delta supports head_dim 128");

@@ -166,7 +166,7 @@ uint64_t g_pair_smem_done[5][1];
 // batch.
 template <int D, int ROPE, bool HYB = false>
 vattn_status launch_pair(const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v, const CUtensorMap& k2,
-                         const CUtensorMap& v2, const vattn::attn::Params& p, cudaStream_t s) {
+                         const CUtensorMap& v2, const CUtensorMap& o, const vattn::attn::Params& p, cudaStream_t s) {
   using Cfg = vattn::attn::PairCfg<D>;
   constexpr int slot = HYB ? 4 : (D == 64 ? 0 : 2) + (ROPE == vattn::attn::kRopeQ ? 1 : 0);
   auto kern = vattn::attn::attn_pair_kernel<D, ROPE, HYB>;
@@ -176,24 +176,24 @@ vattn_status launch_pair(const CUtensorMap& q, const CUtensorMap& k, const CUten
   const long long pairs = static_cast<long long>(segs) * ((p.q_tiles_per_seg + 1) / 2);
   if (pairs > 0x7fffffffLL) return fail(VATTN_ERR_UNSUPPORTED, "too many query tiles");
   const dim3 grid(static_cast<unsigned>(pairs), p.H, p.B);
-  kern<<<grid, vattn::attn::kPairThreads, Cfg::kSmemBytes, s>>>(q, k, v, k2, v2, p);
+  kern<<<grid, vattn::attn::kPairThreads, Cfg::kSmemBytes, s>>>(q, k, v, k2, v2, o, p);
   VATTN_CUDA(cudaGetLastError());
   return VATTN_OK;
 }
 
 vattn_status dispatch_attention(int d, int rope_mode, const CUtensorMap& q, const CUtensorMap& k,
                                 const CUtensorMap& v, const CUtensorMap& k2, const CUtensorMap& v2,
-                                const vattn::attn::Params& p, cudaStream_t s) {
+                                const CUtensorMap& o, const vattn::attn::Params& p, cudaStream_t s) {
   using namespace vattn::attn;
   // keys rotated inside the kernel: the one-tile kernel with the RoPE warpgroup
   if (rope_mode == kRopeQK)
     return d == 64 ? launch_fused<64>(q, k, v, k2, v2, p, s) : launch_fused<128>(q, k, v, k2, v2, p, s);
   // keys already rotated (or no RoPE): the two-tile kernel
   if (d == 64)
-    return rope_mode == kRopeQ ? launch_pair<64, kRopeQ>(q, k, v, k2, v2, p, s)
-                               : launch_pair<64, kRopeNone>(q, k, v, k2, v2, p, s);
-  return rope_mode == kRopeQ ? launch_pair<128, kRopeQ>(q, k, v, k2, v2, p, s)
-                             : launch_pair<128, kRopeNone>(q, k, v, k2, v2, p, s);
+    return rope_mode == kRopeQ ? launch_pair<64, kRopeQ>(q, k, v, k2, v2, o, p, s)
+                               : launch_pair<64, kRopeNone>(q, k, v, k2, v2, o, p, s);
+  return rope_mode == kRopeQ ? launch_pair<128, kRopeQ>(q, k, v, k2, v2, o, p, s)
+                             : launch_pair<128, kRopeNone>(q, k, v, k2, v2, o, p, s);
 }
 
 // Rotate K once into k_out (the standalone RoPE kernel on keys only).
@@ -477,19 +477,20 @@ static vattn_status attention_impl(const void* q, const void* k, const void* v, 
   p.test_withhold = withhold;
   fill_rope_params(p, rope, table);
 
-  CUtensorMap mq, mk, mv;
+  CUtensorMap mq, mk, mv, mo;
   if (vattn_status st = make_map(&mq, q, d, H, Lq, B, 128)) return st;
   if (vattn_status st = make_map(&mk, k, d, Hkv, Lk, B, 128)) return st;
   if (vattn_status st = make_map(&mv, v, d, Hkv, Lk, B, 128)) return st;
+  if (vattn_status st = make_map(&mo, o, d, H, Lq, B, 128)) return st;
   if (rope && workspace) {
     // rotate K once into the workspace; the kernel rotates Q tiles itself
     if (vattn_status st = launch_rope_k(k, workspace, B, Lk, Hkv, d, rope, table, k_frame_offset, stream))
       return st;
     CUtensorMap mkr;
     if (vattn_status st = make_map(&mkr, workspace, d, Hkv, Lk, B, 128)) return st;
-    return dispatch_attention(d, vattn::attn::kRopeQ, mq, mkr, mv, mkr, mv, p, stream);
+    return dispatch_attention(d, vattn::attn::kRopeQ, mq, mkr, mv, mkr, mv, mo, p, stream);
   }
-  return dispatch_attention(d, rope ? vattn::attn::kRopeQK : vattn::attn::kRopeNone, mq, mk, mv, mk, mv, p,
+  return dispatch_attention(d, rope ? vattn::attn::kRopeQK : vattn::attn::kRopeNone, mq, mk, mv, mk, mv, mo, p,
                             stream);
 }
 
@@ -654,15 +655,18 @@ vattn_status vattn_attention_stream(vattn_kvcache* c, const void* q, const void*
     p.kseg[n] = vattn::attn::KeySegment{1, 0, 1, 0, 0, c->F, frame_idx, tiles};
   ++n;
   p.n_kseg = n;
+  p.seg_tok = c->F;
   fill_rope_params(p, rope, table);
-  CUtensorMap mq, mk2, mv2;
+  CUtensorMap mq, mk2, mv2, mo;
   if (vattn_status st = make_map(&mq, q, c->d, H, c->F, c->B, 128)) return st;
   if (vattn_status st = make_map(&mk2, k_cur, c->d, c->Hkv, c->F, c->B, 128)) return st;
   if (vattn_status st = make_map(&mv2, v_cur, c->d, c->Hkv, c->F, c->B, 128)) return st;
+  if (vattn_status st = make_map(&mo, o, c->d, H, c->F, c->B, 128)) return st;
   if (rot_ring)
-    return dispatch_attention(c->d, vattn::attn::kRopeQ, mq, c->map_krot, c->map_v, c->map_krot, mv2, p, stream);
+    return dispatch_attention(c->d, vattn::attn::kRopeQ, mq, c->map_krot, c->map_v, c->map_krot, mv2, mo, p,
+                              stream);
   return dispatch_attention(c->d, rope ? vattn::attn::kRopeQK : vattn::attn::kRopeNone, mq, c->map_k,
-                            c->map_v, mk2, mv2, p, stream);
+                            c->map_v, mk2, mv2, mo, p, stream);
 }
 
 vattn_status vattn_kvcache_frame_ids(const vattn_kvcache* c, int32_t* host_ids) {
@@ -776,13 +780,13 @@ uint64_t g_step_smem_done[4][1];
 
 template <int D, int ROPE>
 vattn_status launch_step(const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v, const CUtensorMap& k2,
-                         const CUtensorMap& v2, const vattn::attn::Params& p, cudaStream_t s) {
+                         const CUtensorMap& v2, const CUtensorMap& o, const vattn::attn::Params& p, cudaStream_t s) {
   using Cfg = vattn::attn::PairCfg<D>;
   auto kern = vattn::attn::attn_pair_kernel<D, ROPE, false>;
   vattn_status st = ensure_smem(kern, Cfg::kSmemBytes,
                                 g_step_smem_done[(D == 64 ? 0 : 2) + (ROPE == vattn::attn::kRopeQ ? 1 : 0)]);
   if (st) return st;
-  kern<<<p.total_ctas, vattn::attn::kPairThreads, Cfg::kSmemBytes, s>>>(q, k, v, k2, v2, p);
+  kern<<<p.total_ctas, vattn::attn::kPairThreads, Cfg::kSmemBytes, s>>>(q, k, v, k2, v2, o, p);
   VATTN_CUDA(cudaGetLastError());
   return VATTN_OK;
 }
@@ -878,6 +882,7 @@ vattn_status vattn_kvcache_step(vattn_kvcache* c, const void* q, const void* k_c
     p.kseg[n++] = vattn::attn::KeySegment{1, 0, 1, 0, 0, c->F, frame_idx, tiles};
   tiles += per;
   p.n_kseg = n;
+  p.seg_tok = c->F;
   fill_rope_params(p, rope, table);
 
   // the append: raw K and V into slot frame % capacity (outside the window),
@@ -919,18 +924,19 @@ vattn_status vattn_kvcache_step(vattn_kvcache* c, const void* q, const void* k_c
   if (total > 0x7fffffffLL) return fail(VATTN_ERR_UNSUPPORTED, "grid too large");
   p.total_ctas = static_cast<int>(total);
 
-  CUtensorMap mq, mk2, mv2;
+  CUtensorMap mq, mk2, mv2, mo;
   if (vattn_status st = make_map(&mq, q, c->d, H, c->F, c->B, 128)) return st;
   if (vattn_status st = make_map(&mk2, k_cur, c->d, c->Hkv, c->F, c->B, 128)) return st;
   if (vattn_status st = make_map(&mv2, v_cur, c->d, c->Hkv, c->F, c->B, 128)) return st;
+  if (vattn_status st = make_map(&mo, o, c->d, H, c->F, c->B, 128)) return st;
   const CUtensorMap& mk = rope ? c->map_krot : c->map_k;
   vattn_status st;
   if (c->d == 64)
-    st = rope ? launch_step<64, vattn::attn::kRopeQ>(mq, mk, c->map_v, mk2, mv2, p, stream)
-              : launch_step<64, vattn::attn::kRopeNone>(mq, mk, c->map_v, mk2, mv2, p, stream);
+    st = rope ? launch_step<64, vattn::attn::kRopeQ>(mq, mk, c->map_v, mk2, mv2, mo, p, stream)
+              : launch_step<64, vattn::attn::kRopeNone>(mq, mk, c->map_v, mk2, mv2, mo, p, stream);
   else
-    st = rope ? launch_step<128, vattn::attn::kRopeQ>(mq, mk, c->map_v, mk2, mv2, p, stream)
-              : launch_step<128, vattn::attn::kRopeNone>(mq, mk, c->map_v, mk2, mv2, p, stream);
+    st = rope ? launch_step<128, vattn::attn::kRopeQ>(mq, mk, c->map_v, mk2, mv2, mo, p, stream)
+              : launch_step<128, vattn::attn::kRopeNone>(mq, mk, c->map_v, mk2, mv2, mo, p, stream);
   if (st) return st;
   c->host_ids[slot] = frame_idx;
   c->rotated_k = nullptr;
@@ -1007,8 +1013,8 @@ vattn_status vattn_hybrid_delta(const void* k, const void* v, int B, int L, int 
   uint32_t* status;
   if (vattn_status st = status_ptr(&status)) return st;
   CUtensorMap mk, mv;
-  if (vattn_status st = make_map(&mk, k, d, H, L, B, 128)) return st;
-  if (vattn_status st = make_map(&mv, v, d, H, L, B, 128)) return st;
+  if (vattn_status st = make_map(&mk, k, d, H, L, B, vattn::hyb::kRows)) return st;
+  if (vattn_status st = make_map(&mv, v, d, H, L, B, vattn::hyb::kRows)) return st;
   return launch_delta(mk, mv, wsS, wsz, status, B, L, H, C, chunk_tokens, stream);
 }
 
@@ -1054,13 +1060,18 @@ vattn_status hybrid_impl(const void* q, const void* k, const void* v, void* o, f
   uint32_t* status;
   if (vattn_status st = status_ptr(&status)) return st;
 
-  CUtensorMap mq, mk, mv;
+  CUtensorMap mq, mk, mv, mo;
   if (vattn_status st = make_map(&mq, q, d, H, L, B, 128)) return st;
   if (vattn_status st = make_map(&mk, k, d, H, L, B, 128)) return st;
   if (vattn_status st = make_map(&mv, v, d, H, L, B, 128)) return st;
+  if (vattn_status st = make_map(&mo, o, d, H, L, B, 128)) return st;
 
-  // (1) per-range state deltas, (2) exclusive scan over ranges (+ state out)
-  if (vattn_status st = launch_delta(mk, mv, wsS, wsz, status, B, L, H, R, chunk_tokens, stream, overlap, fmap,
+  // (1) per-range state deltas (tiles of vattn::hyb::kRows tokens), (2)
+  // exclusive scan over ranges (+ state out)
+  CUtensorMap mkd, mvd;
+  if (vattn_status st = make_map(&mkd, k, d, H, L, B, vattn::hyb::kRows)) return st;
+  if (vattn_status st = make_map(&mvd, v, d, H, L, B, vattn::hyb::kRows)) return st;
+  if (vattn_status st = launch_delta(mkd, mvd, wsS, wsz, status, B, L, H, R, chunk_tokens, stream, overlap, fmap,
                                      coef))
     return st;
   if (vattn_status st = launch_scan(wsS, wsz, S, z, B, H, d, R, stream)) return st;
@@ -1088,7 +1099,7 @@ vattn_status hybrid_impl(const void* q, const void* k, const void* v, void* o, f
   p.hyb_fmap = fmap;
   p.hyb_coef = coef;
   p.lead = overlap;
-  return launch_pair<128, vattn::attn::kRopeNone, true>(mq, mk, mv, mk, mv, p, stream);
+  return launch_pair<128, vattn::attn::kRopeNone, true>(mq, mk, mv, mk, mv, mo, p, stream);
 }
 }  // namespace
 
