@@ -163,7 +163,9 @@ def wan13b_workload(va, torch, device):
     dev = lambda x: torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).to(device)
     rope = va.Rope(Hg=Hg, Wg=Wg, pairs=c["pairs"], max_pos=max(T, Hg, Wg), theta=c["theta"])
     tab = va.rope_table(rope, d, device=device)
-    ws = torch.empty(va.vattn_attention_workspace_bytes(B, L, H, d, rope), dtype=torch.uint8, device=device)
+    # rotated keys, then the tail split of the last partial wave (zero-filled)
+    ws = torch.zeros(va.vattn_attention_workspace_bytes_ex(B, L, L, H, H, d, "full", rope, device=device),
+                     dtype=torch.uint8, device=device)
     w = dict(name="wan13b", B=B, H=H, d=d, L=L, T=T, Hg=Hg, Wg=Wg, rope=rope, tab=tab, ws=ws,
              q_host=q, k_host=k, v_host=v, q=dev(q), k=dev(k), v=dev(v),
              o=torch.empty((B, L, H, d), dtype=torch.bfloat16, device=device),

@@ -113,7 +113,9 @@ vattn_status vattn_rope_qk(const void* q, const void* k, void* q_out, void* k_ou
  *   rope->Hg * rope->Wg.  The query tile is rotated inside the kernel on its
  *   shared-memory copy.  Keys: see vattn_attention_workspace_bytes.
  *   workspace (nullable, device, 16-byte aligned) of workspace_bytes: scratch
- *   for the rotated keys; unused without rope.
+ *   for the rotated keys (unused without rope) and, when workspace_bytes
+ *   reaches vattn_attention_workspace_bytes_ex, for the tail split of a FULL
+ *   call (zero-filled before first use, see there).
  * o = softmax(scale * q k^T restricted to visible keys) v, computed with an
  * online softmax (fp32 statistics, fp32 accumulation, bf16 P and output).
  * Tiles with no visible key are never loaded.
@@ -131,6 +133,19 @@ vattn_status vattn_attention(const void* q, const void* k, const void* v, void* 
    kernel rotates only its Q tile (once per tile); with workspace == NULL
    the kernel also rotates every K tile it loads, in shared memory. */
 size_t vattn_attention_workspace_bytes(int B, int Lk, int Hkv, int d, const vattn_rope* rope);
+
+/* Bytes of workspace that also enable the tail split of a VATTN_FULL call:
+   when the call's work units (pairs of 128-row query tiles x heads x batch)
+   leave a last partial wave that fills at most half the SMs of the current
+   device, each unit of that wave runs as several CTAs over parts of its
+   keys, merged exactly inside the kernel, so the otherwise idle SMs share
+   the last wave.  The extra bytes (after the rotated keys, from a 256-byte
+   boundary) hold arrival counters and fp32 partials: zero-fill the
+   workspace before its first use; every call leaves the counters at zero.
+   Calls sharing a workspace must not overlap on the GPU.  Equals
+   vattn_attention_workspace_bytes when the split does not apply. */
+size_t vattn_attention_workspace_bytes_ex(int B, int Lq, int Lk, int H, int Hkv, int d, vattn_mode mode,
+                                          const vattn_rope* rope);
 
 /*
  * Exact combination of R partial attentions of the same queries over

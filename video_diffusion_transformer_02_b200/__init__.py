@@ -75,6 +75,7 @@ _rope_qk = _sig("vattn_rope_qk", _I, _P, _P, _P, _P, _I, _I, _I, _I, _I, _RP, _P
 _attention = _sig("vattn_attention", _I, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _I, _I, _I,
                   _I, _I, _I, _I, _RP, _P, _P, _S, _P)
 _attn_ws = _sig("vattn_attention_workspace_bytes", _S, _I, _I, _I, _I, _RP)
+_attn_ws_ex = _sig("vattn_attention_workspace_bytes_ex", _S, _I, _I, _I, _I, _I, _I, _I, _RP)
 _merge = _sig("vattn_attention_merge", _I, _P, _P, _I, _P, _P, _I, _I, _I, _I, _P)
 _kv_init = _sig("vattn_kvcache_init", _I, ctypes.POINTER(_P), _P, _P, _P, _I, _I, _I, _I, _I, _P)
 _kv_append = _sig("vattn_kvcache_append", _I, _P, _P, _P, _I, _P)
@@ -249,6 +250,18 @@ def vattn_attention_workspace_bytes(B, Lk, Hkv, d, rope: Rope | None) -> int:
     return _attn_ws(B, Lk, Hkv, d, _rope_c(rope))
 
 
+def vattn_attention_workspace_bytes_ex(B, Lq, Lk, H, Hkv, d, mode="full", rope: Rope | None = None,
+                                       device=None) -> int:
+    """Workspace bytes for the rotated keys plus the tail split of a FULL
+    call (zero-fill it before first use); depends on the SM count of `device`
+    (the current device when None)."""
+    m = MODES[mode] if isinstance(mode, str) else int(mode)
+    if device is None:
+        return _attn_ws_ex(B, Lq, Lk, H, Hkv, d, m, _rope_c(rope))
+    with torch.cuda.device(device):
+        return _attn_ws_ex(B, Lq, Lk, H, Hkv, d, m, _rope_c(rope))
+
+
 def vattn_attention(q, k, v, o, lse=None, scale=None, mode="full", tokens_per_frame=0,
                     chunk_frames=1, window_back=0, window_fwd=0, q_frame_offset=0,
                     k_frame_offset=0, rope: Rope | None = None, table=None, workspace=None,
@@ -257,7 +270,9 @@ def vattn_attention(q, k, v, o, lse=None, scale=None, mode="full", tokens_per_fr
 
     With rope, keys are rotated once into `workspace` (allocated here with
     torch when not given); fuse_k_rope=True passes no workspace, so the kernel
-    rotates every K tile in shared memory instead.
+    rotates every K tile in shared memory instead.  A zero-filled uint8
+    workspace of vattn_attention_workspace_bytes_ex bytes also enables the
+    tail split of FULL calls.
     """
     _rank(q, "q", 4)
     _rank(k, "k", 4)
@@ -285,7 +300,9 @@ def vattn_attention(q, k, v, o, lse=None, scale=None, mode="full", tokens_per_fr
         if workspace is None:
             workspace = torch.empty(need, dtype=torch.uint8, device=dev)
         _min_bytes(workspace, "workspace", need)
-        ws_ptr, ws_bytes = _ptr(workspace), workspace.numel() * workspace.element_size()
+    if workspace is not None and not fuse_k_rope:
+        _expect(workspace, "workspace", None, torch.uint8)
+        ws_ptr, ws_bytes = _ptr(workspace), workspace.numel()
     with torch.cuda.device(dev):
         _ok(_attention(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, Lq, Lk, H, Hkv, d, float(scale), m,
                        tokens_per_frame, chunk_frames, window_back, window_fwd, q_frame_offset,

@@ -132,6 +132,12 @@ struct Params {
   uint32_t* step_sync;      // [0] append shares done, [1] CTAs exited; back to 0 at the last exit
   int wait_tile;            // key tiles >= this read keys the append CTAs write (-1: none)
   int total_ctas;
+  // tail split (linear grid): the first n_normal (pair, head, batch) items
+  // run whole, each later item as n_split CTAs over parts of its key
+  // range, with partials in a compact layout ([item - n_normal][split][256
+  // rows of the pair])
+  int tail_split;
+  int n_normal;
 };
 
 template <int D>

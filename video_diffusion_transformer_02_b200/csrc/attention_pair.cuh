@@ -43,32 +43,26 @@ struct PairCfg {
   static constexpr int kOffK = 2 * kTileBytes;
   static constexpr int kOffV = kOffK + kStages * kTileBytes;
   static constexpr int kOffBar = kOffV + kStages * kTileBytes;
-  static constexpr int kNumBars = 4 + 4 * kStages + 12 + 2 + 5 + 2 + 3;
+  static constexpr int kNumBars = 4 + 4 * kStages + 12 + 2 + 5 + 3;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
   static constexpr int kOffZ = kOffMisc + 64;        // hybrid: z_c, fp32 [D]
   static constexpr int kSmemBytes = kOffZ + D * 4;
 };
 
 constexpr int kPairThreads = 384;
-// The two softmax warpgroups take turns on their exponential phases at head
-// dim 64, where the exponentials outweigh the tensor-core work per score
-// (measured: +4 % on the 16-head stream); at head dim 128 the turns cost
-// 3 % and are off.
-template <int D>
-struct TakeTurns {
-  static constexpr bool value = D == 64;
-};
+
 
 // Rows of the two query tiles of pair `pr` and the key tiles they need
 // (the union of both tiles' visible ranges; rows mask what they do not see).
 struct PairGeom {
   int q0[2], q_end[2];
   bool hasB;
-  TileGeom tg;   // q0 / q_end span both tiles; kbeg, kend, n_tiles: the union
-  int t0;        // segment mode: the CTA's first key tile (key split); 0 otherwise
+  TileGeom tg;   // q0 / q_end span both tiles; kbeg, kend: the union; n_tiles: this CTA's share
+  int t0;        // the CTA's first key tile of the union (key split; 0 without)
 };
 
-__device__ __forceinline__ PairGeom pair_geom(const Params& p, int pr, int split) {
+// The pair's key tiles split into nsplit near-equal parts; part `split`.
+__device__ __forceinline__ PairGeom pair_geom(const Params& p, int pr, int split, int nsplit) {
   PairGeom g;
   const int pps = (p.q_tiles_per_seg + 1) / 2;
   const int seg = pr / pps;
@@ -89,16 +83,29 @@ __device__ __forceinline__ PairGeom pair_geom(const Params& p, int pr, int split
     key_range(p, g.tg.q_end - 1, lo1, hi1);
     g.tg.kbeg = lo0;
     g.tg.kend = hi1;
-    g.tg.n_tiles = g.tg.kend > g.tg.kbeg ? (g.tg.kend - g.tg.kbeg + kTileN - 1) / kTileN : 0;
+    const int total = g.tg.kend > g.tg.kbeg ? (g.tg.kend - g.tg.kbeg + kTileN - 1) / kTileN : 0;
+    const int per = (total + nsplit - 1) / nsplit;
+    g.t0 = min(total, split * per);
+    g.tg.n_tiles = min(total, g.t0 + per) - g.t0;
   } else {
     g.tg.kbeg = g.tg.kend = 0;
     const KeySegment& last = p.kseg[p.n_kseg - 1];
     const int total = last.tile0 + (last.n_tok + kTileN - 1) / kTileN;
-    const int per = p.n_split > 1 ? p.split_tiles : total;
+    const int per = nsplit > 1 ? p.split_tiles : total;
     g.t0 = min(total, split * per);
     g.tg.n_tiles = min(total, g.t0 + per) - g.t0;
   }
   return g;
+}
+
+// Where split `s`'s partial of query row `row` lives (row index into
+// part_lse; times D into part_o): the streaming step's [split][B][H][Lq]
+// layout, or the tail split's compact [tail item][split][256 pair rows].
+__device__ __forceinline__ size_t part_row(const Params& p, const PairGeom& g, int b, int h, int s, int nsplit,
+                                           int tail_item, int row) {
+  if (p.tail_split)
+    return (static_cast<size_t>(tail_item) * nsplit + s) * (2 * kTileM) + (row - g.q0[0]);
+  return ((static_cast<size_t>(s) * p.B + b) * p.H + h) * p.Lq + row;
 }
 
 // A streaming step's append share: CTA `part` of the n_append leading CTAs
@@ -169,21 +176,21 @@ __device__ __forceinline__ void append_share(const Params& p, int part) {
 // then the warp walks the rows, lane l reading and writing columns
 // [l D/32, (l+1) D/32) (coalesced rows of the partials, from L2).
 template <int D>
-__device__ __forceinline__ void merge_splits(const Params& p, const PairGeom& g, int b, int h, int warp, int lane) {
+__device__ __forceinline__ void merge_splits(const Params& p, const PairGeom& g, int b, int h, int warp, int lane,
+                                             int S, int tail_item) {
   const int x = (warp - 4) >> 2;
   if (x == 1 && !g.hasB) return;
   const int r0 = (x ? g.q0[1] : g.q0[0]) + (warp & 3) * 32;
   const int q_end = x ? g.q_end[1] : g.q_end[0];
   if (r0 >= q_end) return;
-  const int S = p.n_split;
-  const size_t split_rows = static_cast<size_t>(p.B) * p.H * p.Lq;   // rows of one split's partials
   const size_t bh = (static_cast<size_t>(b) * p.H + h) * p.Lq;
   const int myrow = r0 + lane;
   float wts[kMaxSplit];
   float M = -INFINITY;
 #pragma unroll
   for (int s = 0; s < kMaxSplit; ++s) {
-    wts[s] = (s < S && myrow < q_end) ? __ldcg(p.part_lse + s * split_rows + bh + myrow) : -INFINITY;
+    wts[s] = (s < S && myrow < q_end) ? __ldcg(p.part_lse + part_row(p, g, b, h, s, S, tail_item, myrow))
+                                      : -INFINITY;
     M = fmaxf(M, wts[s]);
   }
   float W = 0.f;
@@ -206,7 +213,7 @@ __device__ __forceinline__ void merge_splits(const Params& p, const PairGeom& g,
     for (int s = 0; s < kMaxSplit; ++s) {
       if (s < S) {
         const float w = __shfl_sync(0xffffffffu, wts[s], rr);
-        const float* src = p.part_o + (s * split_rows + bh + r0 + rr) * D + lane * CPL;
+        const float* src = p.part_o + part_row(p, g, b, h, s, S, tail_item, r0 + rr) * D + lane * CPL;
         if constexpr (CPL == 2) {
           const float2 v = __ldcg(reinterpret_cast<const float2*>(src));
           acc[0] = fmaf(w, v.x, acc[0]);
@@ -274,8 +281,23 @@ __global__ void __launch_bounds__(kPairThreads, 1)
   }
   // which work this CTA does: (pair, head, batch) of a 3-D grid, or an
   // append share / (pair, head, batch, split) of a streaming step's 1-D grid
-  int pr, h, b, split = 0;
-  if (p.linear_grid) {
+  int pr, h, b, split = 0, nsplit = 1, tail_item = 0;
+  if (p.linear_grid && p.tail_split) {
+    // whole items first, then the split items' parts
+    const int idx = static_cast<int>(blockIdx.x);
+    int item = idx;
+    if (idx >= p.n_normal) {
+      const int rel = idx - p.n_normal;
+      tail_item = rel / p.n_split;
+      split = rel - tail_item * p.n_split;
+      nsplit = p.n_split;
+      item = p.n_normal + tail_item;
+    }
+    pr = item % p.n_pairs;
+    item /= p.n_pairs;
+    h = item % p.H;
+    b = item / p.H;
+  } else if (p.linear_grid) {
     int idx = static_cast<int>(blockIdx.x);
     if (idx < p.n_append) {
       append_share<D>(p, idx);
@@ -289,6 +311,7 @@ __global__ void __launch_bounds__(kPairThreads, 1)
     idx /= p.H;
     b = idx % p.B;
     split = idx / p.B;
+    nsplit = p.n_split > 1 ? p.n_split : 1;
   } else {
     h = blockIdx.y;
     b = blockIdx.z;
@@ -312,14 +335,10 @@ __global__ void __launch_bounds__(kPairThreads, 1)
   auto bPhiReady = [&](int x) { return bx + 112 + 8 * x; };
   const uint32_t bScReady = bx + 128;
   auto bLinDone = [&](int x) { return bx + 136 + 8 * x; };
-  // exponential phases of the two softmax warpgroups take turns: tile A's
-  // phase for sub-tile u waits on bTurnA (tile B done with u - 1), tile B's
-  // on bTurnB (tile A done with u)
-  const uint32_t bTurnA = bx + 152, bTurnB = bx + 160;
   // hybrid: each tile's last Q K^T complete (Q_x and, with both, the K
   // stages free); z_c landed in shared memory
-  auto bQKDone = [&](int x) { return bx + 168 + 8 * x; };
-  const uint32_t bZFull = bx + 184;
+  auto bQKDone = [&](int x) { return bx + 152 + 8 * x; };
+  const uint32_t bZFull = bx + 168;
   uint32_t* misc = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
   volatile uint32_t* tmem_slot = misc;
   volatile uint32_t* abort_flag = misc + 1;
@@ -327,7 +346,7 @@ __global__ void __launch_bounds__(kPairThreads, 1)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int kvh = h / (p.H / p.Hkv);
-  const PairGeom g = pair_geom(p, pr, split);
+  const PairGeom g = pair_geom(p, pr, split, nsplit);
   if (g.q0[0] >= g.q_end[0]) {   // pair past the end of a short last segment
     if (stepping) step_exit(p);
     return;
@@ -364,8 +383,6 @@ __global__ void __launch_bounds__(kPairThreads, 1)
     mbar_init(bZFull, 1);
     mbar_init(bLinDone(0), 1);
     mbar_init(bLinDone(1), 1);
-    mbar_init(bTurnA, 4);
-    mbar_init(bTurnB, 4);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -594,7 +611,7 @@ __global__ void __launch_bounds__(kPairThreads, 1)
         const uint32_t tS = trow + static_cast<uint32_t>(x * 128 + bb * kSub);
         int col_lo = 0, col_hi = kSub;
         if (p.n_kseg == 0) {
-          const int k0 = g.tg.kbeg + u * kSub;
+          const int k0 = g.tg.kbeg + g.t0 * kTileN + u * kSub;
           col_lo = lo - k0;
           col_hi = hi - k0;
         } else if (p.seg_tok > 0) {
@@ -636,15 +653,6 @@ __global__ void __launch_bounds__(kPairThreads, 1)
           resc = true;
         }
         const float nm = (m_run == -INFINITY) ? 0.f : -m_run;
-        // turns: the MUFU serves one warpgroup's exponentials at a time
-        // while the other loads, reduces and publishes
-        if (TakeTurns<D>::value && hasB) {
-          if (x == 0) {
-            if (u > 0 && !mbar_wait(bTurnA, (u - 1) & 1, ab, kStatusTimeoutSoftmax)) ok = false;
-          } else if (!mbar_wait(bTurnB, u & 1, ab, kStatusTimeoutSoftmax)) {
-            ok = false;
-          }
-        }
         // P = exp2(s * scale * log2e - m) into the first half of the S
         // buffer, 16 columns (32 keys) at a time; row sums as packed fp32x2
         float rs2[2][2] = {{0.f, 0.f}, {0.f, 0.f}};
@@ -680,10 +688,6 @@ __global__ void __launch_bounds__(kPairThreads, 1)
             }
           }
           tmem_st16(tS + q * 16, pk);
-        }
-        if (TakeTurns<D>::value && hasB) {
-          __syncwarp();
-          if (lane == 0 && (x == 0 || u + 1 < ns)) mbar_arrive(x == 0 ? bTurnB : bTurnA);
         }
         const float rs = (rs2[0][0] + rs2[0][1]) + (rs2[1][0] + rs2[1][1]);
         // O_x rescale: wait until the P V of the previous sub-tile (which
@@ -761,7 +765,7 @@ __global__ void __launch_bounds__(kPairThreads, 1)
           if (hasB) okh = okh && mbar_wait(bQKDone(1), 0, ab, kStatusTimeoutSoftmax);
           tc_fence_after();
           const float* src = p.hyb_S + ((static_cast<size_t>(c) * p.B + b) * p.H + h) * D * D;
-#pragma unroll 4
+#pragma unroll 8
           for (int i = 0; i < D * D / (8 * kTileM); ++i) {
             const int id = i * kTileM + r;        // 8-float piece: row id / 16, piece id % 16
             const int a = id >> 4, cc = id & 15;
@@ -794,11 +798,11 @@ __global__ void __launch_bounds__(kPairThreads, 1)
         tc_fence_after();
       }
       ok = __all_sync(0xffffffffu, ok);   // the TMEM loads below are warp-collective
-      if (ok && !HYB && p.n_split > 1) {
+      if (ok && !HYB && nsplit > 1) {
         // key split: this CTA's partial result, o / l in fp32 and m + log2 l,
         // for the pair's merging CTA
         const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
-        const size_t prow = ((static_cast<size_t>(split) * p.B + b) * p.H + h) * p.Lq + qn;
+        const size_t prow = part_row(p, g, b, h, split, nsplit, tail_item, qn);
         float* dst = p.part_o + prow * D;
 #pragma unroll 1
         for (int c = 0; c < D / 32; ++c) {
@@ -866,7 +870,7 @@ __global__ void __launch_bounds__(kPairThreads, 1)
           p.lse[(static_cast<size_t>(b) * p.H + h) * p.Lq + qn] = lse;
         }
       }
-      if (full_tile && (HYB || p.n_split <= 1)) {
+      if (full_tile && (HYB || nsplit <= 1)) {
         // every thread of the warpgroup takes part (no early exit above), so
         // the barrier completes; the store runs only if all rows were staged
         fence_proxy_async_smem();
@@ -883,20 +887,21 @@ __global__ void __launch_bounds__(kPairThreads, 1)
     }
   }
 
-  if (!HYB && p.n_split > 1 && warp >= 4 && warp < 12) {
+  if (!HYB && nsplit > 1 && warp >= 4 && warp < 12) {
     // key split: count this CTA's partial in; the pair's last CTA merges
     __threadfence();
     asm volatile("bar.sync 2, 256;" ::: "memory");
     volatile uint32_t* last = misc + 2;
-    const size_t pc = (static_cast<size_t>(b) * p.H + h) * p.n_pairs + pr;
+    const size_t pc = p.tail_split ? static_cast<size_t>(tail_item)
+                                   : (static_cast<size_t>(b) * p.H + h) * p.n_pairs + pr;
     if (threadIdx.x == 128) {
       const uint32_t old = atomicAdd(p.pair_count + pc, 1u);
-      *last = old == static_cast<uint32_t>(p.n_split) - 1u ? 1u : 0u;
+      *last = old == static_cast<uint32_t>(nsplit) - 1u ? 1u : 0u;
       __threadfence();
     }
     asm volatile("bar.sync 2, 256;" ::: "memory");
     if (*last) {
-      merge_splits<D>(p, g, b, h, warp, lane);
+      merge_splits<D>(p, g, b, h, warp, lane, nsplit, tail_item);
       if (threadIdx.x == 128) p.pair_count[pc] = 0u;
     }
   }

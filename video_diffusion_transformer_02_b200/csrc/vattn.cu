@@ -51,6 +51,54 @@ vattn_status cuda_fail(cudaError_t e, const char* where) {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+int sm_count() {
+  int sms = 148, dev;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  return sms;
+}
+
+size_t round256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+// Tail split of a FULL attention call: with `items` (pair, head, batch)
+// work units on `sms` SMs (one two-tile CTA per SM), the last partial wave of
+// r items leaves sms - r SMs idle for a whole item; when r <= sms / 2 those
+// items run as s = min(sms / r, 16, key tiles) CTAs each (fewer when some
+// would get no key tile), over parts of their keys, merged in the kernel.
+// Workspace: r arrival counters, then the partials (lse fp32 and o fp32) of
+// r * s CTAs x 256 query rows.
+struct TailLayout {
+  long long n_normal = 0;
+  int n_split = 1, tail_items = 0;
+  size_t off_count = 0, off_lse = 0, off_o = 0, bytes = 0;
+};
+
+TailLayout tail_layout(int B, int Lq, int Lk, int H, int d) {
+  TailLayout t;
+  if (B < 1 || Lq < 1 || Lk < 1 || H < 1 || d < 1) return t;
+  const long long pairs = ((Lq + 127) / 128 + 1) / 2;
+  const long long items = pairs * H * B;
+  const int sms = sm_count();
+  const long long waves = items / sms, r = items - waves * sms;
+  const int key_tiles = (Lk + 127) / 128;
+  if (waves < 1 || r == 0 || 2 * r > sms || key_tiles < 2) return t;
+  int sp = static_cast<int>(sms / r);
+  sp = std::min(sp, vattn::attn::kMaxSplit);
+  sp = std::min(sp, key_tiles);
+  // the kernel gives each split ceil(key_tiles / sp) key tiles: drop the
+  // splits that would be left with none
+  const int per = (key_tiles + sp - 1) / sp;
+  sp = (key_tiles + per - 1) / per;
+  if (sp < 2) return t;
+  t.n_split = sp;
+  t.tail_items = static_cast<int>(r);
+  t.n_normal = items - r;
+  t.off_count = 0;
+  t.off_lse = round256(static_cast<size_t>(r) * 4);
+  t.off_o = t.off_lse + round256(static_cast<size_t>(r) * sp * 256 * 4);
+  t.bytes = t.off_o + static_cast<size_t>(r) * sp * 256 * d * 4;
+  return t;
+}
+
 // ---------------------------------------------------------------- devices
 constexpr int kMaxDevices = 64;
 uint32_t* g_status_ptr[kMaxDevices];
@@ -175,7 +223,8 @@ vattn_status launch_pair(const CUtensorMap& q, const CUtensorMap& k, const CUten
   const int segs = p.n_q_tiles / p.q_tiles_per_seg;
   const long long pairs = static_cast<long long>(segs) * ((p.q_tiles_per_seg + 1) / 2);
   if (pairs > 0x7fffffffLL) return fail(VATTN_ERR_UNSUPPORTED, "too many query tiles");
-  const dim3 grid(static_cast<unsigned>(pairs), p.H, p.B);
+  const dim3 grid = p.linear_grid ? dim3(static_cast<unsigned>(p.total_ctas))
+                                  : dim3(static_cast<unsigned>(pairs), p.H, p.B);
   kern<<<grid, vattn::attn::kPairThreads, Cfg::kSmemBytes, s>>>(q, k, v, k2, v2, o, p);
   VATTN_CUDA(cudaGetLastError());
   return VATTN_OK;
@@ -408,6 +457,15 @@ size_t vattn_attention_workspace_bytes(int B, int Lk, int Hkv, int d, const vatt
   return static_cast<size_t>(B) * Lk * Hkv * d * 2;
 }
 
+size_t vattn_attention_workspace_bytes_ex(int B, int Lq, int Lk, int H, int Hkv, int d, vattn_mode mode,
+                                          const vattn_rope* rope) {
+  const size_t rot = vattn_attention_workspace_bytes(B, Lk, Hkv, d, rope);
+  if (mode != VATTN_FULL) return rot;
+  const TailLayout t = tail_layout(B, Lq, Lk, H, d);
+  if (t.n_split <= 1) return rot;
+  return (rope ? round256(rot) : 0) + t.bytes;
+}
+
 // vattn_attention with the two self-test knobs of the parameter block (a
 // wait bound other than the default, one withheld softmax arrival).
 static vattn_status attention_impl(const void* q, const void* k, const void* v, void* o, float* lse, int B,
@@ -482,6 +540,25 @@ static vattn_status attention_impl(const void* q, const void* k, const void* v, 
   if (vattn_status st = make_map(&mk, k, d, Hkv, Lk, B, 128)) return st;
   if (vattn_status st = make_map(&mv, v, d, Hkv, Lk, B, 128)) return st;
   if (vattn_status st = make_map(&mo, o, d, H, Lq, B, 128)) return st;
+  // tail split (FULL mode, two-tile kernel, workspace of the _ex size)
+  if (workspace && mode == VATTN_FULL) {
+    const size_t base = rope ? round256(vattn_attention_workspace_bytes(B, Lk, Hkv, d, rope)) : 0;
+    const TailLayout t = tail_layout(B, Lq, Lk, H, d);
+    if (t.n_split > 1 && workspace_bytes >= base + t.bytes) {
+      uint8_t* ws = static_cast<uint8_t*>(workspace) + base;
+      p.linear_grid = 1;
+      p.tail_split = 1;
+      p.n_split = t.n_split;
+      p.n_normal = static_cast<int>(t.n_normal);
+      p.n_pairs = (p.q_tiles_per_seg + 1) / 2;
+      p.pair_count = reinterpret_cast<uint32_t*>(ws + t.off_count);
+      p.part_lse = reinterpret_cast<float*>(ws + t.off_lse);
+      p.part_o = reinterpret_cast<float*>(ws + t.off_o);
+      const long long total = t.n_normal + static_cast<long long>(t.tail_items) * t.n_split;
+      if (total > 0x7fffffffLL) return fail(VATTN_ERR_UNSUPPORTED, "grid too large");
+      p.total_ctas = static_cast<int>(total);
+    }
+  }
   if (rope && workspace) {
     // rotate K once into the workspace; the kernel rotates Q tiles itself
     if (vattn_status st = launch_rope_k(k, workspace, B, Lk, Hkv, d, rope, table, k_frame_offset, stream))
@@ -719,11 +796,6 @@ vattn_status vattn_kvcache_destroy(vattn_kvcache* c) {
 
 // ------------------------------------------------- fused streaming step
 namespace {
-int sm_count() {
-  int sms = 148, dev;
-  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  return sms;
-}
 
 // Key splits for `items` (pair, head, batch) work units of n_tiles key tiles
 // each on `sms` SMs (one CTA per SM): the count minimising
