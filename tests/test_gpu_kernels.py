@@ -141,6 +141,34 @@ def test_attention_single_token_and_tiny_lengths(va):
         assert_parity(from_dev(o), ref, "L=%d" % L)
 
 
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("mode,kw", [("full", {}), ("sliding", dict(wb=1, wf=0))])
+def test_attention_large_logit_jumps(va, d, mode, kw):
+    # Every block of 64 keys is scaled by its own seeded factor 2^(0..9), so
+    # a row's max jumps by up to ~2000 log2 units from one sub-tile to the
+    # next, in both directions: the reference max must move (O rescaled)
+    # and exponentials taken against a stale reference must be redone.
+    import torch
+    B, H, F, T = 1, 2, 100, 15
+    L = F * T
+    q = si.normal_bf16(80 + d, (B, L, H, d))
+    k = si.normal_bf16(81 + d, (B, L, H, d))
+    v = si.normal_bf16(82 + d, (B, L, H, d))
+    f = 2.0 ** np.floor(10.0 * si.uniform01(83 + d, (L + 63) // 64))
+    kf = si.bf16_bits_to_f64(k) * np.repeat(f, 64)[:L][None, :, None, None]
+    k = si.f64_to_bf16_bits(kf)
+    og = guarded((B, L, H, d), torch.bfloat16, float("nan"))
+    lg = guarded((B, H, L), torch.float32, float("nan"))
+    va.vattn_attention(to_dev(q), to_dev(k), to_dev(v), og.t, lg.t, scale=d ** -0.5, mode=mode,
+                       tokens_per_frame=F, window_back=kw.get("wb", 0), window_fwd=kw.get("wf", 0))
+    va.vattn_check()
+    check_guards(og, lg, what="o / lse")
+    ro, rl = oracle.attention(q, k, v, d ** -0.5, mode=mode, F=F, wb=kw.get("wb", 0), wf=kw.get("wf", 0))
+    assert_parity(from_dev(og.t), ro, "large logit jumps d=%d %s" % (d, mode))
+    # |lse| reaches ~1e3 here; fp32 holds it to ~1e-4 absolute
+    assert np.max(np.abs(lg.t.cpu().numpy().astype(np.float64) - rl)) < LSE_TOL, "lse"
+
+
 def test_bounded_wait_reports_timeout_and_context_survives(va):
     # A barrier nothing arrives on: the kernel's bounded wait gives up after
     # 50 ms, the status word reports a timeout, and the next call still works.

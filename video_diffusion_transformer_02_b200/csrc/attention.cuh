@@ -29,6 +29,8 @@
 // S = Q K^T is an SS MMA (both operands K-major, 128B swizzle);
 // O += P V is a TS MMA (P from TMEM, V MN-major in shared memory).
 #pragma once
+#include <type_traits>
+
 #include "common.cuh"
 
 namespace vattn {
@@ -45,6 +47,17 @@ constexpr uint32_t kTmemCols = 512;
 // units): stale maxima keep every exp2 argument below it, so fp32 stays
 // far from overflow while most tiles skip the O correction.
 constexpr float kRescaleThreshold = 8.0f;
+// Speculative exponentials in the two-tile kernel: an unmasked sub-tile
+// after a CTA's first is exponentiated against the current reference max,
+// and its own max is taken only when the row sum exceeds 2^threshold.  Used
+// at head dim 64, where the softmax alone sets the pace (measured +2 % on
+// B200), not at head dim 128, where the extra live registers cost more than
+// the row max they save (measured -2 %).
+template <int D>
+struct SpecExp {
+  static constexpr bool value = D == 64;
+};
+constexpr float kSpecSumBound = 256.0f;   // 2^kRescaleThreshold
 // Which of every 8 consecutive score pairs take the FMA-pipe polynomial
 // exp2 instead of MUFU ex2 (bit i set: pair i mod 8).  At head dim 128 the
 // MUFU keeps pace with the tensor core and the polynomial only adds issue

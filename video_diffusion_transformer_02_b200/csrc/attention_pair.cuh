@@ -626,46 +626,38 @@ __global__ void __launch_bounds__(kPairThreads, 1)
         tmem_ld32(tS + 32, s1);
         tmem_ld_wait_dep(s0);
         reg_tie32(s1);
-        // row max over the visible columns
-        float mx8[8];
+        // row max over all 64 columns of an unmasked sub-tile
+        auto row_max = [&]() {
+          float mx8[8];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) mx8[i] = -INFINITY;
-        if (!masked) {
+          for (int i = 0; i < 8; ++i) mx8[i] = -INFINITY;
 #pragma unroll
           for (int c = 0; c < 32; ++c)
             mx8[c & 7] = fmax3(mx8[c & 7], __uint_as_float(s0[c]), __uint_as_float(s1[c]));
-        } else {
+          return fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                       fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+        };
+        // P = exp2(s * scale * log2e + nm) of an unmasked sub-tile into the
+        // first half of the S buffer, 16 columns (32 keys) at a time; returns
+        // the row sum (packed fp32x2 partial sums).  CLAMP caps the
+        // polynomial's argument at 64, where its exponent insertion would
+        // otherwise wrap (MUFU ex2 saturates to inf by itself).
+        auto exps = [&](float nm, auto clamp) {
+          constexpr bool CLAMP = decltype(clamp)::value;
+          float rs2[2][2] = {{0.f, 0.f}, {0.f, 0.f}};
 #pragma unroll
-          for (int c = 0; c < 32; ++c) {
-            const float v0 = (c >= col_lo && c < col_hi) ? __uint_as_float(s0[c]) : -INFINITY;
-            const float v1 = (c + 32 >= col_lo && c + 32 < col_hi) ? __uint_as_float(s1[c]) : -INFINITY;
-            mx8[c & 7] = fmax3(mx8[c & 7], v0, v1);
-          }
-        }
-        const float mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
-                               fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
-        const float m_new = fmaxf(m_run, mx * sl2);
-        float factor = 1.f;
-        bool resc = false;
-        if (m_new > m_run + kRescaleThreshold) {
-          factor = ex2_approx(m_run - m_new);   // 0 when m_run = -inf
-          m_run = m_new;
-          resc = true;
-        }
-        const float nm = (m_run == -INFINITY) ? 0.f : -m_run;
-        // P = exp2(s * scale * log2e - m) into the first half of the S
-        // buffer, 16 columns (32 keys) at a time; row sums as packed fp32x2
-        float rs2[2][2] = {{0.f, 0.f}, {0.f, 0.f}};
-#pragma unroll
-        for (int q = 0; q < 2; ++q) {
-          const uint32_t* sq = q == 0 ? s0 : s1;
-          uint32_t pk[16];
-          if (!masked) {
+          for (int q = 0; q < 2; ++q) {
+            const uint32_t* sq = q == 0 ? s0 : s1;
+            uint32_t pk[16];
 #pragma unroll
             for (int c = 0; c < 32; c += 2) {
               float x0, x1, p0, p1;
               ffma2(x0, x1, __uint_as_float(sq[c]), __uint_as_float(sq[c + 1]), sl2, sl2, nm, nm);
               if ((PolyMask<D>::value >> ((c >> 1) & 7)) & 1u) {
+                if constexpr (CLAMP) {
+                  x0 = fminf(x0, 64.f);
+                  x1 = fminf(x1, 64.f);
+                }
                 ex2_poly2(p0, p1, x0, x1);
               } else {
                 p0 = ex2_approx(x0);
@@ -674,22 +666,108 @@ __global__ void __launch_bounds__(kPairThreads, 1)
               fadd2(rs2[(c >> 1) & 1][0], rs2[(c >> 1) & 1][1], p0, p1);
               pk[c / 2] = pack_bf16x2(p0, p1);
             }
-          } else {
-#pragma unroll
-            for (int c = 0; c < 32; c += 2) {
-              const int col = q * 32 + c;
-              float p0 = ex2_approx(fmaf(__uint_as_float(sq[c]), sl2, nm));
-              float p1 = ex2_approx(fmaf(__uint_as_float(sq[c + 1]), sl2, nm));
-              p0 = (col >= col_lo && col < col_hi) ? p0 : 0.f;
-              p1 = (col + 1 >= col_lo && col + 1 < col_hi) ? p1 : 0.f;
-              rs2[(c >> 1) & 1][0] += p0;
-              rs2[(c >> 1) & 1][1] += p1;
-              pk[c / 2] = pack_bf16x2(p0, p1);
+            tmem_st16(tS + q * 16, pk);
+          }
+          return (rs2[0][0] + rs2[0][1]) + (rs2[1][0] + rs2[1][1]);
+        };
+        float factor = 1.f;
+        bool resc = false;
+        float rs;
+        // Every tcgen05.st below (and each full-mask vote) is warp-collective,
+        // so both branches are taken by the whole warp: the speculative one
+        // only when no row of the warp is masked in this sub-tile (masks
+        // differ per row in the chunk-causal and sliding modes).
+        const bool spec = SpecExp<D>::value && u > 0 && !__any_sync(0xffffffffu, masked);
+        if (spec) {
+          // exponentials against the current reference max before this
+          // sub-tile's max is known.  The row sum bounds every term, so a sum
+          // of at most 2^threshold proves each exponent argument is at most
+          // the threshold, which is all the reference needs: the max is then
+          // never taken.  Otherwise take it, move the reference if it grew by
+          // more than the threshold, and redo the sub-tile.
+          rs = exps(m_run == -INFINITY ? 0.f : -m_run, std::true_type{});
+          // a row with no visible key before this sub-tile has no reference
+          // yet (its terms above were taken against 0): it sets one now;
+          // !(rs <= bound) also catches inf and NaN
+          const bool need = m_run == -INFINITY || !(rs <= kSpecSumBound);
+          if (__any_sync(0xffffffffu, need)) {
+            if (need) {   // per lane; no collective operation inside
+              const float m_new = fmaxf(m_run, row_max() * sl2);
+              if (m_new > m_run + kRescaleThreshold) {
+                factor = ex2_approx(m_run - m_new);   // 0 when m_run = -inf
+                m_run = m_new;
+                resc = true;
+              }
+            }
+            if (__any_sync(0xffffffffu, resc)) {
+              tmem_st_wait();   // the first stores land before they are replaced
+              rs = exps(m_run == -INFINITY ? 0.f : -m_run, std::false_type{});
             }
           }
-          tmem_st16(tS + q * 16, pk);
+        } else {
+          // row max over the visible columns (per lane; no collective inside)
+          float mx;
+          if (!masked) {
+            mx = row_max();
+          } else {
+            float mx8[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) mx8[i] = -INFINITY;
+#pragma unroll
+            for (int c = 0; c < 32; ++c) {
+              const float v0 = (c >= col_lo && c < col_hi) ? __uint_as_float(s0[c]) : -INFINITY;
+              const float v1 = (c + 32 >= col_lo && c + 32 < col_hi) ? __uint_as_float(s1[c]) : -INFINITY;
+              mx8[c & 7] = fmax3(mx8[c & 7], v0, v1);
+            }
+            mx = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                       fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+          }
+          const float m_new = fmaxf(m_run, mx * sl2);
+          if (m_new > m_run + kRescaleThreshold) {
+            factor = ex2_approx(m_run - m_new);   // 0 when m_run = -inf
+            m_run = m_new;
+            resc = true;
+          }
+          const float nm = (m_run == -INFINITY) ? 0.f : -m_run;
+          // P = exp2(s * scale * log2e - m) into the first half of the S
+          // buffer, 16 columns (32 keys) at a time; the per-lane branch only
+          // picks the values, the stores run converged after it
+          float rs2[2][2] = {{0.f, 0.f}, {0.f, 0.f}};
+#pragma unroll
+          for (int q = 0; q < 2; ++q) {
+            const uint32_t* sq = q == 0 ? s0 : s1;
+            uint32_t pk[16];
+            if (!masked) {
+#pragma unroll
+              for (int c = 0; c < 32; c += 2) {
+                float x0, x1, p0, p1;
+                ffma2(x0, x1, __uint_as_float(sq[c]), __uint_as_float(sq[c + 1]), sl2, sl2, nm, nm);
+                if ((PolyMask<D>::value >> ((c >> 1) & 7)) & 1u) {
+                  ex2_poly2(p0, p1, x0, x1);
+                } else {
+                  p0 = ex2_approx(x0);
+                  p1 = ex2_approx(x1);
+                }
+                fadd2(rs2[(c >> 1) & 1][0], rs2[(c >> 1) & 1][1], p0, p1);
+                pk[c / 2] = pack_bf16x2(p0, p1);
+              }
+            } else {
+#pragma unroll
+              for (int c = 0; c < 32; c += 2) {
+                const int col = q * 32 + c;
+                float p0 = ex2_approx(fmaf(__uint_as_float(sq[c]), sl2, nm));
+                float p1 = ex2_approx(fmaf(__uint_as_float(sq[c + 1]), sl2, nm));
+                p0 = (col >= col_lo && col < col_hi) ? p0 : 0.f;
+                p1 = (col + 1 >= col_lo && col + 1 < col_hi) ? p1 : 0.f;
+                rs2[(c >> 1) & 1][0] += p0;
+                rs2[(c >> 1) & 1][1] += p1;
+                pk[c / 2] = pack_bf16x2(p0, p1);
+              }
+            }
+            tmem_st16(tS + q * 16, pk);
+          }
+          rs = (rs2[0][0] + rs2[0][1]) + (rs2[1][0] + rs2[1][1]);
         }
-        const float rs = (rs2[0][0] + rs2[0][1]) + (rs2[1][0] + rs2[1][1]);
         // O_x rescale: wait until the P V of the previous sub-tile (which
         // accumulates into O_x) has completed; the next one waits for P below
         if (__any_sync(0xffffffffu, resc && u > 0)) {
