@@ -25,8 +25,9 @@
 // TMEM columns (512): S_X buffer b at [128 x + 64 b, +64) fp32 for tiles
 // x = A, B and b = 0, 1; O_A [256, 256+D), O_B [384, 384+D) fp32.  P (bf16
 // pairs, 32 columns) overwrites the first half of its S buffer once the
-// softmax holds the scores in registers; an issuer reuses a buffer for
-// sub-tile j+2 only after the P V of sub-tile j has completed.
+// softmax holds the scores in registers; an issuer issues the scores of
+// sub-tile j+2 into that buffer right after the P V of sub-tile j (one
+// thread's tcgen05.mma operations run in issue order).
 #pragma once
 #include "attention.cuh"
 #include "feature_map.cuh"
@@ -38,15 +39,22 @@ template <int D>
 struct PairCfg {
   static constexpr int kTileBytes = kTileM * D * 2;
   static constexpr int kBlocks = D / 64;
-  static constexpr int kStages = D == 128 ? 2 : 4;
+  // K and V stages of 128 keys.  K runs one stage deeper at head dim 128:
+  // a K stage is refilled only after the lagging tile's last Q K^T on it,
+  // and the refill's latency under load (about 3.6k cycles measured) is
+  // longer than the two sub-tile periods two stages leave; V is read one
+  // softmax later, which gives it that slack.
+  static constexpr int kStagesK = D == 128 ? 3 : 4;
+  static constexpr int kStagesV = D == 128 ? 2 : 4;
   static constexpr int kOffQ = 0;                          // Q_A, Q_B
   static constexpr int kOffK = 2 * kTileBytes;
-  static constexpr int kOffV = kOffK + kStages * kTileBytes;
-  static constexpr int kOffBar = kOffV + kStages * kTileBytes;
-  static constexpr int kNumBars = 4 + 4 * kStages + 12 + 2 + 5 + 3;
+  static constexpr int kOffV = kOffK + kStagesK * kTileBytes;
+  static constexpr int kOffBar = kOffV + kStagesV * kTileBytes;
+  static constexpr int kNumBars = 4 + 2 * kStagesK + 2 * kStagesV + 12 + 2 + 5 + 3;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
   static constexpr int kOffZ = kOffMisc + 64;        // hybrid: z_c, fp32 [D]
   static constexpr int kSmemBytes = kOffZ + D * 4;
+  static_assert(kSmemBytes <= 227 * 1024, "shared memory of one CTA");
 };
 
 constexpr int kPairThreads = 384;
@@ -267,7 +275,7 @@ __global__ void __launch_bounds__(kPairThreads, 1)
   static_assert(ROPE == kRopeNone || ROPE == kRopeQ, "keys are rotated before this kernel");
   static_assert(!HYB || (D == 128 && ROPE == kRopeNone), "hybrid: head dim 128, no RoPE");
   using C = PairCfg<D>;
-  constexpr int NS = C::kStages;
+  constexpr int NSK = C::kStagesK, NSV = C::kStagesV;
   constexpr int kSub = kTileN / 2;                 // keys per score sub-tile
   constexpr uint32_t kSubBytes = kSub * 128;       // sub-tile offset inside a 64-column block
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -322,10 +330,10 @@ __global__ void __launch_bounds__(kPairThreads, 1)
   auto bQFull = [&](int x) { return bar0 + 8 * x; };
   auto bQReady = [&](int x) { return bar0 + 16 + 8 * x; };
   auto bKFull = [&](int s) { return bar0 + 32 + 8 * s; };
-  auto bKEmpty = [&](int s) { return bar0 + 32 + 8 * (NS + s); };
-  auto bVFull = [&](int s) { return bar0 + 32 + 8 * (2 * NS + s); };
-  auto bVEmpty = [&](int s) { return bar0 + 32 + 8 * (3 * NS + s); };
-  const uint32_t bx = bar0 + 32 + 32 * NS;
+  auto bKEmpty = [&](int s) { return bar0 + 32 + 8 * (NSK + s); };
+  auto bVFull = [&](int s) { return bar0 + 32 + 8 * (2 * NSK + s); };
+  auto bVEmpty = [&](int s) { return bar0 + 32 + 8 * (2 * NSK + NSV + s); };
+  const uint32_t bx = bar0 + 32 + 16 * NSK + 16 * NSV;
   auto bSFull = [&](int x, int b) { return bx + 8 * (2 * x + b); };
   auto bPFull = [&](int x, int b) { return bx + 32 + 8 * (2 * x + b); };
   auto bPvDone = [&](int x) { return bx + 64 + 8 * x; };
@@ -367,9 +375,11 @@ __global__ void __launch_bounds__(kPairThreads, 1)
       }
     }
     // a stage is released once by the MMA issuer of each query tile
-    for (int s = 0; s < NS; ++s) {
+    for (int s = 0; s < NSK; ++s) {
       mbar_init(bKFull(s), 1);
       mbar_init(bKEmpty(s), hasB ? 2 : 1);
+    }
+    for (int s = 0; s < NSV; ++s) {
       mbar_init(bVFull(s), 1);
       mbar_init(bVEmpty(s), hasB ? 2 : 1);
     }
@@ -413,8 +423,8 @@ __global__ void __launch_bounds__(kPairThreads, 1)
       int j = 0;
       bool waited = p.wait_tile < 0 || !stepping;
       for (; j < nk; ++j) {
-        const int s = j % NS;
-        if (j >= NS && !mbar_wait(bKEmpty(s), ((j / NS) - 1) & 1, ab, kStatusTimeoutProducer)) break;
+        const int s = j % NSK;
+        if (j >= NSK && !mbar_wait(bKEmpty(s), ((j / NSK) - 1) & 1, ab, kStatusTimeoutProducer)) break;
         if (!waited && g.t0 + j >= p.wait_tile) {
           // this tile's keys are written by the step's append CTAs
           if (!wait_counter(p.step_sync, static_cast<uint32_t>(p.n_append), ab, kStatusTimeoutStep)) break;
@@ -430,8 +440,8 @@ __global__ void __launch_bounds__(kPairThreads, 1)
                       kt.kc3 + b);
       }
       // drain: every load issued so far has landed before the CTA exits
-      for (int i = max(0, j - NS); i < j; ++i) {
-        mbar_drain(bKFull(i % NS), (i / NS) & 1, ab.limit_ns);
+      for (int i = max(0, j - NSK); i < j; ++i) {
+        mbar_drain(bKFull(i % NSK), (i / NSK) & 1, ab.limit_ns);
       }
       for (int x = 0; x < (hasB ? 2 : 1); ++x) {
         mbar_drain(bQFull(x), 0, ab.limit_ns);
@@ -448,8 +458,8 @@ __global__ void __launch_bounds__(kPairThreads, 1)
       }
       int j = 0;
       for (; j < nk; ++j) {
-        const int s = j % NS;
-        if (j >= NS && !mbar_wait(bVEmpty(s), ((j / NS) - 1) & 1, ab, kStatusTimeoutProducer)) break;
+        const int s = j % NSV;
+        if (j >= NSV && !mbar_wait(bVEmpty(s), ((j / NSV) - 1) & 1, ab, kStatusTimeoutProducer)) break;
         const KeyTile kt = key_tile(p, g.tg, g.t0 + j);
         const CUtensorMap* m = kt.vmap ? &tmV2 : &tmV;
         mbar_arrive_expect_tx(bVFull(s), C::kTileBytes);
@@ -458,8 +468,8 @@ __global__ void __launch_bounds__(kPairThreads, 1)
           tma_load_4d(sV + s * C::kTileBytes + blk * (kTileM * 128), m, bVFull(s), blk * 64, kvh, kt.k0,
                       kt.vc3 + b);
       }
-      for (int i = max(0, j - NS); i < j; ++i) {
-        mbar_drain(bVFull(i % NS), (i / NS) & 1, ab.limit_ns);
+      for (int i = max(0, j - NSV); i < j; ++i) {
+        mbar_drain(bVFull(i % NSV), (i / NSV) & 1, ab.limit_ns);
       }
       if constexpr (HYB) mbar_drain(bZFull, 0, ab.limit_ns);
     }
@@ -478,13 +488,13 @@ __global__ void __launch_bounds__(kPairThreads, 1)
       const uint64_t dV = sdesc_sw128(sV, kTileM * 128, 1024);
       const uint32_t tSx = tmem + static_cast<uint32_t>(x * 128);
       const uint32_t tOx = tmem + 256u + static_cast<uint32_t>(x * 128);
-      // start-address step (>> 4) of sub-tile u: stage (u / 2) % NS, half u % 2
-      auto sub_step = [](int u) -> uint64_t {
-        return static_cast<uint64_t>(((u >> 1) & (NS - 1)) * (C::kTileBytes >> 4) + (u & 1) * (kSubBytes >> 4));
+      // start-address step (>> 4) of sub-tile u: stage (u / 2) % stages, half u % 2
+      auto sub_step = [](int u, int stages) -> uint64_t {
+        return static_cast<uint64_t>(((u >> 1) % stages) * (C::kTileBytes >> 4) + (u & 1) * (kSubBytes >> 4));
       };
       // S_x(u) = Q_x K(u)^T into S buffer u & 1
       auto issue_qk = [&](int u) {
-        const uint64_t dk = dK + sub_step(u);
+        const uint64_t dk = dK + sub_step(u, NSK);
         const uint32_t tS = tSx + static_cast<uint32_t>((u & 1) * kSub);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
@@ -495,7 +505,7 @@ __global__ void __launch_bounds__(kPairThreads, 1)
       };
       // O_x += P_x(u) V(u), P_x(u) in the first half of S buffer u & 1
       auto issue_pv = [&](int u) {
-        const uint64_t dv = dV + sub_step(u);
+        const uint64_t dv = dV + sub_step(u, NSV);
         const uint32_t tP = tSx + static_cast<uint32_t>((u & 1) * kSub);
         const uint32_t acc0 = u > 0 ? 1u : 0u;
 #pragma unroll
@@ -508,37 +518,34 @@ __global__ void __launch_bounds__(kPairThreads, 1)
       // softmax warpgroups do not start in lockstep (measured 2-3 % faster
       // than starting both together)
       if (x == 1 && ok && nk > 0) ok = mbar_wait(bPFull(0, 0), 0, ab, kStatusTimeoutMma);
-      if (ok && nk > 0) {
-        ok = mbar_wait(bKFull(0), 0, ab, kStatusTimeoutMma);
-        if (ok) {
-          tc_fence_after();
-          issue_qk(0);
-          if (HYB && ns == 1) umma_commit(bQKDone(x));
-        }
-      }
-      // per sub-tile u: S_x(u + 1) into the buffer that P_x(u - 1) V released,
-      // then O_x += P_x(u) V(u) once the softmax has published P_x(u); the
-      // tensor core computes the next scores while the softmax works
+      // S_x(j) once its K stage has landed (a stage is waited for at its
+      // first sub-tile only, and released once its second one is issued)
+      auto qk_step = [&](int j) -> bool {
+        const int stj = (j >> 1) % NSK;
+        if (!(j & 1) && !mbar_wait(bKFull(stj), ((j >> 1) / NSK) & 1, ab, kStatusTimeoutMma)) return false;
+        tc_fence_after();
+        issue_qk(j);
+        if (HYB && j == ns - 1) umma_commit(bQKDone(x));
+        if (j & 1) umma_commit(bKEmpty(stj));   // both sub-tiles of the stage issued
+        return true;
+      };
+      // both S buffers first (ns = 2 nk is even)
+      if (ok && nk > 0) ok = qk_step(0) && qk_step(1);
+      // per sub-tile u: O_x += P_x(u) V(u) once the softmax has published
+      // P_x(u), then at once S_x(u + 2) into the same buffer.  tcgen05.mma
+      // operations issued by one thread run in issue order, so the P V reads
+      // P before the next scores overwrite it; not waiting for the P V to
+      // complete keeps its latency off the softmax's path to S_x(u + 2).
       int u = 0;
       for (; ok && u < ns; ++u) {
-        const int un = u + 1;
-        if (un < ns) {
-          const int stn = (un >> 1) & (NS - 1);
-          // a stage is waited for at its first sub-tile only
-          if (!(un & 1) && !mbar_wait(bKFull(stn), ((un >> 1) / NS) & 1, ab, kStatusTimeoutMma)) break;
-          if (u > 0 && !mbar_wait(bPvDone(x), (u - 1) & 1, ab, kStatusTimeoutMma)) break;
-          tc_fence_after();
-          issue_qk(un);
-          if (HYB && un == ns - 1) umma_commit(bQKDone(x));
-          if (un & 1) umma_commit(bKEmpty(stn));   // both sub-tiles of the stage issued
-        }
-        const int st = (u >> 1) & (NS - 1);
-        if (!(u & 1) && !mbar_wait(bVFull(st), ((u >> 1) / NS) & 1, ab, kStatusTimeoutMma)) break;
+        const int st = (u >> 1) % NSV;
+        if (!(u & 1) && !mbar_wait(bVFull(st), ((u >> 1) / NSV) & 1, ab, kStatusTimeoutMma)) break;
         if (!mbar_wait(bPFull(x, u & 1), (u >> 1) & 1, ab, kStatusTimeoutMma)) break;
         tc_fence_after();
         issue_pv(u);
         if (u == ns - 1) umma_commit(bODone(x));
         if (u & 1) umma_commit(bVEmpty(st));
+        if (u + 2 < ns && !qk_step(u + 2)) break;
       }
       if constexpr (HYB) {
         // linear read-out phi(Q_x) S_c into the S buffers of tile x (free
@@ -807,29 +814,38 @@ __global__ void __launch_bounds__(kPairThreads, 1)
         const fmap::Poly aq = fmap::load_poly(p.hyb_coef, 0, p.H, h);
         const uint32_t qrow = sQ + static_cast<uint32_t>(x * C::kTileBytes);
         const uint32_t sz = sbase + C::kOffZ;
+        // one loop per feature map (the map is uniform over the launch); four
+        // partial sums keep the dot product's dependency chain short
+        auto phi_rows = [&](auto kind) {
+          constexpr int K = decltype(kind)::value;
+          float d4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll 1
-        for (int blk = 0; blk < D / 64; ++blk) {
+          for (int blk = 0; blk < D / 64; ++blk) {
 #pragma unroll
-          for (int c8 = 0; c8 < 8; ++c8) {
-            const uint32_t addr = qrow + blk * (kTileM * 128) + sw128_offset(r, c8);
-            const uint4 v = lds128(addr);
-            const uint4 z0 = lds128(sz + (blk * 64 + c8 * 8) * 4);
-            const uint4 z1 = lds128(sz + (blk * 64 + c8 * 8 + 4) * 4);
-            const uint32_t zz[8] = {z0.x, z0.y, z0.z, z0.w, z1.x, z1.y, z1.z, z1.w};
-            uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+            for (int c8 = 0; c8 < 8; ++c8) {
+              const uint32_t addr = qrow + blk * (kTileM * 128) + sw128_offset(r, c8);
+              const uint4 v = lds128(addr);
+              const uint4 z0 = lds128(sz + (blk * 64 + c8 * 8) * 4);
+              const uint4 z1 = lds128(sz + (blk * 64 + c8 * 8 + 4) * 4);
+              const uint32_t zz[8] = {z0.x, z0.y, z0.z, z0.w, z1.x, z1.y, z1.z, z1.w};
+              uint32_t w4[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              float x0 = bf16lo_to_f32(w4[e]), x1 = bf16hi_to_f32(w4[e]);
-              x0 = fmap::feature(p.hyb_fmap, aq, x0);
-              x1 = fmap::feature(p.hyb_fmap, aq, x1);
-              w4[e] = pack_bf16x2(x0, x1);
-              // the denominator takes the same bf16 values the read-out MMA multiplies
-              dl = fmaf(bf16lo_to_f32(w4[e]), __uint_as_float(zz[2 * e]), dl);
-              dl = fmaf(bf16hi_to_f32(w4[e]), __uint_as_float(zz[2 * e + 1]), dl);
+              for (int e = 0; e < 4; ++e) {
+                float x0 = bf16lo_to_f32(w4[e]), x1 = bf16hi_to_f32(w4[e]);
+                x0 = fmap::feature(K, aq, x0);
+                x1 = fmap::feature(K, aq, x1);
+                w4[e] = pack_bf16x2(x0, x1);
+                // the denominator takes the same bf16 values the read-out MMA multiplies
+                d4[e] = fmaf(bf16lo_to_f32(w4[e]), __uint_as_float(zz[2 * e]), d4[e]);
+                d4[e] = fmaf(bf16hi_to_f32(w4[e]), __uint_as_float(zz[2 * e + 1]), d4[e]);
+              }
+              sts128(addr, make_uint4(w4[0], w4[1], w4[2], w4[3]));
             }
-            sts128(addr, make_uint4(w4[0], w4[1], w4[2], w4[3]));
           }
-        }
+          return (d4[0] + d4[1]) + (d4[2] + d4[3]);
+        };
+        dl = p.hyb_fmap == fmap::kFmapPoly3 ? phi_rows(std::integral_constant<int, fmap::kFmapPoly3>{})
+                                            : phi_rows(std::integral_constant<int, fmap::kFmapElu1>{});
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) mbar_arrive(bPhiReady(x));

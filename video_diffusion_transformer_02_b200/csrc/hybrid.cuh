@@ -4,7 +4,8 @@
 // feature_map.cuh).
 //
 //   dS_c = sum_{j in range c} phi(k_j) v_j^T   (D x D, fp32)   -- tcgen05 MMA
-//   dz_c = sum_{j in range c} phi(k_j)          (D, fp32)       -- CUDA cores
+//   dz_c = sum_{j in range c} phi(k_j)          (D, fp32)       -- tcgen05 MMA
+//                                                  (phi(K)^T times a ones block)
 //   S_c  = S_in + sum_{c' < c} dS_c'  (exclusive scan over ranges), same for z
 //
 // Range c holds the tokens [c ct - ov, (c + 1) ct - ov) clipped to [0, L):
@@ -46,22 +47,26 @@ struct DeltaCfg {
   static constexpr int kStages = 3;
   static constexpr int kOffK = 0;
   static constexpr int kOffV = kStages * kTileBytes;
-  static constexpr int kOffBar = 2 * kStages * kTileBytes;
+  static constexpr int kOffOnes = 2 * kStages * kTileBytes;   // bf16 ones, one 64-column block of kRows rows
+  static constexpr int kOnesBytes = kRows * 128;
+  static constexpr int kOffBar = kOffOnes + kOnesBytes;
   static constexpr int kNumBars = 3 * kStages + 1;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
   static constexpr int kSmemBytes = kOffMisc + 64 + 1024;
+  static constexpr int kTmemCols = 256;                       // dS in [0, D), dz in [D, D + 16)
 };
 
 // grid (H, C, B), 384 threads: warp 0 TMA, warp 1 TMEM + MMA, warps 4..11
-// feature map, column sums and epilogue.  Feature-map thread t owns the
-// 16-byte chunk t % 16 (eight features) of rows t / 16 + 16 i of every tile,
-// so the column sums of its eight features stay in registers; the eight
+// feature map and epilogue.  Feature-map thread t owns the 16-byte chunk
+// t % 16 (eight features) of rows t / 16 + 16 i of every tile; the eight
 // warps release a stage with one arrive each, with no block-wide barrier
-// per tile, and the column sums are reduced across rows once at the end.
+// per tile.  The column sums dz come from the tensor core as well: per
+// stage, phi(K)^T times a block of ones (N = 16) accumulates them next to
+// dS in TMEM, from the same bf16 values the dS product multiplies.
 constexpr int kDeltaThreads = 384;
 constexpr int kPhiThreads = 256;
 
-template <int D>
+template <int D, int FMAP>
 __global__ void __launch_bounds__(kDeltaThreads, 2)
     delta_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                  const DeltaParams p) {
@@ -101,8 +106,14 @@ __global__ void __launch_bounds__(kDeltaThreads, 2)
     fence_barrier_init();
   }
   if (warp == 1) {
-    tmem_alloc(smem_addr(const_cast<uint32_t*>(tmem_slot)), 128);
+    tmem_alloc(smem_addr(const_cast<uint32_t*>(tmem_slot)), C::kTmemCols);
     tmem_relinquish();
+  }
+  if (warp >= 4) {
+    // the ones block (bf16 1.0 pairs), an operand of the async proxy
+    uint32_t* ones = reinterpret_cast<uint32_t*>(smem + C::kOffOnes);
+    for (int i = threadIdx.x - 128; i < C::kOnesBytes / 4; i += kPhiThreads) ones[i] = 0x3F803F80u;
+    fence_proxy_async_smem();
   }
   tc_fence_before();
   __syncthreads();
@@ -132,6 +143,8 @@ __global__ void __launch_bounds__(kDeltaThreads, 2)
       // D[a][e] += sum_tokens phiK[token][a] * V[token][e]: A = phiK^T and
       // B = V are both MN-major (tokens are the K dimension of the MMA).
       constexpr uint32_t id = idesc_bf16_f32(D, D, true, true);
+      constexpr uint32_t idz = idesc_bf16_f32(D, 16, true, true);
+      const uint32_t ob = sbase + C::kOffOnes;
       for (int t = 0; t < nt; ++t) {
         const int s = t % NS;
         if (!mbar_wait(bPhi(s), (t / NS) & 1, ab, kStatusTimeoutMma)) break;
@@ -141,6 +154,12 @@ __global__ void __launch_bounds__(kDeltaThreads, 2)
         for (int kk = 0; kk < kRows / 16; ++kk)
           umma_ss(tmem, sdesc_sw128(kb + kk * 2048, kRows * 128, 1024),
                   sdesc_sw128(vb + kk * 2048, kRows * 128, 1024), id, (t > 0 || kk > 0) ? 1u : 0u);
+        // dz: every column of the ones block is 1, so each of the 16 result
+        // columns is the column sum of phi(K) over the stage's rows
+#pragma unroll
+        for (int kk = 0; kk < kRows / 16; ++kk)
+          umma_ss(tmem + D, sdesc_sw128(kb + kk * 2048, kRows * 128, 1024),
+                  sdesc_sw128(ob + kk * 2048, kRows * 128, 1024), idz, (t > 0 || kk > 0) ? 1u : 0u);
         umma_commit(bEmpty(s));
       }
       umma_commit(bDone);
@@ -152,9 +171,6 @@ __global__ void __launch_bounds__(kDeltaThreads, 2)
     // address of this thread's chunk in row rg of a tile; row rg + 16 i adds
     // 16 i * 128 bytes and keeps the swizzle phase (16 i is a multiple of 8)
     const uint32_t off0 = (ch >> 3) * (kRows * 128) + sw128_offset(rg, ch & 7);
-    float zacc[8];
-#pragma unroll
-    for (int e = 0; e < 8; ++e) zacc[e] = 0.f;
     const fmap::Poly ak = fmap::load_poly(p.coef, 1, p.H, h);
     bool ok = true;
     // No early exit (a failed wait only follows an abort): every thread
@@ -174,12 +190,9 @@ __global__ void __launch_bounds__(kDeltaThreads, 2)
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           float x0 = bf16lo_to_f32(w4[e]), x1 = bf16hi_to_f32(w4[e]);
-          x0 = valid ? fmap::feature(p.fmap, ak, x0) : 0.f;
-          x1 = valid ? fmap::feature(p.fmap, ak, x1) : 0.f;
+          x0 = valid ? fmap::feature(FMAP, ak, x0) : 0.f;
+          x1 = valid ? fmap::feature(FMAP, ak, x1) : 0.f;
           w4[e] = pack_bf16x2(x0, x1);
-          // z sums the same bf16 values the MMA multiplies
-          zacc[2 * e] += bf16lo_to_f32(w4[e]);
-          zacc[2 * e + 1] += bf16hi_to_f32(w4[e]);
         }
         sts128(kb + i * (kRowGroups * 128), make_uint4(w4[0], w4[1], w4[2], w4[3]));
       }
@@ -190,18 +203,6 @@ __global__ void __launch_bounds__(kDeltaThreads, 2)
     if (ok && nt > 0) {
       ok = mbar_wait(bDone, 0, ab, kStatusTimeoutAux);
       tc_fence_after();
-    }
-    // reduce the column sums over the row groups (stage 0 of K is free now:
-    // every load has landed and every MMA has completed or the kernel aborts)
-    float* red = reinterpret_cast<float*>(smem + C::kOffK);
-#pragma unroll
-    for (int e = 0; e < 8; ++e) red[rg * D + ch * 8 + e] = zacc[e];
-    asm volatile("bar.sync 1, %0;" ::"n"(kPhiThreads) : "memory");
-    if (tid < D) {
-      float zs = 0.f;
-#pragma unroll
-      for (int g = 0; g < kRowGroups; ++g) zs += red[g * D + tid];
-      p.wsz[((static_cast<size_t>(c) * p.B + b) * p.H + h) * D + tid] = zs;
     }
     ok = __all_sync(0xffffffffu, ok);   // the TMEM loads below are warp-collective
     // S rows from TMEM: warp w reads lanes 32 (w % 4) ..; warps 4..7 take
@@ -226,13 +227,24 @@ __global__ void __launch_bounds__(kDeltaThreads, 2)
         d4[e] = make_float4(__uint_as_float(v[4 * e]), __uint_as_float(v[4 * e + 1]),
                             __uint_as_float(v[4 * e + 2]), __uint_as_float(v[4 * e + 3]));
     }
+    if (warp < 8) {
+      // dz[r] from TMEM lane r, column D (the 16 dz columns are equal)
+      uint32_t v[32];
+      if (ok && nt > 0) {
+        tmem_ld32(trow - cb + D, v);
+        tmem_ld_wait();
+      } else {
+        v[0] = 0u;
+      }
+      p.wsz[((static_cast<size_t>(c) * p.B + b) * p.H + h) * D + r] = __uint_as_float(v[0]);
+    }
   }
 
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, 128);
+    tmem_dealloc(tmem, C::kTmemCols);
   }
 }
 

@@ -1046,10 +1046,12 @@ vattn_status check_hybrid(int B, int L, int H, int d, int chunk_tokens, const vo
 vattn_status launch_delta(const CUtensorMap& mk, const CUtensorMap& mv, float* wsS, float* wsz, uint32_t* status,
                           int B, int L, int H, int C, int chunk_tokens, cudaStream_t stream, int overlap = 0,
                           int fmap = vattn::fmap::kFmapElu1, const float* coef = nullptr) {
-  static uint64_t done[1];
-  auto kern = vattn::hyb::delta_kernel<128>;
+  static uint64_t done[2][1];
+  const bool poly = fmap == vattn::fmap::kFmapPoly3;
+  auto kern = poly ? vattn::hyb::delta_kernel<128, vattn::fmap::kFmapPoly3>
+                   : vattn::hyb::delta_kernel<128, vattn::fmap::kFmapElu1>;
   const int smem = vattn::hyb::DeltaCfg<128>::kSmemBytes;
-  if (vattn_status st = ensure_smem(kern, smem, done)) return st;
+  if (vattn_status st = ensure_smem(kern, smem, done[poly ? 1 : 0])) return st;
   vattn::hyb::DeltaParams dp{wsS, wsz, status, B, L, H, chunk_tokens, overlap, fmap, coef};
   kern<<<dim3(H, C, B), vattn::hyb::kDeltaThreads, smem, stream>>>(mk, mv, dp);
   VATTN_CUDA(cudaGetLastError());
