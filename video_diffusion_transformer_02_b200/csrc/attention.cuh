@@ -49,13 +49,14 @@ constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleThreshold = 8.0f;
 // Speculative exponentials in the two-tile kernel: an unmasked sub-tile
 // after a CTA's first is exponentiated against the current reference max,
-// and its own max is taken only when the row sum exceeds 2^threshold.  Used
-// at head dim 64, where the softmax alone sets the pace (measured +2 % on
-// B200), not at head dim 128, where the extra live registers cost more than
-// the row max they save (measured -2 %).
-template <int D>
+// and its own max is taken only when the row sum exceeds 2^threshold.  On
+// for head dim 64 (+2.3 % measured on B200), for the instantiation that
+// rotates Q in the kernel (+2.0 % and +1.6 % on the 1.3B- and 14B-like
+// calls) and for the hybrid (+1.2 %); off for head dim 128 without RoPE,
+// where its extra live registers cost more than the row max saves (-0.9 %).
+template <int D, int ROPE, bool HYB>
 struct SpecExp {
-  static constexpr bool value = D == 64;
+  static constexpr bool value = D == 64 || ROPE != 0 || HYB;
 };
 constexpr float kSpecSumBound = 256.0f;   // 2^kRescaleThreshold
 // Which of every 8 consecutive score pairs take the FMA-pipe polynomial

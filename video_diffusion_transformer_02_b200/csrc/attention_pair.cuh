@@ -695,7 +695,7 @@ __global__ void __launch_bounds__(kPairThreads, 1)
         // so both branches are taken by the whole warp: the speculative one
         // only when no row of the warp is masked in this sub-tile (masks
         // differ per row in the chunk-causal and sliding modes).
-        const bool spec = SpecExp<D>::value && u > 0 && !__any_sync(0xffffffffu, masked);
+        const bool spec = SpecExp<D, ROPE, HYB>::value && u > 0 && !__any_sync(0xffffffffu, masked);
         if (spec) {
           // exponentials against the current reference max before this
           // sub-tile's max is known.  The row sum bounds every term, so a sum
