@@ -19,6 +19,7 @@
 #pragma once
 #include "common.cuh"
 #include "feature_map.cuh"
+#include "grid_dep.cuh"
 
 namespace vattn {
 namespace hyb {
@@ -71,6 +72,8 @@ __global__ void __launch_bounds__(kDeltaThreads, 2)
     delta_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                  const DeltaParams p) {
   static_assert(D == 128, "state delta supports head_dim 128");
+  pdl::grid_dep_wait();
+  pdl::grid_dep_launch();
   using C = DeltaCfg<D>;
   constexpr int NS = C::kStages;
   constexpr int kChunks = D / 8;                       // 16-byte chunks per row
@@ -257,6 +260,8 @@ constexpr int kScanBatch = 12;
 __global__ void __launch_bounds__(256, 2) scan_kernel(float4* __restrict__ wsS, float4* __restrict__ S, long long nS4,
                                                       float4* __restrict__ wsz, float4* __restrict__ z, long long nz4,
                                                       int C) {
+  pdl::grid_dep_wait();
+  pdl::grid_dep_launch();
   const long long total = nS4 + nz4;
   for (long long idx = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; idx < total;
        idx += static_cast<long long>(gridDim.x) * blockDim.x) {

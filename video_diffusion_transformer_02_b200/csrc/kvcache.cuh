@@ -4,6 +4,7 @@
 // 16-byte vectors, both tensors' loads in flight before the stores.
 #pragma once
 #include "common.cuh"
+#include "grid_dep.cuh"
 
 namespace vattn {
 namespace kv {
@@ -15,6 +16,8 @@ constexpr int kUnroll = 4;
 __global__ void __launch_bounds__(256) append_kernel(const uint4* __restrict__ k, const uint4* __restrict__ v,
                                                      uint4* __restrict__ kr, uint4* __restrict__ vr,
                                                      long long n16, int32_t* ids, int slot, int frame) {
+  pdl::grid_dep_wait();
+  pdl::grid_dep_launch();
   const long long stride = static_cast<long long>(gridDim.x) * blockDim.x;
   const long long tid = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
   for (long long base = tid; base < n16; base += stride * kUnroll) {

@@ -8,6 +8,7 @@
 // as in the Kaleido review; RoFormer frequencies).
 #pragma once
 #include "common.cuh"
+#include "grid_dep.cuh"
 
 namespace vattn {
 namespace rope {
@@ -62,6 +63,8 @@ struct RotParams {
 
 template <bool COPY>
 __global__ void __launch_bounds__(512) rotate_rows_kernel(const RotParams p) {
+  pdl::grid_dep_wait();
+  pdl::grid_dep_launch();
   const int cpt = p.heads * (p.d / 8);                 // chunks per row
   const long long rows_per_block = (p.rows + gridDim.x - 1) / gridDim.x;
   const long long r0 = static_cast<long long>(blockIdx.x) * rows_per_block;

@@ -59,6 +59,27 @@ int sm_count() {
 
 size_t round256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
+// Launch with programmatic stream serialisation (the memory-bound kernels):
+// the grid may be scheduled while the previous grid on the stream is still
+// running, and its first act is griddepcontrol.wait, so it reads and writes
+// nothing before that grid has completed; it then releases the next grid.
+// Back-to-back launches (a CUDA graph of appends, the hybrid's delta and
+// scan) thereby hide their launch gaps.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_after(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s, Args... args) {
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, args...);
+}
+
 // Tail split of a FULL attention call: with `items` (pair, head, batch)
 // work units on `sms` SMs (one two-tile CTA per SM), the last partial wave of
 // r items leaves sms - r SMs idle for a whole item; when r <= sms / 2 those
@@ -277,8 +298,7 @@ cudaError_t launch_rotate_rows(const vattn::rope::RotParams& p, cudaStream_t str
   long long blocks = (p.rows + rpb - 1) / rpb;
   if (blocks > p.rows) blocks = p.rows;
   if (blocks > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
-  vattn::rope::rotate_rows_kernel<COPY><<<static_cast<int>(blocks), threads, 0, stream>>>(p);
-  return cudaGetLastError();
+  return launch_after(vattn::rope::rotate_rows_kernel<COPY>, dim3(static_cast<unsigned>(blocks)), dim3(threads), 0, stream, p);
 }
 
 }  // namespace
@@ -649,9 +669,8 @@ vattn_status vattn_kvcache_append(vattn_kvcache* c, const void* k, const void* v
   const long long want = (n16 + 256LL * vattn::kv::kUnroll - 1) / (256LL * vattn::kv::kUnroll);
   const long long per_sm = (want + sms - 1) / sms;
   const int blocks = static_cast<int>(sms * (per_sm < 2 ? per_sm : 2));
-  vattn::kv::append_kernel<<<blocks, 256, 0, stream>>>(static_cast<const uint4*>(k), static_cast<const uint4*>(v),
-                                                       kr, vr, n16, c->frame_ids, slot, frame_idx);
-  VATTN_CUDA(cudaGetLastError());
+  VATTN_CUDA(launch_after(vattn::kv::append_kernel, dim3(blocks), dim3(256), 0, stream, static_cast<const uint4*>(k),
+                          static_cast<const uint4*>(v), kr, vr, n16, c->frame_ids, slot, frame_idx));
   c->host_ids[slot] = frame_idx;
   return VATTN_OK;
 }
@@ -1056,8 +1075,7 @@ vattn_status launch_delta(const CUtensorMap& mk, const CUtensorMap& mv, float* w
   const int smem = vattn::hyb::DeltaCfg<128>::kSmemBytes;
   if (vattn_status st = ensure_smem(kern, smem, done[poly ? 1 : 0])) return st;
   vattn::hyb::DeltaParams dp{wsS, wsz, status, B, L, H, chunk_tokens, overlap, fmap, coef};
-  kern<<<dim3(H, C, B), vattn::hyb::kDeltaThreads, smem, stream>>>(mk, mv, dp);
-  VATTN_CUDA(cudaGetLastError());
+  VATTN_CUDA(launch_after(kern, dim3(H, C, B), dim3(vattn::hyb::kDeltaThreads), smem, stream, mk, mv, dp));
   return VATTN_OK;
 }
 
@@ -1069,10 +1087,9 @@ vattn_status launch_scan(float* wsS, float* wsz, float* S, float* z, int B, int 
   if (current_device(&dev) == VATTN_OK) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const long long want = (nS4 + nz4 + 255) / 256;
   const int blocks = static_cast<int>(want < sms * 4LL ? want : sms * 4LL);
-  vattn::hyb::scan_kernel<<<blocks, 256, 0, stream>>>(reinterpret_cast<float4*>(wsS), reinterpret_cast<float4*>(S),
-                                                      nS4, reinterpret_cast<float4*>(wsz),
-                                                      reinterpret_cast<float4*>(z), nz4, C);
-  VATTN_CUDA(cudaGetLastError());
+  VATTN_CUDA(launch_after(vattn::hyb::scan_kernel, dim3(blocks), dim3(256), 0, stream, reinterpret_cast<float4*>(wsS),
+                          reinterpret_cast<float4*>(S), nS4, reinterpret_cast<float4*>(wsz),
+                          reinterpret_cast<float4*>(z), nz4, C));
   return VATTN_OK;
 }
 }  // namespace
