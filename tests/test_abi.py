@@ -94,6 +94,54 @@ def test_hybrid_workspace_and_checks(lib):
     assert hyb(FAKE, FAKE, FAKE, FAKE, FAKE, None, 1, 100, 2, 128, 50, 0.1, FAKE, 1 << 30, None) == 1
 
 
+def _tail_bytes(B, Lq, Lk, H, d, sms=148):
+    """The tail-split workspace layout as include/vattn.h documents it: r
+    arrival counters, then lse fp32 [r][s][256] and o fp32 [r][s][256][d],
+    each part from a 256-byte boundary; 0 when the split does not apply."""
+    up = lambda x: (x + 255) // 256 * 256
+    items = ((Lq + 127) // 128 + 1) // 2 * H * B
+    waves, r = divmod(items, sms)
+    kt = (Lk + 127) // 128
+    if waves < 1 or r == 0 or 2 * r > sms or kt < 2:
+        return 0
+    s = min(sms // r, 16, kt)
+    per = -(-kt // s)
+    s = -(-kt // per)
+    if s < 2:
+        return 0
+    off_o = up(r * 4) + up(r * s * 256 * 4)
+    return off_o + r * s * 256 * d * 4
+
+
+@pytest.mark.parametrize("shape", [
+    (1, 32760, 32760, 12, 12, 128),    # the 1.3B-like call: 10 waves + 56 pairs, 2 splits each
+    (1, 10240, 3001, 4, 4, 128),       # 160 pairs: 12 left over, 12 splits
+    (1, 12700, 12700, 3, 1, 64),       # GQA, 2 left over, 15 splits (16 would leave one empty)
+    (1, 75600, 75600, 40, 40, 128),    # the 14B-like call: exactly 80 waves, no split
+    (1, 2040, 2040, 16, 16, 64),       # one partial wave only: no split
+])
+@pytest.mark.parametrize("with_rope", [False, True])
+def test_attention_workspace_sizes(lib, shape, with_rope):
+    # Without a GPU the library sizes for 148 SMs (a B200).
+    class Rope(ctypes.Structure):
+        _fields_ = [("Hg", I), ("Wg", I), ("pt", I), ("ph", I), ("pw", I), ("max_pos", I),
+                    ("theta", ctypes.c_double)]
+    B, Lq, Lk, H, Hkv, d = shape
+    base = _sig(lib, "vattn_attention_workspace_bytes", ctypes.c_size_t, I, I, I, I, ctypes.POINTER(Rope))
+    ex = _sig(lib, "vattn_attention_workspace_bytes_ex", ctypes.c_size_t, I, I, I, I, I, I, I,
+              ctypes.POINTER(Rope))
+    rope = ctypes.byref(Rope(10, 10, d // 2 - 2 * (d // 6), d // 6, d // 6, 8192, 1e4)) if with_rope else None
+    rot = B * Lk * Hkv * d * 2 if with_rope else 0
+    assert base(B, Lk, Hkv, d, rope) == rot
+    tail = _tail_bytes(B, Lq, Lk, H, d)
+    want = ((rot + 255) // 256 * 256 + tail) if tail else rot
+    assert ex(B, Lq, Lk, H, Hkv, d, 0, rope) == want
+    for mode in (1, 2):   # masked modes never split the tail
+        assert ex(B, Lq, Lk, H, Hkv, d, mode, rope) == rot
+    if shape[:3] == (1, 32760, 32760) and with_rope:
+        assert want == 115433728   # the size the 1.3B-like benchmark allocates
+
+
 def test_kvcache_checks(lib):
     init = _sig(lib, "vattn_kvcache_init", I, ctypes.POINTER(P), P, P, P, I, I, I, I, I, P)
     h = P()
