@@ -788,7 +788,9 @@ __global__ void __launch_bounds__(kPairThreads, 1)
           rs = (rs2[0][0] + rs2[0][1]) + (rs2[1][0] + rs2[1][1]);
         }
         // O_x rescale: wait until the P V of the previous sub-tile (which
-        // accumulates into O_x) has completed; the next one waits for P below
+        // accumulates into O_x) has completed; the next one waits for P below.
+        // The single-phase parity wait is sound because S_x(u), issued after
+        // P_x(u - 2) V, has completed: bPvDone is at most one phase behind.
         if (__any_sync(0xffffffffu, resc && u > 0)) {
           if (pv_seen < u) {
             if (!mbar_wait(bPvDone(x), (u - 1) & 1, ab, kStatusTimeoutSoftmax)) ok = false;
