@@ -584,8 +584,10 @@ def stream_step_figure(va, torch, device, frames, c, pk, window_relative):
                                                      "window-relative" if window_relative else "absolute"))
 
 
-def cpu_baseline(w, rows=20480):
-    """The fp64 oracle, as it stands, on a bounded sample of the workload."""
+def cpu_baseline(w, rows=20480, configs=True):
+    """The fp64 oracle, as it stands, on a bounded sample of the workload;
+    with `configs`, also the oracle's own timings of the other configurations
+    (tiny and hybrid whole, the stream on sampled rows with a projection)."""
     import oracle
     rows_arr = si.sample_rows(0xBA5E, rows, w["B"], 2, w["L"])
     t0 = time.perf_counter()
@@ -593,10 +595,50 @@ def cpu_baseline(w, rows=20480):
                      rope=dict(Hg=w["Hg"], Wg=w["Wg"], pairs=w["pairs"], theta=w["theta"]), rows=rows_arr)
     dt = time.perf_counter() - t0
     flops = 4.0 * w["d"] * w["L"] * len(rows_arr)
-    return {"value": flops / dt / 1e12, "unit": "TFLOP/s", "cores": oracle.num_threads(), "kind": "oracle",
-            "seconds": dt,
-            "sample": "%d query rows (2 of 12 heads) of the wan13b workload, all 32760 keys each, "
-                      "fp64 with 3D-RoPE; TFLOP/s of mask-adjusted work" % len(rows_arr)}
+    out = {"value": flops / dt / 1e12, "unit": "TFLOP/s", "cores": oracle.num_threads(), "kind": "oracle",
+           "seconds": dt,
+           "sample": "%d query rows (2 of 12 heads) of the wan13b workload, all 32760 keys each, "
+                     "fp64 with 3D-RoPE; TFLOP/s of mask-adjusted work" % len(rows_arr)}
+    if configs:
+        out["configs"] = oracle_config_timings(w, len(rows_arr), dt)
+    return out
+
+
+def oracle_config_timings(w, wan_rows, wan_seconds, stream_rows=1024):
+    """Host timings of the fp64 oracle per configuration: tiny and hybrid in
+    full, the stream and the 1.3B-like workload on sampled query rows with
+    the full time projected from rows/s (labelled as a projection)."""
+    import oracle
+    res = {}
+    wan_rps = wan_rows / wan_seconds
+    res["wan13b"] = {"rows_sampled": wan_rows, "seconds": wan_seconds, "rows_per_s": wan_rps,
+                     "projected_full_s": w["L"] * w["H"] * w["B"] / wan_rps, "projected": True}
+    c = si.CONFIGS["tiny"]
+    q, k, v = si.qkv("tiny")
+    t0 = time.perf_counter()
+    oracle.attention(q, k, v, c["d"] ** -0.5, rope=dict(Hg=c["Hg"], Wg=c["Wg"], pairs=c["pairs"], theta=c["theta"]))
+    res["tiny"] = {"rows": int(q.shape[1] * q.shape[2]), "seconds": time.perf_counter() - t0, "projected": False}
+    c = si.CONFIGS["hybrid"]
+    q, k, v = si.qkv("hybrid")
+    ct = c["chunk_frames"] * c["Hg"] * c["Wg"]
+    t0 = time.perf_counter()
+    oracle.hybrid_recurrent(q, k, v, ct, c["d"] ** -0.5)
+    res["hybrid"] = {"rows": int(q.shape[1] * q.shape[2]), "seconds": time.perf_counter() - t0, "projected": False}
+    del q, k, v
+    c = si.CONFIGS["stream"]
+    F = c["Hg"] * c["Wg"]
+    q, k, v = si.qkv("stream")
+    L = q.shape[1]
+    srows = si.sample_rows(0x57A, stream_rows, 1, c["H"], L)
+    t0 = time.perf_counter()
+    oracle.stream(q, k, v, F, c["d"] ** -0.5, c["window_back"],
+                  rope=dict(Hg=c["Hg"], Wg=c["Wg"], pairs=c["pairs"], theta=c["theta"]), rows=srows)
+    dt = time.perf_counter() - t0
+    rps = len(srows) / dt
+    res["stream"] = {"rows_sampled": int(len(srows)), "seconds": dt, "rows_per_s": rps,
+                     "projected_full_s": L * c["H"] / rps, "projected": True}
+    del q, k, v
+    return res
 
 
 def workload_config(flops, world):
