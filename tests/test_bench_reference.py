@@ -30,3 +30,31 @@ def test_reference_arm_json_line():
     assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] >= 1
     assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["d2h_bytes_per_step"] == 0
     assert d["e2e"]["value"] == d["value"]
+
+
+def test_cpu_baseline_config_timings(monkeypatch):
+    # The oracle timings the bench adds to cpu_baseline, on shrunken copies of
+    # the configurations (same code path as the benchmark, a few seconds).
+    sys.path.insert(0, ROOT)
+    import importlib.util
+    import numpy as np
+    import seeded_inputs as si
+    spec = importlib.util.spec_from_file_location("bench_mod2", os.path.join(ROOT, "bench.py"))
+    bench = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(bench)
+    small = dict(si.CONFIGS)
+    small["hybrid"] = dict(si.CONFIGS["hybrid"], T=4, H=2)
+    small["stream"] = dict(si.CONFIGS["stream"], T=3, H=2)
+    monkeypatch.setattr(si, "CONFIGS", small)
+    monkeypatch.setattr(bench.si, "CONFIGS", small)
+    w = dict(B=1, H=12, L=32760)
+    res = bench.oracle_config_timings(w, wan_rows=100, wan_seconds=0.5, stream_rows=64)
+    assert set(res) == {"wan13b", "tiny", "hybrid", "stream"}
+    assert res["wan13b"]["projected"] and res["wan13b"]["projected_full_s"] == 32760 * 12 / 200.0
+    assert not res["tiny"]["projected"] and res["tiny"]["rows"] == 48 * 2
+    c = small["hybrid"]
+    assert not res["hybrid"]["projected"] and res["hybrid"]["rows"] == 4 * c["Hg"] * c["Wg"] * 2
+    st = res["stream"]
+    assert st["projected"] and 0 < st["rows_sampled"] <= 64
+    L = 3 * small["stream"]["Hg"] * small["stream"]["Wg"]
+    assert np.isclose(st["projected_full_s"], L * 2 / st["rows_per_s"])
